@@ -1,0 +1,326 @@
+"""Pins for the fp64 oracle: values that do not come from the oracle itself.
+
+Each pin is a checker function taking the oracle callable(s) it pins, so that the mutation
+tests at the bottom can plant a plausible mistake in a copy of the oracle (on the CPU) and
+show that some pin fails.
+
+Sources: 《DeepSeek-V2》深度解读报告 §2.1-§2.4 and §3.1; DeepSeek-V2论文解读 (xdnf.cn) §2.1;
+DeepSeek V2技术解析 (devpress) §1.  The RoPE anchors follow the original RoPE definition
+(theta_i = 10000^(-2i/d)), which the pages name but do not print.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+
+import mla_inputs as mi
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+SCALE = 1.0 / math.sqrt(mi.D_HEAD + mi.D_ROPE)
+
+
+# ------------------------------------------------------------------ brute-force helpers
+def bf_matvec_uk(w_uk, c):
+    """k^C[h][j] = sum_k W_UK[h][j][k] c[k], by scalar loops."""
+    H, dh, dc = w_uk.shape
+    return [[sum(float(w_uk[h, j, k]) * float(c[k]) for k in range(dc)) for j in range(dh)]
+            for h in range(H)]
+
+
+def bf_matvec_uv(w_uv, c):
+    """v^C[h][j] = sum_k W_UV[h][k][j] c[k], by scalar loops."""
+    H, dc, dh = w_uv.shape
+    return [[sum(float(w_uv[h, k, j]) * float(c[k]) for k in range(dc)) for j in range(dh)]
+            for h in range(H)]
+
+
+def bf_attention(q_nope, q_pe, c, kr_rot, w_uk, w_uv, scale):
+    """Scalar-loop MLA attention for tiny shapes (no numpy arithmetic)."""
+    H, dh = q_nope.shape
+    L = c.shape[0]
+    kC = [bf_matvec_uk(w_uk, c[t]) for t in range(L)]
+    vC = [bf_matvec_uv(w_uv, c[t]) for t in range(L)]
+    out, out_lat, lse = [], [], []
+    for h in range(H):
+        s = []
+        for t in range(L):
+            acc = 0.0
+            for j in range(dh):
+                acc += float(q_nope[h, j]) * kC[t][h][j]
+            for j in range(q_pe.shape[1]):
+                acc += float(q_pe[h, j]) * float(kr_rot[t, j])
+            s.append(acc * scale)
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        z = sum(e)
+        p = [x / z for x in e]
+        out.append([sum(p[t] * vC[t][h][j] for t in range(L)) for j in range(dh)])
+        out_lat.append([sum(p[t] * float(c[t, k]) for t in range(L)) for k in range(c.shape[1])])
+        lse.append(m + math.log(z))
+    return np.array(out), np.array(out_lat), np.array(lse)
+
+
+def tiny_case(seed, L, H=2, dh=3, dc=4, dr=2):
+    rng = np.random.default_rng(seed)
+    return dict(q_nope=rng.standard_normal((H, dh)), q_pe=rng.standard_normal((H, dr)),
+                c=rng.standard_normal((L, dc)), kr_rot=rng.standard_normal((L, dr)),
+                w_uk=rng.standard_normal((H, dh, dc)) * 0.5, w_uv=rng.standard_normal((H, dc, dh)) * 0.5)
+
+
+# ------------------------------------------------------------------ pin checkers
+def check_rope_anchors(apply_rope):
+    """Closed-form anchors: theta_0 = 1, theta_8 = 0.1, theta_16 = 0.01, theta_24 = 0.001 (d=64)."""
+    for i, pos in ((0, 1), (8, 10), (16, 100), (24, 1000), (0, 7), (16, 300)):
+        for odd in (0, 1):
+            x = np.zeros(64)
+            x[2 * i + odd] = 1.0
+            y = apply_rope(x, pos)
+            a = float(pos) * (10.0 ** (-4.0 * (2 * i) / 64.0))   # 10000^(-2i/64)
+            z = np.exp(1j * a) * (1.0 if odd == 0 else 1j)          # (x_e + i x_o) e^{i a}
+            expect = np.zeros(64)
+            expect[2 * i], expect[2 * i + 1] = z.real, z.imag
+            assert np.allclose(y, expect, rtol=0, atol=1e-12), (i, pos, odd)
+
+
+def check_rope_invariants(apply_rope):
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((5, 64))
+    assert np.array_equal(apply_rope(x, 0), x)                           # identity at t = 0
+    for pos in (1, 37, 4095, 131071):
+        y = apply_rope(x, pos)
+        assert np.allclose((y[:, 0::2] ** 2 + y[:, 1::2] ** 2), (x[:, 0::2] ** 2 + x[:, 1::2] ** 2),
+                           rtol=1e-12, atol=1e-12)                         # each pair keeps its norm
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    for m, n in ((5, 2), (100, 97), (3000, 10)):
+        lhs = apply_rope(q, m) @ apply_rope(k, n)
+        rhs = apply_rope(q, m - n) @ k
+        assert abs(lhs - rhs) < 1e-9 * (1 + abs(lhs))                     # depends only on m - n
+
+
+def check_attention_bruteforce(attend):
+    for seed, L in ((1, 1), (2, 2), (3, 5), (4, 4)):
+        t = tiny_case(seed, L)
+        out, lat, lse = bf_attention(t["q_nope"], t["q_pe"], t["c"], t["kr_rot"], t["w_uk"], t["w_uv"], 0.37)
+        r = attend(t["q_nope"], t["q_pe"], t["c"], t["kr_rot"], t["w_uk"], t["w_uv"], 0.37)
+        assert np.allclose(r["out"], out, rtol=1e-12, atol=1e-12)
+        assert np.allclose(r["out_lat"], lat, rtol=1e-12, atol=1e-12)
+        assert np.allclose(r["lse"], lse, rtol=1e-12, atol=1e-12)
+
+
+def check_special_cases(attend):
+    # L = 1: all weight on the single token, out = v^C of that token, out_lat = c, lse = s.
+    t = tiny_case(11, 1)
+    r = attend(t["q_nope"], t["q_pe"], t["c"], t["kr_rot"], t["w_uk"], t["w_uv"], 0.5)
+    vC = np.array(bf_matvec_uv(t["w_uv"], t["c"][0]))
+    assert np.allclose(r["out"], vC, rtol=0, atol=1e-13)
+    assert np.allclose(r["out_lat"], np.broadcast_to(t["c"][0], r["out_lat"].shape), rtol=0, atol=1e-13)
+    # zero query: uniform weights, out_lat = mean of the rows, lse = log L.
+    t = tiny_case(12, 5)
+    r = attend(np.zeros_like(t["q_nope"]), np.zeros_like(t["q_pe"]), t["c"], t["kr_rot"], t["w_uk"], t["w_uv"], 0.5)
+    assert np.allclose(r["out_lat"], np.broadcast_to(t["c"].mean(axis=0), r["out_lat"].shape), atol=1e-13)
+    assert np.allclose(r["lse"], math.log(5), atol=1e-13)
+    # L = 2: the weight of token 0 is the logistic sigmoid of s_0 - s_1.
+    t = tiny_case(13, 2)
+    r = attend(t["q_nope"], t["q_pe"], t["c"], t["kr_rot"], t["w_uk"], t["w_uv"], 0.5)
+    kC = [bf_matvec_uk(t["w_uk"], t["c"][i]) for i in range(2)]
+    for h in range(2):
+        s = [0.5 * (sum(t["q_nope"][h, j] * kC[i][h][j] for j in range(3)) +
+                    sum(t["q_pe"][h, j] * t["kr_rot"][i, j] for j in range(2))) for i in range(2)]
+        p0 = scipy.special.expit(s[0] - s[1])
+        assert np.allclose(r["out_lat"][h], p0 * t["c"][0] + (1 - p0) * t["c"][1], atol=1e-13)
+
+
+def check_absorb_unabsorb(absorb_q, unabsorb_v):
+    rng = np.random.default_rng(21)
+    w_uk = rng.standard_normal((2, 3, 4))
+    w_uv = rng.standard_normal((2, 4, 3))
+    qn = rng.standard_normal((2, 3))
+    lat = rng.standard_normal((2, 4))
+    qa = absorb_q(qn, w_uk)
+    ov = unabsorb_v(lat, w_uv)
+    for h in range(2):
+        for k in range(4):
+            assert abs(qa[h, k] - sum(qn[h, j] * w_uk[h, j, k] for j in range(3))) < 1e-13
+        for j in range(3):
+            assert abs(ov[h, j] - sum(lat[h, k] * w_uv[h, k, j] for k in range(4))) < 1e-13
+
+
+# ------------------------------------------------------------------ the pins
+def test_cache_size_against_pages():
+    g = json.load(open(os.path.join(GOLDEN, "mla_sizes.json")))
+    assert (mi.N_HEADS, mi.D_HEAD, mi.D_LATENT, mi.D_ROPE) == (g["n_heads"], g["d_head"], g["d_latent"], g["d_rope"])
+    assert oracle.mla_cache_elems_per_token(mi.D_LATENT, mi.D_ROPE) == g["mla_elems_per_token_per_layer"] == mi.D_ROW
+    assert oracle.mla_cache_elems_per_token(mi.D_LATENT, mi.D_ROPE, g["n_layers"]) == g["mla_elems_per_token_60_layers"]
+    mha = oracle.mha_cache_elems_per_token(mi.N_HEADS, mi.D_HEAD)
+    assert mha == 32768
+    # the page's printed MHA product is an arithmetic slip (formula gives 1,966,080)
+    assert oracle.mha_cache_elems_per_token(mi.N_HEADS, mi.D_HEAD, g["n_layers"]) == 1966080 != g["mha_figure_printed_on_page"]
+    # GQA equivalence: 576 cached elements = 2.25 groups of (K, V) of width d_h
+    assert oracle.mla_cache_elems_per_token(mi.D_LATENT, mi.D_ROPE) / (2 * mi.D_HEAD) == g["gqa_equivalent_groups"]
+    assert mi.D_LATENT == 4 * mi.D_HEAD and mi.D_ROPE == mi.D_HEAD // 2
+
+
+def test_rope_anchors():
+    check_rope_anchors(oracle.apply_rope)
+
+
+def test_rope_invariants():
+    check_rope_invariants(oracle.apply_rope)
+
+
+def test_rope_inv_freq_anchors():
+    th = oracle.rope_inv_freq(64)
+    assert th.shape == (32,)
+    assert th[0] == 1.0 and abs(th[16] - 0.01) < 1e-16 and abs(th[8] - 0.1) < 1e-16
+
+
+def test_softmax_against_scipy():
+    rng = np.random.default_rng(3)
+    for s in (rng.standard_normal((4, 9)) * 3, np.array([[1000.0, 999.0, -1000.0]]), np.zeros((2, 6))):
+        p, lse = oracle.softmax_stats(s)
+        assert np.allclose(p, scipy.special.softmax(s, axis=-1), rtol=1e-14, atol=1e-300)
+        assert np.allclose(lse, scipy.special.logsumexp(s, axis=-1), rtol=1e-14)
+
+
+@pytest.mark.parametrize("form", ["explicit", "absorbed"])
+def test_bruteforce_tiny(form):
+    check_attention_bruteforce(oracle.attend_explicit if form == "explicit" else oracle.attend_absorbed)
+
+
+@pytest.mark.parametrize("form", ["explicit", "absorbed"])
+def test_special_cases(form):
+    check_special_cases(oracle.attend_explicit if form == "explicit" else oracle.attend_absorbed)
+
+
+def test_absorb_unabsorb_bruteforce():
+    check_absorb_unabsorb(oracle.absorb_q, oracle.unabsorb_v)
+
+
+def test_absorbed_equals_explicit_full_dims():
+    """Associativity ([DR] §2.3): the absorbed and explicit forms agree to 1e-10 in fp64."""
+    w = mi.layer_weights(5)
+    b = mi.decode_batch(6, [97])
+    f = mi.bf16_to_f64
+    L = 97
+    kr = oracle.apply_rope(f(b.kr[0]), np.arange(L))
+    args = (f(b.q_nope[0]), f(b.q_pe[0]), f(b.c[0]), kr, f(w.w_uk), f(w.w_uv), SCALE)
+    e = oracle.attend_explicit(*args)
+    a = oracle.attend_absorbed(*args)
+    for k in ("out", "out_lat", "lse"):
+        rel = np.abs(e[k] - a[k]).max() / np.abs(e[k]).max()
+        assert rel <= 1e-10, (k, rel)
+
+
+def test_token_permutation_invariance():
+    t = tiny_case(31, 7, H=3, dh=4, dc=6, dr=2)
+    r0 = oracle.attend_explicit(**{k: t[k] for k in ("q_nope", "q_pe", "c", "kr_rot", "w_uk", "w_uv")}, scale=0.4)
+    perm = np.random.default_rng(1).permutation(7)
+    r1 = oracle.attend_explicit(t["q_nope"], t["q_pe"], t["c"][perm], t["kr_rot"][perm], t["w_uk"], t["w_uv"], 0.4)
+    for k in ("out", "out_lat", "lse"):
+        assert np.allclose(r0[k], r1[k], rtol=1e-13, atol=1e-13)
+
+
+def test_split_merge_identity():
+    rng = np.random.default_rng(9)
+    qf = rng.standard_normal((4, 10))
+    rows = rng.standard_normal((37, 10))
+    full = oracle.attend_rows(qf, rows, 0.8, 8)
+    for cuts in ([0, 37], [0, 16, 37], [0, 1, 2, 30, 37], [0, 12, 24, 36, 37]):
+        parts = [oracle.partial_rows(qf, rows[a:b], 0.8, 8) for a, b in zip(cuts[:-1], cuts[1:])]
+        lat, lse = oracle.merge_partials(parts)
+        assert np.allclose(lat, full["out_lat"], rtol=1e-13, atol=1e-13)
+        assert np.allclose(lse, full["lse"], rtol=1e-13, atol=1e-13)
+
+
+def test_score_scale_sanity():
+    """With the workload distributions the scaled score has std ~1: q_abs.c has variance ~128,
+    q_pe.k_R has variance 64, total 192, times 1/192."""
+    w = mi.layer_weights(41)
+    b = mi.decode_batch(42, [512])
+    f = mi.bf16_to_f64
+    qa = oracle.absorb_q(f(b.q_nope[0]), f(w.w_uk))
+    rows = oracle.cache_rows(f(b.c[0]), f(b.kr[0]), np.arange(512))
+    s = oracle.attend_rows(oracle.q_full(qa, f(b.q_pe[0])), rows, SCALE, mi.D_LATENT)["s"]
+    assert 0.9 < s.std() < 1.1, s.std()
+
+
+def test_decode_step_forms_agree():
+    w = mi.layer_weights(51)
+    b = mi.decode_batch(52, [1, 65, 130])
+    f = mi.bf16_to_f64
+    args = (f(b.q_nope), f(b.q_pe), [f(x) for x in b.c], [f(x) for x in b.kr], f(w.w_uk), f(w.w_uv), SCALE)
+    e = oracle.decode_step(*args, form="explicit", q_pos=[0, 64, 129])
+    a = oracle.decode_step(*args, form="absorbed", q_pos=[0, 64, 129])
+    for k in ("out", "out_lat", "lse", "q_abs"):
+        assert np.allclose(e[k], a[k], rtol=1e-10, atol=1e-12)
+
+
+def test_bf16_rounding_ties_even():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 65504.0, 1e-40])
+    b = mi.f64_to_bf16(x)
+    # 1+2^-8 is halfway between 1 and 1+2^-7: ties go to the even mantissa (1.0);
+    # 1+3*2^-8 is halfway between 1+2^-7 and 1+2^-6... ties to even -> 1+2^-6
+    assert list(mi.bf16_to_f64(b)[:4]) == [1.0, 1.0, 1.0 + 2 ** -6, -2.5]
+
+
+# ------------------------------------------------------------------ planted mistakes
+def _fails(fn, *a):
+    try:
+        fn(*a)
+    except AssertionError:
+        return True
+    return False
+
+
+def test_pins_catch_planted_rope_mistakes():
+    def sign_flip(x, pos, base=oracle.ROPE_BASE):
+        return oracle.apply_rope(x, -np.asarray(pos), base)
+
+    def half_split(x, pos, base=oracle.ROPE_BASE):
+        x = np.asarray(x, np.float64)
+        d = x.shape[-1]
+        ang = np.asarray(pos, np.float64)[..., None] * oracle.rope_inv_freq(d, base)
+        a, b = x[..., : d // 2], x[..., d // 2:]
+        return np.concatenate([a * np.cos(ang) - b * np.sin(ang), a * np.sin(ang) + b * np.cos(ang)], -1)
+
+    def wrong_exponent(x, pos, base=oracle.ROPE_BASE):
+        x = np.asarray(x, np.float64)
+        d = x.shape[-1]
+        th = np.power(base, -np.arange(d // 2) / d)
+        ang = np.asarray(pos, np.float64)[..., None] * th
+        y = np.empty_like(x)
+        y[..., 0::2] = x[..., 0::2] * np.cos(ang) - x[..., 1::2] * np.sin(ang)
+        y[..., 1::2] = x[..., 0::2] * np.sin(ang) + x[..., 1::2] * np.cos(ang)
+        return y
+
+    for bad in (sign_flip, half_split, wrong_exponent):
+        assert _fails(check_rope_anchors, bad) or _fails(check_rope_invariants, bad), bad.__name__
+
+
+def test_pins_catch_planted_attention_mistakes():
+    def drop_rope_channel(q_nope, q_pe, c, kr, w_uk, w_uv, scale):
+        return oracle.attend_explicit(q_nope, np.zeros_like(q_pe), c, kr, w_uk, w_uv, scale)
+
+    def reversed_uv_index(q_nope, q_pe, c, kr, w_uk, w_uv, scale):
+        r = oracle.attend_explicit(q_nope, q_pe, c, kr, w_uk, w_uv, scale)
+        r["out"] = np.einsum("hk,hkj->hj", r["out_lat"], np.asarray(w_uv)[:, ::-1, :])
+        return r
+
+    def no_max_shift_but_wrong_norm(q_nope, q_pe, c, kr, w_uk, w_uv, scale):
+        r = oracle.attend_explicit(q_nope, q_pe, c, kr, w_uk, w_uv, scale)
+        r["lse"] = r["lse"] - 1e-3
+        return r
+
+    for bad in (drop_rope_channel, reversed_uv_index, no_max_shift_but_wrong_norm):
+        assert _fails(check_attention_bruteforce, bad), bad.__name__
+
+
+def test_pins_catch_planted_absorb_mistakes():
+    def uk_wrong_index(qn, w_uk):
+        return np.einsum("hj,hjk->hk", qn, w_uk[::-1])          # heads swapped
+
+    assert _fails(check_absorb_unabsorb, uk_wrong_index, oracle.unabsorb_v)
