@@ -1,0 +1,365 @@
+"""Benchmark of one MLA decode step (append -> absorb -> decode attention -> un-absorb).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input: append the batch's
+new token (RoPE on k^R) into the latent cache, absorb W_UK into the queries, split-KV decode
+attention over the cache, apply W_UV.  `value` is latent-cache HBM GB/s for the whole job
+(bytes of cached rows the step must stream, summed over ranks, divided by the max-over-ranks
+device time).  Inputs are resident in HBM before the timed region; the caches are rotated
+between steps (several copies, together larger than the 126 MB L2) so no step reads a cache
+the previous step left in L2.  N > 1 runs independent replicas (weak scaling): the decode of
+disjoint batches needs no data exchange.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import mla_inputs as mi  # noqa: E402
+
+METRIC = "MLA decode step: latent-cache HBM GB/s, TFLOP/s, % roofline; tokens/s"
+UNIT = "GB/s"
+ROW_BYTES = 576 * 2
+FLOP_PER_TOKEN = 2 * 128 * 576 + 2 * 128 * 512          # QK^T over [c|k_R] plus P.V over c
+GEMM_FLOP_PER_SEQ = 2 * (2 * 128 * 128 * 512)           # absorb + un-absorb
+L2_BYTES = 126 * 1024 * 1024
+DEFAULT_WORKLOAD = "b32_l4096"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def workload_shape(name):
+    w = mi.WORKLOADS[name]
+    lens = mi.workload_lengths(name)
+    return w, lens
+
+
+def step_work(lens):
+    """Algorithmic bytes and flops of one step (per replica)."""
+    tokens = int(np.sum(lens))
+    B = len(lens)
+    cache_bytes = tokens * ROW_BYTES
+    flops = tokens * FLOP_PER_TOKEN + B * GEMM_FLOP_PER_SEQ
+    # decode kernel's own algorithmic bytes: cache rows + q_full in + out_lat out
+    decode_bytes = cache_bytes + B * 128 * 576 * 2 + B * 128 * 512 * 2
+    return tokens, cache_bytes, flops, decode_bytes
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------- oracle
+def time_oracle(lens, budget_tokens=1024, seed=4242):
+    """The fp64 oracle (explicit form, as it stands) on a bounded sample of the workload:
+    one sequence of the workload's first length, truncated to `budget_tokens` tokens."""
+    import oracle
+    L = int(min(int(lens[0]), budget_tokens))
+    b = mi.decode_batch(seed, [L])
+    w = mi.layer_weights(seed + 1)
+    f = mi.bf16_to_f64
+    args = (f(b.q_nope), f(b.q_pe), [f(x) for x in b.c], [f(x) for x in b.kr], f(w.w_uk), f(w.w_uv),
+            1.0 / math.sqrt(192.0))
+    t0 = time.perf_counter()
+    oracle.decode_step(*args, form="explicit")
+    dt = time.perf_counter() - t0
+    return L, dt
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        n = 1
+    return max(n, 1), len(os.sched_getaffinity(0))
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w, lens = workload_shape(args.workload)
+    for _ in range(args.warmup):
+        time_oracle(lens, budget_tokens=256)
+    tok, secs = 0, 0.0
+    for _ in range(args.steps):
+        L, dt = time_oracle(lens, budget_tokens=1024)
+        tok += L
+        secs += dt
+    gbs = tok * ROW_BYTES / secs / 1e9
+    threads, cores = cpu_threads()
+    sample = f"{args.steps} steps x one sequence of {L} tokens (explicit fp64 form), extrapolated per cached token"
+    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload, "batch": len(lens),
+                                            "seq_len": int(np.max(lens)), "paged": bool(w["paged"])},
+            "cpu_baseline": {"value": gbs, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+                             "affinity_cores": cores},
+            "e2e": {"value": gbs, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------- ours
+def setup_replica(name, device):
+    import torch
+    from mla_latent_kv_20_b200 import harness as hz
+    w, lens = workload_shape(name)
+    seed = w["seed"]
+    B = len(lens)
+    batch = mi.decode_batch(seed, lens)
+    wts = mi.layer_weights(seed + 1)
+    table, nblk = mi.block_permutation(seed + 2, lens) if w["paged"] else (None, 0)
+    base = hz.Cache(lens, w["paged"], table, nblk, device=device, fill_value=None)
+    base.fill(batch.c, batch.kr)
+    _, cache_bytes, _, _ = step_work(lens)
+    n_copies = max(2, math.ceil(3 * L2_BYTES / max(cache_bytes, 1)))
+    caches = [base]
+    for _ in range(n_copies - 1):
+        c = hz.Cache.__new__(hz.Cache)
+        c.__dict__.update(base.__dict__)
+        c.data = base.data.clone()
+        caches.append(c)
+    last = np.asarray(lens, np.int32) - 1
+    new_c = np.stack([batch.c[i][last[i]] for i in range(B)])
+    new_kr = np.stack([batch.kr[i][last[i]] for i in range(B)])
+    st = dict(
+        B=B, lens=lens, w=w, caches=caches,
+        q_nope=hz.bf16_tensor(batch.q_nope, device), q_pe=hz.bf16_tensor(batch.q_pe, device),
+        c_new=hz.bf16_tensor(new_c, device), kr_new=hz.bf16_tensor(new_kr, device),
+        pos=torch.from_numpy(last).to(device), seq_ids=torch.arange(B, dtype=torch.int32, device=device),
+        w_uk=hz.bf16_tensor(wts.w_uk, device), w_uv=hz.bf16_tensor(wts.w_uv, device),
+        q_full=torch.empty((B, 128, 576), dtype=torch.bfloat16, device=device),
+        out_lat=torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device),
+        lse=torch.empty((B, 128), dtype=torch.float32, device=device),
+        out=torch.empty((B, 128, 128), dtype=torch.bfloat16, device=device),
+        splits=int(w.get("splits", 0)),
+        host=dict(q_nope=batch.q_nope, q_pe=batch.q_pe, c_new=new_c, kr_new=new_kr, pos=last),
+    )
+    import mla_latent_kv_20_b200 as m
+    ws_bytes = m.decode_workspace_size(B, base.capacity(), st["splits"])
+    st["workspace"] = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=device)
+    st["n_splits"] = m.decode_num_splits(B, base.capacity(), st["splits"])
+    return st
+
+
+LAUNCHES_PER_STEP = 6   # append, absorb GEMM, q_pe rotation, decode split, combine, un-absorb GEMM
+
+
+def run_step(st, i, ev=None):
+    import mla_latent_kv_20_b200 as m
+    cache = st["caches"][i % len(st["caches"])]
+    m.cache_append(st["c_new"], st["kr_new"], st["pos"], cache.data, cache.desc, seq_ids=st["seq_ids"],
+                   block_table=cache.block_table)
+    m.absorb_q(st["q_nope"], st["q_pe"], st["w_uk"], st["q_full"], q_pos=st["pos"])
+    if ev is not None:
+        ev[0].record()
+    m.decode_attn(st["q_full"], cache.data, cache.seq_lens, cache.desc, st["workspace"], st["out_lat"],
+                  lse=st["lse"], block_table=cache.block_table, num_splits=st["splits"])
+    if ev is not None:
+        ev[1].record()
+    m.unabsorb_v(st["out_lat"], st["w_uv"], st["out"])
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    import mla_latent_kv_20_b200 as m
+    st = setup_replica(args.workload, dev)
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        run_step(st, i)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t_start.record()
+    for i in range(args.steps):
+        run_step(st, i, evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    dec_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    assert m.get_device_error() == 0
+
+    # end to end through the public API with host buffers: H2D of the step's inputs, the step,
+    # D2H of the result, every step
+    h = st["host"]
+    pin = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16 if v.dtype == np.uint16 else v.dtype))
+           .pin_memory() for k, v in h.items()}
+    out_host = torch.empty(st["out"].shape, dtype=torch.bfloat16).pin_memory()
+    dsts = {"q_nope": st["q_nope"], "q_pe": st["q_pe"], "c_new": st["c_new"], "kr_new": st["kr_new"],
+            "pos": st["pos"]}
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step(i):
+        for k, d in dsts.items():
+            d.view(pin[k].dtype).copy_(pin[k], non_blocking=True)
+        run_step(st, i)
+        out_host.copy_(st["out"], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+
+    t = torch.tensor([ms, e2e_ms, dec_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, e2e_ms, dec_ms = t.tolist()
+    if rank != 0:
+        return
+    tokens, cache_bytes, flops, dec_bytes = step_work(st["lens"])
+    hbm, tc, tc_sus, peak_kind = load_peaks()
+    value = world * cache_bytes / (ms * 1e-3) / 1e9
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    roofline_s = max(cache_bytes / (hbm * 1e9), flops / (tc * 1e12))
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) latents/keys/queries, "
+                                                     "N(0,1/512) weights)",
+        "config": {"workload": args.workload, "batch": st["B"], "seq_len": int(np.max(st["lens"])),
+                   "tokens": tokens, "paged": bool(st["w"]["paged"]), "splits": st["n_splits"],
+                   "cache_copies_rotated": len(st["caches"]),
+                   "l2": "inputs larger than L2: caches rotated, %d copies x %.0f MB" % (
+                       len(st["caches"]), cache_bytes / 1e6),
+                   "parallelism": f"replicas x{world}"},
+        "tflops": world * flops / (ms * 1e-3) / 1e12,
+        "tokens_per_s": world * st["B"] / (ms * 1e-3),
+        "roofline_step_frac": roofline_s / (ms * 1e-3),
+        "roofline": {"kernel": "mla_decode_attn (split-KV decode + combine)", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_kind": peak_kind, "traffic": None, "avg_launch_ms": dec_ms,
+                     "algorithmic_bytes_per_launch": dec_bytes},
+        "e2e": {"value": world * cache_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        L, dt = time_oracle(st["lens"])
+        threads, cores = cpu_threads()
+        line["cpu_baseline"] = {"value": L * ROW_BYTES / dt / 1e9, "unit": UNIT, "cores": threads,
+                                "kind": "oracle", "affinity_cores": cores,
+                                "sample": f"one sequence of {L} tokens, explicit fp64 form "
+                                          f"({dt:.1f} s), GB/s of cached rows processed"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(mi.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

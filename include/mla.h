@@ -1,0 +1,171 @@
+/*
+ * mla.h — C ABI of the B200 (sm_100a) library for DeepSeek-V2 Multi-head Latent Attention (MLA)
+ * decode over the compressed latent KV cache, in its weight-absorbed form.
+ *
+ * Sources (page title, section):
+ *   [DR] 《DeepSeek-V2》深度解读报告 — §2.2 Low-Rank Key-Value Joint Compression,
+ *        §2.3 Absorption, §2.4 Decoupled Rotary Position Embedding, §3.1 MLA 完整计算链路与参数核算.
+ *   [XD] DeepSeek-V2论文解读：MoE架构如何实现训练成本降42.5%与KV缓存压93.3% — §2.1.
+ *
+ * Fixed model dimensions ([DR] §3.1): n_h = 128 heads, d_h = 128, d_c = 512, d_R = 64.
+ * One cached row per token per layer is [c^KV (512) | RoPE(k^R) (64)] = 576 bf16 = 1152 bytes.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library never allocates,
+ *     frees or retains them.  bf16 values are passed as their 16-bit patterns (mla_bf16).
+ *   - Every tensor pointer must be 16-byte aligned (TMA requirement); MLA_ERR_INVALID_ARG otherwise.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only enqueue work on
+ *     it: they return after host-side validation, never synchronise, and are safe to capture in a
+ *     CUDA graph.  The return value reports host-side validation and launch errors only.
+ *   - Data-dependent faults (a position beyond the cache capacity, a block id outside the pool,
+ *     a bounded wait that gave up) are detected on the device: the offending row is skipped and
+ *     a sticky device error word is set; read it with mla_get_device_error().  No kernel traps.
+ */
+#ifndef MLA_B200_H_
+#define MLA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_N_HEADS 128
+#define MLA_D_HEAD 128
+#define MLA_D_LATENT 512
+#define MLA_D_ROPE 64
+#define MLA_D_ROW 576
+#define MLA_PAGE_SIZE 64
+
+typedef uint16_t mla_bf16; /* bfloat16 bit pattern */
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, inconsistent cache descriptor */
+  MLA_ERR_UNSUPPORTED = 2, /* a size outside what the kernels support */
+  MLA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than mla_decode_workspace_size() */
+  MLA_ERR_CUDA = 4,        /* a CUDA runtime/driver call or kernel launch failed */
+  MLA_ERR_DEVICE = 5       /* reported by mla_get_device_error(): a device-side check fired */
+} mla_status;
+
+/* Device error codes (bit flags) reported through mla_get_device_error(). */
+#define MLA_DEVERR_POS_RANGE 0x1     /* append: position >= capacity, or seq id out of range */
+#define MLA_DEVERR_BLOCK_RANGE 0x2   /* a block-table entry outside [0, num_blocks) */
+#define MLA_DEVERR_SEQLEN_RANGE 0x4  /* decode: seq_len < 0 or > capacity */
+#define MLA_DEVERR_WAIT_TIMEOUT 0x8  /* a bounded pipeline wait gave up; outputs of that CTA invalid */
+
+/*
+ * Layout of the latent cache of ONE layer ([DR] §2.4: (d_c + d_R) elements per token per layer).
+ *   page_size == 0  (contiguous): cache is [num_seqs][max_seq_len][576]; row of (seq b, token t)
+ *                   is b * max_seq_len + t.  block_table must be NULL.
+ *   page_size == 64 (paged, PagedAttention-style block table, [XD] §2.1): cache is
+ *                   [num_blocks][64][576]; row of (b, t) is block_table[b*max_blocks_per_seq + t/64]*64
+ *                   + t%64.  Capacity per sequence is max_blocks_per_seq * 64.
+ *   num_seqs: number of sequences the cache holds (contiguous: leading dimension of the buffer;
+ *             paged: rows of block_table).  Sequence ids and decode batch indices must be below it.
+ *   num_rows: total rows in the cache buffer (num_seqs*max_seq_len, or num_blocks*64); every row
+ *             index the library forms is checked against it on the device.
+ */
+typedef struct {
+  int32_t page_size;
+  int32_t max_seq_len;
+  int32_t max_blocks_per_seq;
+  int32_t num_seqs;
+  int64_t num_rows;
+} mla_cache_desc;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* mla_status_string(mla_status s);
+
+/* Library ABI version (major * 100 + minor). */
+int32_t mla_version(void);
+
+/*
+ * (1) Cache append — [DR] §2.4 (decoupled RoPE on the shared key branch) and §3.1 (c^KV and k^R
+ *     are the only cached objects).
+ * For each new token i in [0, n_tokens):
+ *     row = [ c_new[i, 0:512] | RoPE(kr_new[i, 0:64], pos[i]) ]  written to the slot of
+ *     (seq = seq_ids ? seq_ids[i] : i, token position pos[i]).
+ * RoPE rotates interleaved pairs (x[2j], x[2j+1]) by pos * rope_base^(-2j/64), computed in fp64
+ * and rounded once to bf16 (round-to-nearest-even).  c is copied bit-exactly.
+ *   c_new   [n_tokens, 512] bf16     kr_new [n_tokens, 64] bf16 (before RoPE)
+ *   seq_ids [n_tokens] int32 or NULL pos    [n_tokens] int32
+ *   cache   per desc (written)       block_table [num_seqs, max_blocks_per_seq] int32 (paged) or NULL
+ * n_tokens == 0 is a no-op.  Device checks: pos in [0, capacity) and the block id in range,
+ * else the row is skipped and MLA_DEVERR_POS_RANGE / MLA_DEVERR_BLOCK_RANGE is set.
+ */
+mla_status mla_cache_append(const mla_bf16* c_new, const mla_bf16* kr_new, const int32_t* seq_ids,
+                            const int32_t* pos, mla_bf16* cache, const int32_t* block_table,
+                            mla_cache_desc desc, int32_t n_tokens, float rope_base, void* stream);
+
+/*
+ * (2) Query absorption — [DR] §2.3 (q.(W_UK c) = (q W_UK).c by associativity).
+ *     q_full[b, h, 0:512]   = sum_j q_nope[b, h, j] * W_UK[h, j, :]        (tcgen05, fp32 accumulate)
+ *     q_full[b, h, 512:576] = q_pe[b, h, :], rotated at q_pos[b] if q_pos != NULL
+ *   q_nope [batch, 128, 128] bf16   q_pe [batch, 128, 64] bf16   q_pos [batch] int32 or NULL
+ *   w_uk   [128, 128, 512] bf16 (head, d_h, d_c)                  q_full [batch, 128, 576] bf16 (written)
+ * batch == 0 is a no-op; batch must be <= 65536.
+ */
+mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int32_t* q_pos,
+                        const mla_bf16* w_uk, mla_bf16* q_full, int32_t batch, float rope_base,
+                        void* stream);
+
+/*
+ * Number of KV splits the decode uses for this problem when num_splits == 0 (auto), or
+ * num_splits itself when it is positive (clamped to [1, 1024]).  Depends only on its arguments
+ * and the device's SM count.
+ */
+int32_t mla_decode_num_splits(int32_t batch, int32_t max_seq_len, int32_t num_splits);
+
+/*
+ * Bytes of workspace mla_decode_attn needs: split partials O [batch, S, 128, 512] fp32 plus
+ * (m, l) [batch, S, 128] fp32 each, with S = mla_decode_num_splits(batch, max_seq_len, num_splits).
+ */
+size_t mla_decode_workspace_size(int32_t batch, int32_t max_seq_len, int32_t num_splits);
+
+/*
+ * (3) Decode attention over the latent cache — [DR] §2.3/§2.4: score = scale * (q_abs.c + q_pe.k^R),
+ *     the sum of the content and position channels; out_lat = softmax-weighted sum of c.
+ * Split-KV flash decoding: sequence b's tokens [0, seq_lens[b]) are cut into S ranges whose
+ * bounds depend only on seq_lens[b] and S; each range keeps a running max m and sum l
+ * (online softmax) and writes an unnormalised partial; a combine merges the partials in
+ * ascending split order:
+ *     out_lat[b, h, :] = sum_s e^{m_s - M} O_s / sum_s e^{m_s - M} l_s,   M = max_s m_s
+ *     lse[b, h]        = M + log(sum_s e^{m_s - M} l_s)                    (natural log)
+ *   q_full   [batch, 128, 576] bf16     cache / block_table per desc     seq_lens [batch] int32
+ *   softmax_scale: e.g. 1/sqrt(192)     num_splits: 0 = auto, else forced
+ *   workspace: >= mla_decode_workspace_size(batch, desc.max_seq_len or capacity, num_splits) bytes,
+ *              16-byte aligned, contents need not be initialised (fully overwritten)
+ *   out_lat  [batch, 128, 512] bf16 (written)    lse [batch, 128] fp32 (written) or NULL
+ * The result for a sequence does not depend on the cache layout: paged and contiguous caches
+ * holding the same rows give bit-identical outputs.  A sequence with seq_len == 0 yields
+ * out_lat = 0 and lse = -inf.  seq_len > capacity sets MLA_DEVERR_SEQLEN_RANGE and is clamped.
+ */
+mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
+                           const int32_t* seq_lens, mla_cache_desc desc, int32_t batch,
+                           float softmax_scale, int32_t num_splits, void* workspace,
+                           size_t workspace_bytes, mla_bf16* out_lat, float* lse, void* stream);
+
+/*
+ * (4) Value un-absorption — [DR] §2.3 and [XD] §2.1 (W_UV applied after attention; folding
+ *     W_O in is left to the caller).
+ *     out[b, h, j] = sum_k out_lat[b, h, k] * W_UV[h, k, j]          (tcgen05, fp32 accumulate)
+ *   out_lat [batch, 128, 512] bf16   w_uv [128, 512, 128] bf16 (head, d_c, d_h)
+ *   out     [batch, 128, 128] bf16 (written)
+ * batch == 0 is a no-op; batch must be <= 65536.
+ */
+mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf16* out,
+                          int32_t batch, void* stream);
+
+/*
+ * Read and clear the sticky device error word of the current device (MLA_DEVERR_* flags).
+ * Synchronises the device.  Returns MLA_OK with *code == 0 when no check fired.
+ */
+mla_status mla_get_device_error(int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H_ */

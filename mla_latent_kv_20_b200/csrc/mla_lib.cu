@@ -1,0 +1,264 @@
+// mla_lib.cu — the C ABI declared in include/mla.h: host-side validation, TMA descriptor
+// construction and kernel launches.  Single translation unit (the kernels are header-only), so
+// the device error word needs no relocatable device code.
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mla.h"
+#include "append.cuh"
+#include "decode_common.cuh"
+#include "decode_simt.cuh"
+#include "gemm_tc.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+using mla::CacheView;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+mla_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map, 128-byte swizzle; inner is the contiguous dimension.
+bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                 uint32_t box_inner, uint32_t box_outer) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Validates a cache descriptor; on success fills the kernel-side view.
+mla_status check_cache(const mla_cache_desc& d, const void* cache, const int32_t* block_table, CacheView* v) {
+  if (cache == nullptr || !aligned16(cache)) return MLA_ERR_INVALID_ARG;
+  if (d.num_seqs <= 0 || d.num_rows <= 0) return MLA_ERR_INVALID_ARG;
+  if (d.page_size == 0) {
+    if (block_table != nullptr || d.max_seq_len <= 0) return MLA_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(d.num_seqs) * d.max_seq_len > d.num_rows) return MLA_ERR_INVALID_ARG;
+  } else if (d.page_size == MLA_PAGE_SIZE) {
+    if (block_table == nullptr || d.max_blocks_per_seq <= 0 || (d.num_rows % MLA_PAGE_SIZE) != 0)
+      return MLA_ERR_INVALID_ARG;
+    if (d.max_blocks_per_seq > INT_MAX / MLA_PAGE_SIZE) return MLA_ERR_UNSUPPORTED;
+  } else {
+    return MLA_ERR_UNSUPPORTED;
+  }
+  if (d.num_rows > (int64_t(1) << 40)) return MLA_ERR_UNSUPPORTED;
+  v->page_size = d.page_size;
+  v->max_seq_len = d.max_seq_len;
+  v->max_blocks = d.max_blocks_per_seq;
+  v->num_rows = d.num_rows;
+  v->block_table = block_table;
+  v->num_seqs = d.num_seqs;
+  return MLA_OK;
+}
+
+inline int cache_capacity(const mla_cache_desc& d) {
+  return d.page_size == 0 ? d.max_seq_len : d.max_blocks_per_seq * MLA_PAGE_SIZE;
+}
+
+constexpr int kMaxBatch = 65536;
+constexpr int kMaxSplits = 1024;
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE: return "MLA_ERR_DEVICE";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+int32_t mla_version(void) { return 100; }
+
+mla_status mla_get_device_error(int32_t* code) {
+  if (code == nullptr) return MLA_ERR_INVALID_ARG;
+  *code = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MLA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, mla::g_mla_dev_error, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(mla::g_mla_dev_error, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  *code = v;
+  return MLA_OK;
+}
+
+mla_status mla_cache_append(const mla_bf16* c_new, const mla_bf16* kr_new, const int32_t* seq_ids,
+                            const int32_t* pos, mla_bf16* cache, const int32_t* block_table,
+                            mla_cache_desc desc, int32_t n_tokens, float rope_base, void* stream) {
+  if (n_tokens < 0 || !(rope_base > 0.f) || !std::isfinite(rope_base)) return MLA_ERR_INVALID_ARG;
+  CacheView v;
+  const mla_status st = check_cache(desc, cache, block_table, &v);
+  if (st != MLA_OK) return st;
+  if (n_tokens == 0) return MLA_OK;
+  if (c_new == nullptr || kr_new == nullptr || pos == nullptr || !aligned16(c_new) || !aligned16(kr_new))
+    return MLA_ERR_INVALID_ARG;
+  if (seq_ids == nullptr && n_tokens > desc.num_seqs) return MLA_ERR_INVALID_ARG;
+  if (n_tokens > INT_MAX / 2) return MLA_ERR_UNSUPPORTED;
+  mla::cache_append_kernel<<<n_tokens, 72, 0, as_stream(stream)>>>(
+      reinterpret_cast<const uint4*>(c_new), reinterpret_cast<const uint4*>(kr_new), seq_ids, pos,
+      reinterpret_cast<uint4*>(cache), v, static_cast<double>(rope_base));
+  return launch_status();
+}
+
+}  // extern "C"
+
+namespace {
+
+template <int KTOT, int NSTAGE>
+mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, int batch, __nv_bfloat16* out,
+                            int64_t out_bstride, int out_hstride, cudaStream_t stream) {
+  // Weight viewed as [heads * KTOT rows][m_total cols]; activation as [batch rows][heads * KTOT cols].
+  const int nt = batch >= 256 ? 256 : ((batch + 15) / 16) * 16;
+  CUtensorMap ta, tb;
+  if (!make_map_2d(&ta, weight, m_total, static_cast<uint64_t>(mla::kHeads) * KTOT,
+                   static_cast<uint64_t>(m_total) * 2, 64, 64))
+    return MLA_ERR_CUDA;
+  if (!make_map_2d(&tb, act, static_cast<uint64_t>(mla::kHeads) * KTOT, batch,
+                   static_cast<uint64_t>(mla::kHeads) * KTOT * 2, 64, nt))
+    return MLA_ERR_CUDA;
+  const size_t smem = 1024 + NSTAGE * mla::gemm_stage_bytes(nt) + (2 * NSTAGE + 1) * 8 + 16;
+  auto kern = mla::proj_gemm_kernel<KTOT, NSTAGE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return MLA_ERR_CUDA;
+  dim3 grid(m_total / 128, mla::kHeads, (batch + nt - 1) / nt);
+  kern<<<grid, mla::kGemmThreads, smem, stream>>>(ta, tb, out, batch, nt, out_bstride, out_hstride);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int32_t* q_pos,
+                        const mla_bf16* w_uk, mla_bf16* q_full, int32_t batch, float rope_base,
+                        void* stream) {
+  if (batch < 0 || batch > kMaxBatch) return batch < 0 ? MLA_ERR_INVALID_ARG : MLA_ERR_UNSUPPORTED;
+  if (batch == 0) return MLA_OK;
+  if (q_nope == nullptr || q_pe == nullptr || w_uk == nullptr || q_full == nullptr) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(w_uk) || !aligned16(q_full)) return MLA_ERR_INVALID_ARG;
+  if (q_pos != nullptr && (!(rope_base > 0.f) || !std::isfinite(rope_base))) return MLA_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  mla_status st = launch_proj_gemm<mla::kDHead, 2>(w_uk, mla::kDLat, q_nope, batch,
+                                                   reinterpret_cast<__nv_bfloat16*>(q_full),
+                                                   static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow, s);
+  if (st != MLA_OK) return st;
+  mla::qpe_kernel<<<batch, mla::kHeads * 8, 0, s>>>(reinterpret_cast<const uint4*>(q_pe), q_pos,
+                                                    reinterpret_cast<uint4*>(q_full), static_cast<double>(rope_base));
+  return launch_status();
+}
+
+mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf16* out, int32_t batch,
+                          void* stream) {
+  if (batch < 0 || batch > kMaxBatch) return batch < 0 ? MLA_ERR_INVALID_ARG : MLA_ERR_UNSUPPORTED;
+  if (batch == 0) return MLA_OK;
+  if (out_lat == nullptr || w_uv == nullptr || out == nullptr) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(out_lat) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
+  return launch_proj_gemm<mla::kDLat, 4>(w_uv, mla::kDHead, out_lat, batch, reinterpret_cast<__nv_bfloat16*>(out),
+                                         static_cast<int64_t>(mla::kHeads) * mla::kDHead, mla::kDHead,
+                                         as_stream(stream));
+}
+
+int32_t mla_decode_num_splits(int32_t batch, int32_t max_seq_len, int32_t num_splits) {
+  if (num_splits > 0) return num_splits > kMaxSplits ? kMaxSplits : num_splits;
+  if (batch <= 0 || max_seq_len <= 0) return 1;
+  // Aim for about two waves of CTAs (8 head-group CTAs per (sequence, split)), with at least
+  // 256 tokens per split.
+  const int sms = device_sm_count();
+  const int per_split_ctas = mla::kHeads / mla::kSimtHeads;
+  int s = (2 * sms + batch * per_split_ctas - 1) / (batch * per_split_ctas);
+  const int by_len = (max_seq_len + 255) / 256;
+  if (s > by_len) s = by_len;
+  if (s < 1) s = 1;
+  if (s > kMaxSplits) s = kMaxSplits;
+  return s;
+}
+
+size_t mla_decode_workspace_size(int32_t batch, int32_t max_seq_len, int32_t num_splits) {
+  if (batch <= 0) return 0;
+  return mla::ws_bytes(batch, mla_decode_num_splits(batch, max_seq_len, num_splits));
+}
+
+mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
+                           const int32_t* seq_lens, mla_cache_desc desc, int32_t batch, float softmax_scale,
+                           int32_t num_splits, void* workspace, size_t workspace_bytes, mla_bf16* out_lat,
+                           float* lse, void* stream) {
+  if (batch < 0 || num_splits < 0) return MLA_ERR_INVALID_ARG;
+  if (batch > kMaxBatch) return MLA_ERR_UNSUPPORTED;
+  if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+  CacheView v;
+  const mla_status st = check_cache(desc, cache, block_table, &v);
+  if (st != MLA_OK) return st;
+  if (batch == 0) return MLA_OK;
+  if (batch > desc.num_seqs) return MLA_ERR_INVALID_ARG;
+  if (q_full == nullptr || seq_lens == nullptr || out_lat == nullptr) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_full) || !aligned16(out_lat) || (lse != nullptr && !aligned16(lse))) return MLA_ERR_INVALID_ARG;
+  const int capacity = cache_capacity(desc);
+  const int S = mla_decode_num_splits(batch, capacity, num_splits);
+  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < mla::ws_bytes(batch, S))
+    return MLA_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const mla::Workspace ws = mla::ws_carve(workspace, batch, S);
+  const size_t smem = mla::simt_smem_bytes();
+  if (cudaFuncSetAttribute(mla::decode_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  dim3 grid(mla::kHeads / mla::kSimtHeads, S, batch);
+  mla::decode_simt_kernel<<<grid, 256, smem, s>>>(reinterpret_cast<const __nv_bfloat16*>(q_full),
+                                                  reinterpret_cast<const __nv_bfloat16*>(cache), v, seq_lens, S,
+                                                  softmax_scale * mla::kLog2e, ws);
+  mla_status ls = launch_status();
+  if (ls != MLA_OK) return ls;
+  mla::combine_kernel<<<dim3(batch, mla::kHeads / 4), 128, 0, s>>>(
+      ws, seq_lens, S, mla::kSplitAlign, capacity, reinterpret_cast<__nv_bfloat16*>(out_lat), lse);
+  return launch_status();
+}
+
+}  // extern "C"

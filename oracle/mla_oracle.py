@@ -87,8 +87,8 @@ def decompress(c: np.ndarray, w_uk: np.ndarray, w_uv: np.ndarray):
     c: [L, d_c]; w_uk: [H, d_h, d_c]; w_uv: [H, d_c, d_h].  Returns kC, vC of shape [L, H, d_h].
     """
     c = np.asarray(c, dtype=np.float64)
-    kC = np.einsum("hjk,lk->lhj", np.asarray(w_uk, np.float64), c)
-    vC = np.einsum("hkj,lk->lhj", np.asarray(w_uv, np.float64), c)
+    kC = np.einsum("hjk,lk->lhj", np.asarray(w_uk, np.float64), c, optimize=True)
+    vC = np.einsum("hkj,lk->lhj", np.asarray(w_uv, np.float64), c, optimize=True)
     return kC, vC
 
 
@@ -124,7 +124,7 @@ def attend_explicit(q_nope, q_pe, c, kr_rot, w_uk, w_uv, scale):
         k = np.concatenate([kC[:, h, :], kr_rot], axis=1)   # [L, d_h + d_R]
         s[h] = scale * (k @ q)
     p, lse = softmax_stats(s)
-    out = np.einsum("ht,thj->hj", p, vC)
+    out = np.einsum("ht,thj->hj", p, vC, optimize=True)
     out_lat = p @ c
     return dict(out=out, out_lat=out_lat, lse=lse, p=p, s=s)
 
@@ -134,12 +134,12 @@ def attend_explicit(q_nope, q_pe, c, kr_rot, w_uk, w_uv, scale):
 # ----------------------------------------------------------------------------------------
 def absorb_q(q_nope: np.ndarray, w_uk: np.ndarray) -> np.ndarray:
     """q_abs[..., h, k] = sum_j q_nope[..., h, j] W_UK[h, j, k]   ([..., H, d_h] -> [..., H, d_c])."""
-    return np.einsum("...hj,hjk->...hk", np.asarray(q_nope, np.float64), np.asarray(w_uk, np.float64))
+    return np.einsum("...hj,hjk->...hk", np.asarray(q_nope, np.float64), np.asarray(w_uk, np.float64), optimize=True)
 
 
 def unabsorb_v(out_lat: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
     """out[..., h, j] = sum_k out_lat[..., h, k] W_UV[h, k, j]   ([..., H, d_c] -> [..., H, d_h])."""
-    return np.einsum("...hk,hkj->...hj", np.asarray(out_lat, np.float64), np.asarray(w_uv, np.float64))
+    return np.einsum("...hk,hkj->...hj", np.asarray(out_lat, np.float64), np.asarray(w_uv, np.float64), optimize=True)
 
 
 def q_full(q_abs: np.ndarray, q_pe: np.ndarray) -> np.ndarray:

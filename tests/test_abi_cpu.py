@@ -1,0 +1,97 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every entry point that
+include/mla.h declares, and its host-side validation returns the documented status codes
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def mla():
+    import __graft_entry__
+    __graft_entry__._build_module().build()
+    import mla_latent_kv_20_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "mla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(mla_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ("mla_cache_append", "mla_absorb_q", "mla_decode_attn", "mla_unabsorb_v",
+              "mla_decode_workspace_size", "mla_get_device_error", "mla_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(mla):
+    lib = ctypes.CDLL(mla.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings(mla):
+    assert mla.status_string(0) == "MLA_OK"
+    assert mla.status_string(3) == "MLA_ERR_WORKSPACE"
+    assert mla.status_string(99) == "MLA_ERR_UNKNOWN"
+    assert mla.lib.mla_version() >= 100
+
+
+FAKE = 0x10000  # never dereferenced: validation fails first
+
+
+def test_append_validation(mla):
+    lib = mla.lib
+    good = mla.contiguous_desc(4, 128)
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, None, None, good, 4, 10000.0, None) == 1  # null cache
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE + 8, None, good, 4, 10000.0, None) == 1  # misaligned
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE, None, good, -1, 10000.0, None) == 1
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE, None, good, 4, -1.0, None) == 1
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE, None, good, 0, 10000.0, None) == 0   # no-op
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE, None, good, 5, 10000.0, None) == 1   # > num_seqs
+    bad_page = mla.CacheDesc(32, 128, 2, 4, 4 * 128)
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE, FAKE, bad_page, 4, 10000.0, None) == 2
+    paged_no_table = mla.paged_desc(4, 2, 8)
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE, None, paged_no_table, 4, 10000.0, None) == 1
+    contiguous_with_table = mla.contiguous_desc(4, 128)
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE, FAKE, contiguous_with_table, 4, 10000.0, None) == 1
+    too_few_rows = mla.CacheDesc(0, 128, 0, 4, 100)
+    assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE, None, too_few_rows, 1, 10000.0, None) == 1
+
+
+def test_projection_validation(mla):
+    lib = mla.lib
+    assert lib.mla_absorb_q(FAKE, FAKE, None, FAKE, FAKE, 0, 10000.0, None) == 0
+    assert lib.mla_absorb_q(FAKE, FAKE, None, FAKE, FAKE, -1, 10000.0, None) == 1
+    assert lib.mla_absorb_q(FAKE, FAKE, None, FAKE, FAKE, 70000, 10000.0, None) == 2
+    assert lib.mla_absorb_q(None, FAKE, None, FAKE, FAKE, 4, 10000.0, None) == 1
+    assert lib.mla_absorb_q(FAKE, FAKE, None, FAKE, FAKE + 2, 4, 10000.0, None) == 1
+    assert lib.mla_absorb_q(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 0.0, None) == 1
+    assert lib.mla_unabsorb_v(FAKE, FAKE, FAKE, 0, None) == 0
+    assert lib.mla_unabsorb_v(FAKE, None, FAKE, 4, None) == 1
+    assert lib.mla_unabsorb_v(FAKE, FAKE, FAKE + 4, 4, None) == 1
+
+
+def test_decode_validation_and_workspace(mla):
+    lib = mla.lib
+    d = mla.contiguous_desc(8, 4096)
+    S = lib.mla_decode_num_splits(8, 4096, 16)
+    assert S == 16 and lib.mla_decode_num_splits(8, 4096, 5000) == 1024
+    need = lib.mla_decode_workspace_size(8, 4096, 16)
+    assert need == 8 * 16 * 128 * (512 + 2) * 4
+    args = lambda ws, nbytes, scale=0.072, batch=8, splits=16, desc=d: (  # noqa: E731
+        FAKE, FAKE, None, FAKE, desc, batch, scale, splits, ws, nbytes, FAKE, None, None)
+    assert lib.mla_decode_attn(*args(FAKE, need - 16)) == 3           # workspace too small
+    assert lib.mla_decode_attn(*args(None, need)) == 3                # workspace missing
+    assert lib.mla_decode_attn(*args(FAKE, need, scale=0.0)) == 1     # bad scale
+    assert lib.mla_decode_attn(*args(FAKE, need, batch=9)) == 1       # batch > num_seqs
+    assert lib.mla_decode_attn(*args(FAKE, need, batch=0)) == 0       # empty batch is a no-op
+    assert lib.mla_decode_attn(*args(FAKE, need, splits=-1)) == 1
+    assert lib.mla_get_device_error(None) == 1
