@@ -159,8 +159,10 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
                           int32_t batch, void* stream);
 
 /*
- * Read and clear the sticky device error word of the current device (MLA_DEVERR_* flags).
- * Synchronises the device.  Returns MLA_OK with *code == 0 when no check fired.
+ * Read and clear the sticky device error word of the current device: bits 0..7 are MLA_DEVERR_*
+ * flags; when MLA_DEVERR_WAIT_TIMEOUT is set, bits 8..15 hold the id of the first pipeline wait
+ * that gave up (a diagnostic for locating a protocol error).  Synchronises the device.
+ * Returns MLA_OK with *code == 0 when no check fired.
  */
 mla_status mla_get_device_error(int32_t* code);
 

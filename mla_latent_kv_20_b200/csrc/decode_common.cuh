@@ -26,6 +26,8 @@ __host__ __device__ __forceinline__ int splits_used(int L, int S, int align) {
   return (L + c - 1) / c;
 }
 
+constexpr int kSplitAlign = 128;  // split boundaries are multiples of this many tokens
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -62,8 +64,12 @@ __device__ __forceinline__ int seq_len_checked(const int32_t* seq_lens, int b, i
 
 // Combine: one warp per (b, h); lanes own 16 of the 512 latent columns.  Splits are merged in
 // ascending order.  grid = (batch, 128 / 4), block = 128.
+// Sequences whose tokens fit in one split were finalised by the decode kernel itself
+// (`single_done`); the combine only writes empty sequences (out_lat = 0, lse = -inf) and merges
+// sequences with two or more used splits.
 __global__ void __launch_bounds__(128) combine_kernel(Workspace ws, const int32_t* __restrict__ seq_lens, int S,
-                                                      int align, int capacity, __nv_bfloat16* __restrict__ out_lat,
+                                                      int align, int capacity, int single_done,
+                                                      __nv_bfloat16* __restrict__ out_lat,
                                                       float* __restrict__ lse) {
   const int b = blockIdx.x;
   const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
@@ -71,6 +77,7 @@ __global__ void __launch_bounds__(128) combine_kernel(Workspace ws, const int32_
   int L = seq_lens[b];
   L = L < 0 ? 0 : (L > capacity ? capacity : L);
   const int n = splits_used(L, S, align);
+  if (n == 1 && single_done) return;
   const int64_t base = static_cast<int64_t>(b) * S * kHeads;
   float M = -INFINITY;
   for (int s = 0; s < n; ++s) M = fmaxf(M, ws.m[base + static_cast<int64_t>(s) * kHeads + h]);

@@ -14,7 +14,7 @@
 #include "../../include/mla.h"
 #include "append.cuh"
 #include "decode_common.cuh"
-#include "decode_simt.cuh"
+#include "decode_tc.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 
@@ -96,6 +96,27 @@ inline int cache_capacity(const mla_cache_desc& d) {
   return d.page_size == 0 ? d.max_seq_len : d.max_blocks_per_seq * MLA_PAGE_SIZE;
 }
 
+// Number of CTA pairs of the decode kernel that can be resident at once on the current device.
+int decode_cluster_slots() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 74;
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaFuncSetAttribute(mla::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           mla::kTcSmemBytes) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(192, 1, 1);
+    cfg.dynamicSmemBytes = mla::kTcSmemBytes;
+    if (cudaOccupancyMaxActiveClusters(&n, mla::decode_tc_kernel, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  if (n <= 0) n = device_sm_count() / 2;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
 constexpr int kMaxBatch = 65536;
 constexpr int kMaxSplits = 1024;
 
@@ -121,11 +142,13 @@ mla_status mla_get_device_error(int32_t* code) {
   if (code == nullptr) return MLA_ERR_INVALID_ARG;
   *code = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return MLA_ERR_CUDA;
-  int v = 0;
+  int v = 0, site = 0;
   if (cudaMemcpyFromSymbol(&v, mla::g_mla_dev_error, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&site, mla::g_mla_dev_error_site, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
   const int zero = 0;
   if (cudaMemcpyToSymbol(mla::g_mla_dev_error, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
-  *code = v;
+  if (cudaMemcpyToSymbol(mla::g_mla_dev_error_site, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  *code = v | ((site & 0xFF) << 8);
   return MLA_OK;
 }
 
@@ -209,16 +232,26 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
 int32_t mla_decode_num_splits(int32_t batch, int32_t max_seq_len, int32_t num_splits) {
   if (num_splits > 0) return num_splits > kMaxSplits ? kMaxSplits : num_splits;
   if (batch <= 0 || max_seq_len <= 0) return 1;
-  // Aim for about two waves of CTAs (8 head-group CTAs per (sequence, split)), with at least
-  // 256 tokens per split.
-  const int sms = device_sm_count();
-  const int per_split_ctas = mla::kHeads / mla::kSimtHeads;
-  int s = (2 * sms + batch * per_split_ctas - 1) / (batch * per_split_ctas);
-  const int by_len = (max_seq_len + 255) / 256;
-  if (s > by_len) s = by_len;
-  if (s < 1) s = 1;
-  if (s > kMaxSplits) s = kMaxSplits;
-  return s;
+  // Each (sequence, split) is one CTA pair.  Pick the split count whose pairs fill the resident
+  // pair slots best (fewest idle slots in the last wave), with at least two 128-token tiles per
+  // split; ties go to fewer splits (less partial traffic).
+  const int slots = decode_cluster_slots();
+  int s_max = (max_seq_len + 2 * mla::kTcTile - 1) / (2 * mla::kTcTile);
+  if (s_max < 1) s_max = 1;
+  if (s_max > kMaxSplits) s_max = kMaxSplits;
+  int best = 1;
+  double best_eff = -1.0;
+  for (int s = 1; s <= s_max; ++s) {
+    const long long units = static_cast<long long>(batch) * s;
+    const long long waves = (units + slots - 1) / slots;
+    const double eff = static_cast<double>(units) / static_cast<double>(waves * slots);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+    if (units >= 4LL * slots) break;
+  }
+  return best;
 }
 
 size_t mla_decode_workspace_size(int32_t batch, int32_t max_seq_len, int32_t num_splits) {
@@ -244,20 +277,31 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
   const int S = mla_decode_num_splits(batch, capacity, num_splits);
   if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < mla::ws_bytes(batch, S))
     return MLA_ERR_WORKSPACE;
+  if (desc.num_rows >= (int64_t(1) << 31) || static_cast<int64_t>(batch) * mla::kHeads >= (int64_t(1) << 31))
+    return MLA_ERR_UNSUPPORTED;
   cudaStream_t s = as_stream(stream);
-  const mla::Workspace ws = mla::ws_carve(workspace, batch, S);
-  const size_t smem = mla::simt_smem_bytes();
-  if (cudaFuncSetAttribute(mla::decode_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
+  mla::DecodeTcArgs a;
+  a.v = v;
+  a.seq_lens = seq_lens;
+  a.S = S;
+  a.scale_log2 = softmax_scale * mla::kLog2e;
+  a.ws = mla::ws_carve(workspace, batch, S);
+  a.out_lat = reinterpret_cast<__nv_bfloat16*>(out_lat);
+  a.lse = lse;
+  CUtensorMap tkc, tvc, tq;
+  if (!make_map_2d(&tkc, cache, mla::kDRow, desc.num_rows, mla::kDRow * 2, 64, 64) ||
+      !make_map_2d(&tvc, cache, mla::kDRow, desc.num_rows, mla::kDRow * 2, 64, 32) ||
+      !make_map_2d(&tq, q_full, mla::kDRow, static_cast<uint64_t>(batch) * mla::kHeads, mla::kDRow * 2, 64, 64))
     return MLA_ERR_CUDA;
-  dim3 grid(mla::kHeads / mla::kSimtHeads, S, batch);
-  mla::decode_simt_kernel<<<grid, 256, smem, s>>>(reinterpret_cast<const __nv_bfloat16*>(q_full),
-                                                  reinterpret_cast<const __nv_bfloat16*>(cache), v, seq_lens, S,
-                                                  softmax_scale * mla::kLog2e, ws);
+  if (cudaFuncSetAttribute(mla::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kTcSmemBytes) !=
+      cudaSuccess)
+    return MLA_ERR_CUDA;
+  mla::decode_tc_kernel<<<dim3(2 * S, batch), 192, mla::kTcSmemBytes, s>>>(tkc, tvc, tq, a);
   mla_status ls = launch_status();
   if (ls != MLA_OK) return ls;
   mla::combine_kernel<<<dim3(batch, mla::kHeads / 4), 128, 0, s>>>(
-      ws, seq_lens, S, mla::kSplitAlign, capacity, reinterpret_cast<__nv_bfloat16*>(out_lat), lse);
+      a.ws, seq_lens, S, mla::kSplitAlign, capacity, /*single_done=*/1, reinterpret_cast<__nv_bfloat16*>(out_lat),
+      lse);
   return launch_status();
 }
 

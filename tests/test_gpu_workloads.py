@@ -1,0 +1,59 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py times (auto split count,
+or the forced 128 splits of the long-context workload), checked on sampled sequences that the
+fp64 oracle computes one by one."""
+import numpy as np
+import pytest
+
+import mla_inputs as mi
+import oracle
+from gpu_common import SCALE, assert_full_path, mean_rel
+
+pytestmark = pytest.mark.gpu
+f64 = mi.bf16_to_f64
+
+
+def _run_workload(name, sample, explicit_first=True):
+    import torch
+    from mla_latent_kv_20_b200 import get_device_error
+    from mla_latent_kv_20_b200 import harness as hz
+    w = mi.WORKLOADS[name]
+    lens = mi.workload_lengths(name)
+    seed = w["seed"]
+    batch = mi.decode_batch(seed, lens)
+    wts = mi.layer_weights(seed + 1)
+    table, nblk = mi.block_permutation(seed + 2, lens) if w["paged"] else (None, 0)
+    cache = hz.Cache(lens, w["paged"], table, nblk, fill_value=None)
+    cache.fill(batch.c, batch.kr)
+    qpos = torch.from_numpy(np.asarray(lens, np.int32) - 1).cuda()
+    out, out_lat, lse, _ = hz.decode_step(hz.bf16_tensor(batch.q_nope), hz.bf16_tensor(batch.q_pe),
+                                          hz.bf16_tensor(wts.w_uk), hz.bf16_tensor(wts.w_uv), cache,
+                                          q_pos=qpos, num_splits=int(w.get("splits", 0)))
+    torch.cuda.synchronize()
+    assert get_device_error() == 0
+    g_out = f64(hz.bf16_bits(out))
+    g_lse = lse.cpu().numpy()
+    for k, i in enumerate(sample):
+        L = int(lens[i])
+        form = "explicit" if (explicit_first and k == 0) else "absorbed"
+        ref = oracle.decode_step(f64(batch.q_nope[i:i + 1]), f64(batch.q_pe[i:i + 1]), [f64(batch.c[i])],
+                                 [f64(batch.kr[i])], f64(wts.w_uk), f64(wts.w_uv), SCALE, q_pos=[L - 1], form=form)
+        assert_full_path(g_out[i], ref["out"][0])
+        assert np.abs(g_lse[i] - ref["lse"][0]).max() <= 5e-3
+        assert mean_rel(g_out[i], ref["out"][0]) <= 5e-3
+
+
+def test_b1_l256():
+    _run_workload("b1_l256", [0])
+
+
+def test_b32_l4096():
+    _run_workload("b32_l4096", [0, 17, 31])
+
+
+def test_b128_paged_uniform_lengths():
+    lens = mi.workload_lengths("b128_u1024_8192_paged")
+    _run_workload("b128_u1024_8192_paged", [int(np.argmin(lens)), int(np.argmax(lens)), 64])
+
+
+def test_b4_l131072_128_splits():
+    _run_workload("b4_l131072", [2], explicit_first=False)
