@@ -160,64 +160,117 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------------------------- ours
-def setup_replica(name, device):
-    import torch
+def _new_token_inputs(batch, lens):
+    last = np.asarray(lens, np.int32) - 1
+    new_c = np.stack([batch.c[i][last[i]] for i in range(len(lens))])
+    new_kr = np.stack([batch.kr[i][last[i]] for i in range(len(lens))])
+    return last, new_c, new_kr
+
+
+def _layer_from_host(name, device):
+    """One layer whose inputs come from the seeded host generator (workloads that fit through numpy)."""
     from mla_latent_kv_20_b200 import harness as hz
     w, lens = workload_shape(name)
     seed = w["seed"]
-    B = len(lens)
     batch = mi.decode_batch(seed, lens)
     wts = mi.layer_weights(seed + 1)
     table, nblk = mi.block_permutation(seed + 2, lens) if w["paged"] else (None, 0)
-    base = hz.Cache(lens, w["paged"], table, nblk, device=device, fill_value=None)
-    base.fill(batch.c, batch.kr)
-    _, cache_bytes, _, _ = step_work(lens)
-    n_copies = max(2, math.ceil(3 * L2_BYTES / max(cache_bytes, 1)))
-    caches = [base]
-    for _ in range(n_copies - 1):
-        c = hz.Cache.__new__(hz.Cache)
-        c.__dict__.update(base.__dict__)
-        c.data = base.data.clone()
-        caches.append(c)
-    last = np.asarray(lens, np.int32) - 1
-    new_c = np.stack([batch.c[i][last[i]] for i in range(B)])
-    new_kr = np.stack([batch.kr[i][last[i]] for i in range(B)])
-    st = dict(
-        B=B, lens=lens, w=w, caches=caches,
-        q_nope=hz.bf16_tensor(batch.q_nope, device), q_pe=hz.bf16_tensor(batch.q_pe, device),
-        c_new=hz.bf16_tensor(new_c, device), kr_new=hz.bf16_tensor(new_kr, device),
-        pos=torch.from_numpy(last).to(device), seq_ids=torch.arange(B, dtype=torch.int32, device=device),
-        w_uk=hz.bf16_tensor(wts.w_uk, device), w_uv=hz.bf16_tensor(wts.w_uv, device),
-        q_full=torch.empty((B, 128, 576), dtype=torch.bfloat16, device=device),
-        out_lat=torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device),
-        lse=torch.empty((B, 128), dtype=torch.float32, device=device),
-        out=torch.empty((B, 128, 128), dtype=torch.bfloat16, device=device),
-        splits=int(w.get("splits", 0)),
-        host=dict(q_nope=batch.q_nope, q_pe=batch.q_pe, c_new=new_c, kr_new=new_kr, pos=last),
-    )
+    cache = hz.Cache(lens, w["paged"], table, nblk, device=device, fill_value=None)
+    cache.fill(batch.c, batch.kr)
+    last, new_c, new_kr = _new_token_inputs(batch, lens)
+    host = dict(q_nope=batch.q_nope, q_pe=batch.q_pe, c_new=new_c, kr_new=new_kr)
+    return dict(caches=[cache], w_uk=hz.bf16_tensor(wts.w_uk, device), w_uv=hz.bf16_tensor(wts.w_uv, device),
+                host=host, dev={k: hz.bf16_tensor(v, device) for k, v in host.items()})
+
+
+def _layer_on_device(name, layer, device, chunk_tokens=1 << 18):
+    """One layer of a workload too large for host generation: every value is drawn on the device
+    from a seeded torch generator (N(0,1) latents/keys/queries, N(0,1/512) weights), then the cache
+    is filled through mla_cache_append."""
+    import torch
     import mla_latent_kv_20_b200 as m
-    ws_bytes = m.decode_workspace_size(B, base.capacity(), st["splits"])
-    st["workspace"] = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=device)
-    st["n_splits"] = m.decode_num_splits(B, base.capacity(), st["splits"])
+    from mla_latent_kv_20_b200 import harness as hz
+    w, lens = workload_shape(name)
+    seed = w["seed"] + 7919 * layer
+    B = len(lens)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+
+    def normal(shape, std=1.0):
+        return (torch.randn(shape, generator=g, device=device, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    table, nblk = mi.block_permutation(seed + 2, lens) if w["paged"] else (None, 0)
+    cache = hz.Cache(lens, w["paged"], table, nblk, device=device, fill_value=None)
+    seq_ids = torch.from_numpy(np.concatenate([np.full(L, i, np.int32) for i, L in enumerate(lens)])).to(device)
+    pos = torch.from_numpy(np.concatenate([np.arange(L, dtype=np.int32) for L in lens])).to(device)
+    for o in range(0, len(pos), chunk_tokens):
+        n = min(chunk_tokens, len(pos) - o)
+        m.cache_append(normal((n, 512)), normal((n, 64)), pos[o:o + n], cache.data, cache.desc,
+                       seq_ids=seq_ids[o:o + n], block_table=cache.block_table)
+    dev = dict(q_nope=normal((B, 128, 128)), q_pe=normal((B, 128, 64)), c_new=normal((B, 512)),
+               kr_new=normal((B, 64)))
+    return dict(caches=[cache], w_uk=normal((128, 128, 512), 1 / math.sqrt(512)),
+                w_uv=normal((128, 512, 128), 1 / math.sqrt(512)), host=None, dev=dev)
+
+
+def setup_replica(name, device):
+    import torch
+    import mla_latent_kv_20_b200 as m
+    w, lens = workload_shape(name)
+    B = len(lens)
+    n_layers = int(w.get("layers", 1))
+    if n_layers == 1:
+        layers = [_layer_from_host(name, device)]
+        _, cache_bytes, _, _ = step_work(lens)
+        n_copies = max(2, math.ceil(3 * L2_BYTES / max(cache_bytes, 1)))
+        base = layers[0]["caches"][0]
+        for _ in range(n_copies - 1):
+            c = type(base).__new__(type(base))
+            c.__dict__.update(base.__dict__)
+            c.data = base.data.clone()
+            layers[0]["caches"].append(c)
+    else:
+        layers = [_layer_on_device(name, l, device) for l in range(n_layers)]
+    last = np.asarray(lens, np.int32) - 1
+    base = layers[0]["caches"][0]
+    splits = int(w.get("splits", 0))
+    ws_bytes = m.decode_workspace_size(B, base.capacity(), splits)
+    st = dict(B=B, lens=lens, w=w, layers=layers, splits=splits,
+              n_splits=m.decode_num_splits(B, base.capacity(), splits),
+              pos=torch.from_numpy(last).to(device), pos_host=last,
+              seq_ids=torch.arange(B, dtype=torch.int32, device=device),
+              q_full=torch.empty((B, 128, 576), dtype=torch.bfloat16, device=device),
+              out_lat=torch.empty((B, 128, 512), dtype=torch.bfloat16, device=device),
+              lse=torch.empty((B, 128), dtype=torch.float32, device=device),
+              out=torch.empty((B, 128, 128), dtype=torch.bfloat16, device=device),
+              workspace=torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=device))
     return st
 
 
-LAUNCHES_PER_STEP = 6   # append, absorb GEMM, q_pe rotation, decode split, combine, un-absorb GEMM
+LAUNCHES_PER_LAYER = 6   # append, absorb GEMM, q_pe rotation, decode split, combine, un-absorb GEMM
 
 
 def run_step(st, i, ev=None):
+    """One decode step over every layer of the workload."""
     import mla_latent_kv_20_b200 as m
-    cache = st["caches"][i % len(st["caches"])]
-    m.cache_append(st["c_new"], st["kr_new"], st["pos"], cache.data, cache.desc, seq_ids=st["seq_ids"],
-                   block_table=cache.block_table)
-    m.absorb_q(st["q_nope"], st["q_pe"], st["w_uk"], st["q_full"], q_pos=st["pos"])
-    if ev is not None:
-        ev[0].record()
-    m.decode_attn(st["q_full"], cache.data, cache.seq_lens, cache.desc, st["workspace"], st["out_lat"],
-                  lse=st["lse"], block_table=cache.block_table, num_splits=st["splits"])
-    if ev is not None:
-        ev[1].record()
-    m.unabsorb_v(st["out_lat"], st["w_uv"], st["out"])
+    for li, layer in enumerate(st["layers"]):
+        cache = layer["caches"][i % len(layer["caches"])]
+        d = layer["dev"]
+        m.cache_append(d["c_new"], d["kr_new"], st["pos"], cache.data, cache.desc, seq_ids=st["seq_ids"],
+                       block_table=cache.block_table)
+        m.absorb_q(d["q_nope"], d["q_pe"], layer["w_uk"], st["q_full"], q_pos=st["pos"])
+        if ev is not None:
+            ev[li][0].record()
+        m.decode_attn(st["q_full"], cache.data, cache.seq_lens, cache.desc, st["workspace"], st["out_lat"],
+                      lse=st["lse"], block_table=cache.block_table, num_splits=st["splits"])
+        if ev is not None:
+            ev[li][1].record()
+        m.unabsorb_v(st["out_lat"], layer["w_uv"], st["out"])
+
+
+def hz_bits(t):
+    from mla_latent_kv_20_b200 import harness as hz
+    return hz.bf16_bits(t)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -237,7 +290,9 @@ def run_ours(args, rank, world, local_rank):
     for i in range(args.warmup):
         run_step(st, i)
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    n_layers = len(st["layers"])
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_layers)]
+           for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
     sampler.start()
@@ -252,23 +307,26 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     clocks = sampler.stop()
     ms = t_start.elapsed_time(t_end) / args.steps
-    dec_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    dec_ms = sum(a.elapsed_time(b) for step in evs for a, b in step) / (args.steps * n_layers)
     assert m.get_device_error() == 0
 
-    # end to end through the public API with host buffers: H2D of the step's inputs, the step,
-    # D2H of the result, every step
-    h = st["host"]
-    pin = {k: torch.from_numpy(np.ascontiguousarray(v).view(np.int16 if v.dtype == np.uint16 else v.dtype))
-           .pin_memory() for k, v in h.items()}
+    # end to end through the public API with host buffers: H2D of the step's inputs (every layer's
+    # new-token row and query), the step, D2H of the result, every step
+    pin, dsts = [], []
+    for layer in st["layers"]:
+        for k, d in layer["dev"].items():
+            hsrc = layer["host"][k] if layer["host"] is not None else hz_bits(d)
+            pin.append(torch.from_numpy(np.ascontiguousarray(hsrc).view(np.int16)).pin_memory())
+            dsts.append(d)
+    pin.append(torch.from_numpy(st["pos_host"]).pin_memory())
+    dsts.append(st["pos"])
     out_host = torch.empty(st["out"].shape, dtype=torch.bfloat16).pin_memory()
-    dsts = {"q_nope": st["q_nope"], "q_pe": st["q_pe"], "c_new": st["c_new"], "kr_new": st["kr_new"],
-            "pos": st["pos"]}
-    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    h2d = sum(v.numel() * v.element_size() for v in pin)
     d2h = out_host.numel() * out_host.element_size()
 
     def e2e_step(i):
-        for k, d in dsts.items():
-            d.view(pin[k].dtype).copy_(pin[k], non_blocking=True)
+        for hsrc, d in zip(pin, dsts):
+            d.view(hsrc.dtype).copy_(hsrc, non_blocking=True)
         run_step(st, i)
         out_host.copy_(st["out"], non_blocking=True)
 
@@ -292,6 +350,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return
     tokens, cache_bytes, flops, dec_bytes = step_work(st["lens"])
+    tokens, cache_bytes, flops = tokens * n_layers, cache_bytes * n_layers, flops * n_layers
     hbm, tc, tc_sus, peak_kind = load_peaks()
     value = world * cache_bytes / (ms * 1e-3) / 1e9
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
@@ -302,13 +361,15 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) latents/keys/queries, "
                                                      "N(0,1/512) weights)",
         "config": {"workload": args.workload, "batch": st["B"], "seq_len": int(np.max(st["lens"])),
-                   "tokens": tokens, "paged": bool(st["w"]["paged"]), "splits": st["n_splits"],
-                   "cache_copies_rotated": len(st["caches"]),
-                   "l2": "inputs larger than L2: caches rotated, %d copies x %.0f MB" % (
-                       len(st["caches"]), cache_bytes / 1e6),
+                   "layers": n_layers, "tokens_per_layer": tokens // n_layers, "paged": bool(st["w"]["paged"]),
+                   "splits": st["n_splits"],
+                   "l2": "inputs larger than L2: %d cache cop%s rotated, %.0f MB each" % (
+                       len(st["layers"][0]["caches"]) * n_layers, "y" if n_layers * len(st["layers"][0]["caches"]) == 1 else "ies",
+                       cache_bytes / n_layers / 1e6),
                    "parallelism": f"replicas x{world}"},
         "tflops": world * flops / (ms * 1e-3) / 1e12,
         "tokens_per_s": world * st["B"] / (ms * 1e-3),
+        "decode_layer_ms": dec_ms,
         "roofline_step_frac": roofline_s / (ms * 1e-3),
         "roofline": {"kernel": "mla_decode_attn (split-KV decode + combine)", "bound": "hbm",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
@@ -316,7 +377,7 @@ def run_ours(args, rank, world, local_rank):
                      "algorithmic_bytes_per_launch": dec_bytes},
         "e2e": {"value": world * cache_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": LAUNCHES_PER_LAYER * n_layers * args.steps,
         "clocks": clocks,
     }
     if not args.no_cpu_baseline:

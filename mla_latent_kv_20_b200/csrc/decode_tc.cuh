@@ -63,7 +63,8 @@ struct TcBars {
   uint64_t s_full[2];            // both: QK^T of a tile done
   uint64_t p_full[2];            // even CTA only: P (and corrected O) of a tile ready in both CTAs
   uint64_t p_empty[2];           // both: PV of a tile done reading P
-  uint64_t o_ready;              // both: PV of a tile done writing O
+  uint64_t o_ready;              // both: PV of a tile done writing O (one phase per tile)
+  uint64_t o_final;              // both: the last PV done (single phase, read by the epilogue)
   uint64_t q_full;               // even CTA only: Q of both CTAs landed
   uint64_t fix;                  // per CTA: local loads of ragged V slabs
 };
@@ -222,6 +223,9 @@ __device__ bool tc_mma(uint8_t* smem, TcBars* bars, uint32_t tmem, int n_tiles, 
   bool ok = qk(0);
   for (int i = 1; ok && i < n_tiles; ++i) ok = qk(i) && pv(i - 1);
   if (ok) ok = pv(n_tiles - 1);
+  // The epilogue cannot wait on o_ready by parity: when it starts, o_ready may still be two
+  // phases short of the last one.  A dedicated single-phase barrier says "all PV done".
+  umma_commit_pair_mc(&bars->o_final, 3);
   if (!ok) *abort_flag = 1;
   return ok;
 }
@@ -278,7 +282,8 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
       need = true;
     }
     if (__any_sync(0xffffffffu, need)) {
-      // O must hold PV(i-1) before it is scaled.
+      // O must hold PV(i-1) before it is scaled.  Waiting on phase i-1 by parity is unambiguous
+      // here: s_full(i) was committed after PV(i-2), so o_ready is in phase i-1 or i.
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_ready, static_cast<uint32_t>(i - 1) & 1u, 0x31))) {
         ok = false;
         break;
@@ -322,7 +327,7 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
     if (lane == 0) mbar_arrive_addr(lbar(&bars->p_full[j]));
   }
   // ---- epilogue
-  if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_ready, static_cast<uint32_t>(n_tiles - 1) & 1u, 0x33))) ok = false;
+  if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0u, 0x33))) ok = false;
   tc_fence_after();
   red[256 + t] = l_run;
   named_bar_sync(1, 128);
@@ -408,6 +413,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_init(&bars->p_empty[j], 1);
     }
     mbar_init(&bars->o_ready, 1);
+    mbar_init(&bars->o_final, 1);
     mbar_init(&bars->q_full, 2);
     mbar_init(&bars->fix, 1);
     *abort_flag = 0;

@@ -306,3 +306,4 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
 }
 
 }  // extern "C"
+

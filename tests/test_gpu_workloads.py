@@ -57,3 +57,36 @@ def test_b128_paged_uniform_lengths():
 
 def test_b4_l131072_128_splits():
     _run_workload("b4_l131072", [2], explicit_first=False)
+
+
+def test_l60_one_layer_full_size():
+    """One layer of the 60-layer whole-model workload at its full per-layer size (batch 256,
+    log-uniform lengths in [64, 32768], paged), sampled sequences against the oracle."""
+    lens = mi.workload_lengths("l60_b256_log64_32768_paged")
+    _run_workload("l60_b256_log64_32768_paged", [int(np.argmin(lens)), int(np.argmax(lens)), 100],
+                  explicit_first=False)
+
+
+def test_multi_layer_step_distinct_weights_and_caches():
+    """A step over several layers, each with its own weights and paged cache, as the whole-model
+    workload runs it: every layer's output matches the oracle for that layer."""
+    import torch
+    from mla_latent_kv_20_b200 import get_device_error
+    from mla_latent_kv_20_b200 import harness as hz
+    lens = mi.log_uniform_lengths(77, 8, 64, 3000)
+    for layer in range(3):
+        seed = 5000 + 7919 * layer
+        b = mi.decode_batch(seed, lens)
+        w = mi.layer_weights(seed + 1)
+        table, nblk = mi.block_permutation(seed + 2, lens)
+        cache = hz.Cache(lens, True, table, nblk, fill_value=float("nan"))
+        cache.fill(b.c, b.kr)
+        qpos = np.asarray(lens, np.int32) - 1
+        out, _, lse, _ = hz.decode_step(hz.bf16_tensor(b.q_nope), hz.bf16_tensor(b.q_pe), hz.bf16_tensor(w.w_uk),
+                                        hz.bf16_tensor(w.w_uv), cache, q_pos=torch.from_numpy(qpos).cuda())
+        torch.cuda.synchronize()
+        assert get_device_error() == 0
+        ref = oracle.decode_step(f64(b.q_nope), f64(b.q_pe), [f64(x) for x in b.c], [f64(x) for x in b.kr],
+                                 f64(w.w_uk), f64(w.w_uv), SCALE, q_pos=qpos, form="absorbed")
+        assert_full_path(f64(hz.bf16_bits(out)), ref["out"])
+        assert np.abs(lse.cpu().numpy() - ref["lse"]).max() <= 5e-3
