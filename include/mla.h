@@ -148,6 +148,29 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
                            size_t workspace_bytes, mla_bf16* out_lat, float* lse, void* stream);
 
 /*
+ * Decode attention that allocates nothing and takes no workspace (the pages have no counterpart:
+ * this is a deployment convenience of this library).
+ * For callers that cannot obtain device memory at decode time, for example a plugin inside a
+ * host engine that owns every device allocation, or a fixed-budget deployment that forbids
+ * cudaMalloc after start-up.  Same arguments, result and checks as mla_decode_attn, except that
+ * the split partials live in a library-owned static device buffer of MLA_NOALLOC_SCRATCH_BYTES
+ * (32 MiB) that every GPU which loads the library holds until the process exits.
+ *   - Returns MLA_ERR_WORKSPACE, launching nothing, when mla_decode_workspace_size(batch,
+ *     capacity, num_splits) exceeds MLA_NOALLOC_SCRATCH_BYTES (use fewer splits or a smaller batch).
+ *   - The first call on a device looks up the buffer's device address (once per device, with that
+ *     device current); make that first call before any stream capture.
+ *   - All calls share the one buffer: calls whose kernels overlap on the GPU (different streams,
+ *     no ordering between them) race and give wrong results.  The buffer keeps the last call's
+ *     contents; nothing in it needs to start at zero (the kernels overwrite what they read).
+ *   - Calls no allocation routine (cudaMalloc, cudaFree, or a library allocator).
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+mla_status mla_decode_attn_noalloc(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
+                                   const int32_t* seq_lens, mla_cache_desc desc, int32_t batch,
+                                   float softmax_scale, int32_t num_splits, mla_bf16* out_lat, float* lse,
+                                   void* stream);
+
+/*
  * (4) Value un-absorption — [DR] §2.3 and [XD] §2.1 (W_UV applied after attention; folding
  *     W_O in is left to the caller).
  *     out[b, h, j] = sum_k out_lat[b, h, k] * W_UV[h, k, j]          (tcgen05, fp32 accumulate)

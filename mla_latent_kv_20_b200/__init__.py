@@ -56,6 +56,7 @@ def _load():
         "mla_decode_workspace_size": (SZ, [I32, I32, I32]),
         "mla_decode_attn": (ctypes.c_int, [P, P, P, P, CacheDesc, I32, F32, I32, P, SZ, P, P, P]),
         "mla_unabsorb_v": (ctypes.c_int, [P, P, P, I32, P]),
+        "mla_decode_attn_noalloc": (ctypes.c_int, [P, P, P, P, CacheDesc, I32, F32, I32, P, P, P]),
         "mla_get_device_error": (ctypes.c_int, [ctypes.POINTER(I32)]),
     }
     for name, (res, args) in sigs.items():
@@ -124,6 +125,20 @@ def decode_attn(q_full, cache, seq_lens, desc: CacheDesc, workspace, out_lat, *,
     _check(lib.mla_decode_attn(_ptr(q_full), _ptr(cache), _ptr(block_table), _ptr(seq_lens), desc, b,
                                softmax_scale, num_splits, _ptr(workspace), wb, _ptr(out_lat), _ptr(lse),
                                _stream(stream)), "mla_decode_attn")
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def decode_attn_noalloc(q_full, cache, seq_lens, desc: CacheDesc, out_lat, *, lse=None, block_table=None,
+                        softmax_scale: float = 1.0 / 192 ** 0.5, num_splits: int = 0, stream=None,
+                        batch: int | None = None):
+    """mla_decode_attn without a workspace: for callers that cannot allocate device memory at
+    decode time; split partials go to the library's static 32 MiB device buffer."""
+    b = q_full.shape[0] if batch is None else batch
+    _check(lib.mla_decode_attn_noalloc(_ptr(q_full), _ptr(cache), _ptr(block_table), _ptr(seq_lens), desc, b,
+                                       softmax_scale, num_splits, _ptr(out_lat), _ptr(lse), _stream(stream)),
+           "mla_decode_attn_noalloc")
 
 
 def unabsorb_v(out_lat, w_uv, out, *, stream=None, batch: int | None = None):

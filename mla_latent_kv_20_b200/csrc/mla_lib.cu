@@ -307,3 +307,48 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
 
 }  // extern "C"
 
+// ------------------------------------------------------------------------------------------
+// Decode without caller memory: split partials in a library-owned static device buffer.
+// ------------------------------------------------------------------------------------------
+namespace {
+
+// One buffer per device (a __device__ array exists once in every context that loads the
+// library).  Host code must not pass its host-side symbol: the device address is looked up with
+// cudaGetSymbolAddress once per device, with that device current.
+__device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+mla_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" mla_status mla_decode_attn_noalloc(const mla_bf16* q_full, const mla_bf16* cache,
+                                              const int32_t* block_table, const int32_t* seq_lens,
+                                              mla_cache_desc desc, int32_t batch, float softmax_scale,
+                                              int32_t num_splits, mla_bf16* out_lat, float* lse, void* stream) {
+  if (batch < 0 || num_splits < 0) return MLA_ERR_INVALID_ARG;
+  if (batch == 0) return MLA_OK;
+  const int capacity = desc.page_size == 0 ? desc.max_seq_len : desc.max_blocks_per_seq * MLA_PAGE_SIZE;
+  if (capacity <= 0) return MLA_ERR_INVALID_ARG;
+  if (mla_decode_workspace_size(batch, capacity, num_splits) > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const mla_status st = noalloc_scratch(&scratch);
+  if (st != MLA_OK) return st;
+  return mla_decode_attn(q_full, cache, block_table, seq_lens, desc, batch, softmax_scale, num_splits, scratch,
+                         MLA_NOALLOC_SCRATCH_BYTES, out_lat, lse, stream);
+}
