@@ -12,19 +12,23 @@
 // receives a 64-head slice of the accumulator folded over all 128 lanes, so
 //   S tile (64 heads x 128 tokens, fp32)  = 64 TMEM columns per CTA (two buffers),
 //   O      (64 heads x 512 latent, fp32)  = 256 TMEM columns per CTA.
-// Per 128-token tile the B operand of QK^T is split by tokens (CTA r loads tokens [64r, 64r+64),
-// all 576 dims, 9 slabs of 64 dims) and the B operand of PV is split by latent columns (CTA r
-// loads latent [256n + 128r, +128) of all 128 tokens, 8 slabs of 32 tokens).  All slabs are 8 KB
-// per CTA and stream through one ring of shared-memory stages filled by TMA (128-byte swizzle)
-// in exactly the order the MMA issuer consumes them:  K(0) K(1) V(0) K(2) V(1) ... V(n-1).
+// Per 128-token tile the B operand of QK^T is split by tokens: CTA r holds tokens [64r, 64r+64)
+// with all 576 dims, as 9 swizzled slabs of 64 dims.  The B operand of PV is split by latent
+// columns: CTA r holds latent [256n + 128r, +128) of all 128 tokens (slabs of 32 tokens), a
+// second read of the tile's rows that hits L2 because the pair reads them within microseconds.
 //
-// Warp roles (192 threads): warps 0-3 softmax / O correction / epilogue (thread = TMEM lane),
-// warp 4 TMA producer, warp 5 TMEM allocation and (even CTA only) MMA issue.
+// Staging.  The TMA unit of a CTA works through its tensor copies one at a time at a roughly
+// fixed cost per copy (measured: ~0.35 us for anything from 8 KB to 72 KB), so every copy is
+// large: K rows (from HBM) come as 3-D boxes of 3 dim-slabs (24 KB, 3 copies per tile) into a
+// 3-slot K ring, and V rows (the L2 re-read) as 4-D boxes of 64 tokens x both 64-wide latent
+// chunks x both latent halves (32 KB, 2 copies per tile) into a 2-slot V ring.  Separate rings let
+// the K copies of the next tile proceed while V of the current tile waits for its softmax.
+// V rows past the split end are zeroed in shared memory before PV (rows past a sequence's end may
+// hold anything, and 0 * NaN would poison the sum).
 //
-// Masking.  Tokens >= the split end are excluded by setting their scores to -inf.  V rows of
-// such tokens are zeroed in shared memory before PV (cache rows past a sequence's end may hold
-// anything, and 0 * NaN would poison the sum); K rows need no fix because their scores are
-// replaced, not scaled.
+// Warp roles (320 threads): warps 0-7 softmax / O correction / epilogue (two warps per TMEM lane
+// quadrant, each owning half of the S columns), warp 8 TMA producer, warp 9 TMEM allocation and
+// (even CTA only) MMA issue.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -33,19 +37,29 @@
 
 namespace mla {
 
-constexpr int kTcTile = 128;         // tokens per tile
-constexpr int kTcStages = 14;        // 8 KB slabs in the ring
-constexpr int kTcSlab = 8192;
+constexpr int kTcTile = 128;                 // tokens per tile
+constexpr int kTcSlab = 8192;                // 64 rows x 128 bytes
+constexpr int kTcKBoxSlabs = 3;              // dim-slabs per K TMA box
+constexpr int kTcKBoxes = 9 / kTcKBoxSlabs;  // K boxes per tile
+constexpr int kTcKSlots = 3;
+constexpr int kTcVSlots = 2;
+constexpr int kTcVBox = 4 * kTcSlab;         // 64 tokens x 2 chunks x 2 latent halves
 constexpr int kTcQBytes = 9 * kTcSlab;
-constexpr int kTcPBytes = 2 * kTcSlab;   // 64 heads x 128 tokens bf16, two 64-token K chunks
+constexpr int kTcPBytes = 2 * kTcSlab;       // 64 heads x 128 tokens bf16, two 64-token K chunks
 constexpr float kTcRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows > 2^8
 
 constexpr int kTcOffQ = 0;
 constexpr int kTcOffP = kTcOffQ + kTcQBytes;
-constexpr int kTcOffRing = kTcOffP + 2 * kTcPBytes;
-constexpr int kTcOffBar = kTcOffRing + kTcStages * kTcSlab;
-constexpr int kTcOffMisc = kTcOffBar + 512;
-constexpr int kTcSmemBytes = kTcOffMisc + 2048 + 1024;   // + slack for 1024-byte alignment
+constexpr int kTcOffK = kTcOffP + kTcPBytes;
+constexpr int kTcOffV = kTcOffK + kTcKSlots * kTcKBoxSlabs * kTcSlab;
+constexpr int kTcOffBar = kTcOffV + kTcVSlots * kTcVBox;
+constexpr int kTcOffMisc = kTcOffBar + 256;
+constexpr int kTcSmemBytes = kTcOffMisc + 64 + 2 * 256 * 4;   // the dynamic base is 1024-aligned (checked)
+
+constexpr int kTcSoftmaxWarps = 8;
+constexpr int kTcProducerWarp = 8;
+constexpr int kTcMmaWarp = 9;
+constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 2);
 
 struct DecodeTcArgs {
   CacheView v;
@@ -58,17 +72,20 @@ struct DecodeTcArgs {
 };
 
 struct TcBars {
-  uint64_t kv_full[kTcStages];   // even CTA only: both CTAs' slab halves landed
-  uint64_t kv_empty[kTcStages];  // both CTAs: slab consumed by the MMAs
+  uint64_t k_full[kTcKSlots];    // even CTA only: both CTAs' K boxes landed (one arrival per CTA + tx)
+  uint64_t k_empty[kTcKSlots];   // both CTAs: K box consumed by the MMAs
+  uint64_t v_full[kTcVSlots];    // even CTA only: both CTAs' V box landed (one arrival per CTA + tx)
+  uint64_t v_empty[kTcVSlots];   // both CTAs: V box consumed
+  uint64_t fix;                  // per CTA: local load of a ragged V box
   uint64_t s_full[2];            // both: QK^T of a tile done
-  uint64_t p_full[2];            // even CTA only: P (and corrected O) of a tile ready in both CTAs
-  uint64_t p_empty[2];           // both: PV of a tile done reading P
+  uint64_t p_full;               // even CTA only: P (and corrected O) of a tile ready in both CTAs
+  uint64_t p_empty;              // both: PV of a tile done reading P
   uint64_t o_ready;              // both: PV of a tile done writing O (one phase per tile)
   uint64_t o_final;              // both: the last PV done (single phase, read by the epilogue)
   uint64_t q_full;               // even CTA only: Q of both CTAs landed
-  uint64_t fix;                  // per CTA: local loads of ragged V slabs
 };
-static_assert(sizeof(TcBars) <= 512, "barrier block");
+static_assert(sizeof(TcBars) <= 256, "barrier block");
+static_assert(kTcSmemBytes <= 232448, "shared memory budget");
 
 // Row of (seq b, token t) for a TMA coordinate; -kTcTile (a fully out-of-bounds box, which the
 // TMA unit fills with zeros) when the mapping is invalid.
@@ -79,88 +96,116 @@ __device__ __forceinline__ int tma_row(const CacheView& v, int b, int t) {
 
 __device__ __forceinline__ uint32_t lbar(const void* p) { return mapa_shared(smem_u32(p), 0); }
 
-// ------------------------------------------------------------------------------ TMA producer
-struct TcRing {
-  int n = 0;  // slabs issued / consumed so far
-  __device__ __forceinline__ int slot() const { return n % kTcStages; }
-  __device__ __forceinline__ uint32_t round_parity() const { return static_cast<uint32_t>(n / kTcStages) & 1u; }
-};
+// 3-D TMA load (x: element in a 64-wide dim-slab, y: cache row, z: dim-slab) into this CTA's
+// shared memory; completion counted on a barrier that may live in the peer CTA.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster_addr, int x,
+                                                 int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster_addr), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 
-// Zero token rows [v, 32) of both 4 KB latent chunks of a V slab (rows are 128 bytes).
-__device__ __forceinline__ void zero_v_rows(uint8_t* slab, int v) {
-  for (int c = 0; c < 2; ++c)
-    for (int row = v; row < 32; ++row) {
-      uint4* p = reinterpret_cast<uint4*>(slab + c * 4096 + row * 128);
+// 4-D TMA load (x: element in a 64-wide chunk, y: cache row, z: chunk, w: latent half).
+__device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster_addr, int x,
+                                                 int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster_addr), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d_local(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y, int z,
+                                                  int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
+// ------------------------------------------------------------------------------ TMA producer
+// Issue order K(0), K(1), V(0), K(2), V(1), ..., V(n-1): the order the MMA issuer consumes them,
+// with K one tile ahead so QK^T of tile i+1 never waits behind V of tile i.
+//  K(i): CTA r's 64 tokens [tile0 + 64r, +64) x 576 dims as kTcKBoxes boxes of kTcKBoxSlabs
+//        dim-slabs.  A half-tile past the split end is loaded from a negative row (zeros); its
+//        scores are masked anyway.
+//  V(i): per 64-token half h of the tile, latent [256n + 128r, +128) for n = 0, 1 in one box,
+//        laid out [n][chunk][64 rows][128 B].
+__device__ __forceinline__ void zero_v_rows(uint8_t* box, int v) {
+  for (int q = 0; q < 4; ++q)
+    for (int row = v; row < 64; ++row) {
+      uint4* p = reinterpret_cast<uint4*>(box + q * kTcSlab + row * 128);
 #pragma unroll
       for (int u = 0; u < 8; ++u) p[u] = make_uint4(0, 0, 0, 0);
     }
 }
 
-__device__ bool tc_producer(const CUtensorMap* tm_kc, const CUtensorMap* tm_vc, const CUtensorMap* tm_q,
-                            const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, uint32_t rank, int b,
-                            int t_begin, int t_end, int n_tiles, volatile int* abort_flag) {
+__device__ bool tc_producer(const CUtensorMap* tm_k, const CUtensorMap* tm_v, const CUtensorMap* tm_q,
+                            const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, uint32_t rank, int b, int t_begin,
+                            int t_end, int n_tiles, volatile int* abort_flag) {
   const bool leader = rank == 0;
-  // Q: 9 boxes of 64 dims x 64 heads.
+  // Q: 3 boxes of 3 dim-slabs x 64 heads.  Arrivals on the even CTA's barriers that only count
+  // (the data and its visibility come with the TMA's complete_tx) are relaxed.
+  for (int kb = 0; kb < kTcKBoxes; ++kb)
+    tma_load_3d_pair(smem + kTcOffQ + kb * kTcKBoxSlabs * kTcSlab, tm_q, lbar(&bars->q_full), 0,
+                     b * kHeads + 64 * static_cast<int>(rank), kb * kTcKBoxSlabs);
   if (leader)
-    mbar_arrive_expect_tx_addr(lbar(&bars->q_full), 2u * kTcQBytes);
+    mbar_arrive_expect_tx_relaxed(lbar(&bars->q_full), 2u * kTcQBytes);
   else
-    mbar_arrive_addr(lbar(&bars->q_full));
-  for (int c = 0; c < 9; ++c)
-    tma_load_2d_pair(smem + kTcOffQ + c * kTcSlab, tm_q, lbar(&bars->q_full), 64 * c, b * kHeads + 64 * rank);
-
-  TcRing ring;
+    mbar_arrive_relaxed(lbar(&bars->q_full));
+  int kn = 0, vn = 0;
   uint32_t fix_phase = 0;
-  auto acquire = [&](int& s) -> bool {
-    s = ring.slot();
-    if (ring.n >= kTcStages && !mbar_wait(&bars->kv_empty[s], ring.round_parity() ^ 1u, 0x10)) return false;
-    return !*abort_flag;
-  };
   auto issue_k = [&](int i) -> bool {
-    const int tile0 = t_begin + i * kTcTile;
-    const int my0 = tile0 + 64 * static_cast<int>(rank);
+    const int my0 = t_begin + i * kTcTile + 64 * static_cast<int>(rank);
     const int y = my0 < t_end ? tma_row(a.v, b, my0) : -kTcTile;
-    for (int c = 0; c < 9; ++c) {
-      int s;
-      if (!acquire(s)) return false;
-      if (leader) mbar_arrive_expect_tx_addr(lbar(&bars->kv_full[s]), 2u * kTcSlab);
-      tma_load_2d_pair(smem + kTcOffRing + s * kTcSlab, tm_kc, lbar(&bars->kv_full[s]), 64 * c, y);
-      mbar_arrive_addr(lbar(&bars->kv_full[s]));
-      ++ring.n;
+    for (int kb = 0; kb < kTcKBoxes; ++kb, ++kn) {
+      const int s = kn % kTcKSlots;
+      if (kn >= kTcKSlots && !mbar_wait(&bars->k_empty[s], static_cast<uint32_t>((kn / kTcKSlots) - 1) & 1u, 0x10))
+        return false;
+      if (*abort_flag) return false;
+      tma_load_3d_pair(smem + kTcOffK + s * kTcKBoxSlabs * kTcSlab, tm_k, lbar(&bars->k_full[s]), 0, y,
+                       kb * kTcKBoxSlabs);
+      if (leader)
+        mbar_arrive_expect_tx_relaxed(lbar(&bars->k_full[s]), 2u * kTcKBoxSlabs * kTcSlab);
+      else
+        mbar_arrive_relaxed(lbar(&bars->k_full[s]));
     }
     return true;
   };
   auto issue_v = [&](int i) -> bool {
-    const int tile0 = t_begin + i * kTcTile;
-    for (int nh = 0; nh < 2; ++nh)
-      for (int kt = 0; kt < 4; ++kt) {
-        int s;
-        if (!acquire(s)) return false;
-        uint8_t* slab = smem + kTcOffRing + s * kTcSlab;
-        const int tok0 = tile0 + 32 * kt;
-        const int vcount = min(max(t_end - tok0, 0), 32);
-        const int x0 = 256 * nh + 128 * static_cast<int>(rank);
-        if (vcount == 32) {
-          const int y = tma_row(a.v, b, tok0);
-          if (leader) mbar_arrive_expect_tx_addr(lbar(&bars->kv_full[s]), 2u * kTcSlab);
-          tma_load_2d_pair(slab, tm_vc, lbar(&bars->kv_full[s]), x0, y);
-          tma_load_2d_pair(slab + 4096, tm_vc, lbar(&bars->kv_full[s]), x0 + 64, y);
-        } else {
-          // Ragged: load locally, zero the rows past the end, then publish.
-          if (leader) mbar_arrive_expect_tx_addr(lbar(&bars->kv_full[s]), 0u);
-          if (vcount > 0) {
-            const int y = tma_row(a.v, b, tok0);
-            mbar_arrive_expect_tx(&bars->fix, 2u * 4096u);
-            tma_load_2d(slab, tm_vc, &bars->fix, x0, y);
-            tma_load_2d(slab + 4096, tm_vc, &bars->fix, x0 + 64, y);
-            if (!mbar_wait(&bars->fix, fix_phase, 0x11)) return false;
-            fix_phase ^= 1u;
-          }
-          zero_v_rows(slab, vcount);
-          fence_proxy_async_smem();
+    for (int h = 0; h < 2; ++h, ++vn) {
+      const int s = vn % kTcVSlots;
+      if (vn >= kTcVSlots && !mbar_wait(&bars->v_empty[s], static_cast<uint32_t>((vn / kTcVSlots) - 1) & 1u, 0x11))
+        return false;
+      if (*abort_flag) return false;
+      uint8_t* box = smem + kTcOffV + s * kTcVBox;
+      const int tok0 = t_begin + i * kTcTile + 64 * h;
+      const int vcount = min(max(t_end - tok0, 0), 64);
+      if (vcount == 64) {
+        tma_load_4d_pair(box, tm_v, lbar(&bars->v_full[s]), 0, tma_row(a.v, b, tok0), 2 * static_cast<int>(rank), 0);
+        if (leader)
+          mbar_arrive_expect_tx_relaxed(lbar(&bars->v_full[s]), 2u * kTcVBox);
+        else
+          mbar_arrive_relaxed(lbar(&bars->v_full[s]));
+      } else {
+        // Ragged: load through a CTA-local barrier, zero the rows past the end, then publish with
+        // release semantics (the zeros are this thread's own shared-memory writes).
+        if (vcount > 0) {
+          mbar_arrive_expect_tx(&bars->fix, kTcVBox);
+          tma_load_4d_local(box, tm_v, &bars->fix, 0, tma_row(a.v, b, tok0), 2 * static_cast<int>(rank), 0);
+          if (!mbar_wait(&bars->fix, fix_phase, 0x13)) return false;
+          fix_phase ^= 1u;
         }
-        mbar_arrive_addr(lbar(&bars->kv_full[s]));
-        ++ring.n;
+        zero_v_rows(box, vcount);
+        fence_proxy_async_smem();
+        if (leader)
+          mbar_arrive_expect_tx_addr(lbar(&bars->v_full[s]), 0u);
+        else
+          mbar_arrive_addr(lbar(&bars->v_full[s]));
       }
+    }
     return true;
   };
   bool ok = issue_k(0);
@@ -170,53 +215,56 @@ __device__ bool tc_producer(const CUtensorMap* tm_kc, const CUtensorMap* tm_vc, 
 }
 
 // ------------------------------------------------------------------------------ MMA issuer (even CTA)
+// Order: QK(0), then for each tile i >= 1: QK(i), PV(i-1); finally PV(n-1).  QK^T of the next tile
+// thus runs on the tensor cores while the softmax warps work on the current one.
 __device__ bool tc_mma(uint8_t* smem, TcBars* bars, uint32_t tmem, int n_tiles, volatile int* abort_flag) {
   const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
   const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
   const uint32_t sq = smem_u32(smem + kTcOffQ);
   const uint32_t sp = smem_u32(smem + kTcOffP);
-  const uint32_t sr = smem_u32(smem + kTcOffRing);
+  const uint32_t sk = smem_u32(smem + kTcOffK);
+  const uint32_t sv = smem_u32(smem + kTcOffV);
   if (!mbar_wait_cluster(&bars->q_full, 0, 0x20)) return false;
   tc_fence_after();
-  TcRing ring;
+  int kn = 0, vn = 0;
   auto qk = [&](int i) -> bool {
     const int j = i & 1;
-    for (int c = 0; c < 9; ++c) {
-      const int s = ring.slot();
-      if (!mbar_wait_cluster(&bars->kv_full[s], ring.round_parity(), 0x21)) return false;
+    for (int kb = 0; kb < kTcKBoxes; ++kb, ++kn) {
+      const int s = kn % kTcKSlots;
+      if (!mbar_wait_cluster(&bars->k_full[s], static_cast<uint32_t>(kn / kTcKSlots) & 1u, 0x21)) return false;
       tc_fence_after();
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint64_t ad = sdesc_sw128(sq + c * kTcSlab + 32 * k, 16, 1024);
-        const uint64_t bd = sdesc_sw128(sr + s * kTcSlab + 32 * k, 16, 1024);
-        umma_bf16_pair(tmem + 64 * j, ad, bd, idesc_qk, (c | k) != 0 ? 1u : 0u);
-      }
-      umma_commit_pair_mc(&bars->kv_empty[s], 3);
-      ++ring.n;
+      for (int c = 0; c < kTcKBoxSlabs; ++c)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = sdesc_sw128(sq + (kb * kTcKBoxSlabs + c) * kTcSlab + 32 * k, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sk + (s * kTcKBoxSlabs + c) * kTcSlab + 32 * k, 16, 1024);
+          umma_bf16_pair(tmem + 64 * j, ad, bd, idesc_qk, (kb | c | k) != 0 ? 1u : 0u);
+        }
+      umma_commit_pair_mc(&bars->k_empty[s], 3);
     }
     umma_commit_pair_mc(&bars->s_full[j], 3);
     return true;
   };
   auto pv = [&](int i) -> bool {
-    const int j = i & 1;
-    if (!mbar_wait_cluster(&bars->p_full[j], static_cast<uint32_t>(i >> 1) & 1u, 0x22)) return false;
+    if (!mbar_wait_cluster(&bars->p_full, static_cast<uint32_t>(i) & 1u, 0x22)) return false;
+    int vs[2];
+    for (int h = 0; h < 2; ++h, ++vn) {
+      vs[h] = vn % kTcVSlots;
+      if (!mbar_wait_cluster(&bars->v_full[vs[h]], static_cast<uint32_t>(vn / kTcVSlots) & 1u, 0x23)) return false;
+    }
     tc_fence_after();
     for (int nh = 0; nh < 2; ++nh)
-      for (int kt = 0; kt < 4; ++kt) {
-        const int s = ring.slot();
-        if (!mbar_wait_cluster(&bars->kv_full[s], ring.round_parity(), 0x23)) return false;
-        tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const int g = 2 * kt + kk;  // 16-token group within the tile
-          const uint64_t ad = sdesc_sw128(sp + j * kTcPBytes + (g >> 2) * kTcSlab + 32 * (g & 3), 16, 1024);
-          const uint64_t bd = sdesc_sw128(sr + s * kTcSlab + kk * 2048, 4096, 1024);
-          umma_bf16_pair(tmem + 128 + 128 * nh, ad, bd, idesc_pv, (i > 0 || kt > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit_pair_mc(&bars->kv_empty[s], 3);
-        ++ring.n;
+      for (int g = 0; g < 8; ++g) {  // 16-token groups of the tile
+        const uint64_t ad = sdesc_sw128(sp + (g >> 2) * kTcSlab + 32 * (g & 3), 16, 1024);
+        const uint32_t vb = sv + vs[g >> 2] * kTcVBox + nh * 2 * kTcSlab + (g & 3) * 2048;
+        const uint64_t bd = sdesc_sw128(vb, kTcSlab, 1024);
+        umma_bf16_pair(tmem + 128 + 128 * nh, ad, bd, idesc_pv, (i > 0 || g > 0) ? 1u : 0u);
       }
-    umma_commit_pair_mc(&bars->p_empty[j], 3);
+    umma_commit_pair_mc(&bars->v_empty[vs[0]], 3);
+    umma_commit_pair_mc(&bars->v_empty[vs[1]], 3);
+    umma_commit_pair_mc(&bars->p_empty, 3);
     umma_commit_pair_mc(&bars->o_ready, 3);
     return true;
   };
@@ -231,16 +279,28 @@ __device__ bool tc_mma(uint8_t* smem, TcBars* bars, uint32_t tmem, int n_tiles, 
 }
 
 // ------------------------------------------------------------------------------ softmax warps
-// Thread t (0..127) owns TMEM lane t: head 64*rank + (t & 63); lanes 0-63 hold tokens [0,64) of a
-// tile and latent columns 256n + [0,128) of O, lanes 64-127 tokens [64,128) and 256n + [128,256).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Eight warps: warp w reads TMEM lane quadrant w % 4 and column half ch = w / 4, so thread
+// (t = TMEM lane, ch) owns head 64*rank + (t & 63), the 32 tokens 64*(t >> 6) + 32*ch + [0, 32)
+// of every tile, and O columns [128*ch, 128*ch + 128) of its lane (latent 256*ch + 128*(t >> 6)
+// + [0, 128)).  The four threads (t, ch), (t ^ 64, ch), (t, ch ^ 1), (t ^ 64, ch ^ 1) share a
+// head and exchange tile maxima and row sums through shared memory.
 __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, float* red, uint32_t tmem,
                            uint32_t rank, int b, int split, int t_begin, int t_end, int n_tiles, bool direct,
                            volatile int* abort_flag) {
-  const int t = threadIdx.x;
-  const int lane = t & 31;
-  const int hl = t & 63;          // head within this CTA
-  const int half = t >> 6;        // token half / latent quarter
-  const uint32_t lane_base = static_cast<uint32_t>(32 * (t >> 5)) << 16;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ch = warp >> 2;
+  const int t = 32 * (warp & 3) + lane;   // TMEM lane
+  const int hl = t & 63;                  // head within this CTA
+  const int half = t >> 6;                // token half of a tile / latent quarter of O
+  const int me = ch * 128 + t;            // slot in the exchange arrays
+  const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
   float m_used = -INFINITY;
   float l_run = 0.f;
   bool ok = true;
@@ -251,33 +311,38 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
       break;
     }
     tc_fence_after();
-    float sc[64];
+    float sc[32];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
       uint32_t r[16];
-      tmem_ld16(tmem + lane_base + 64 * j + 16 * q, r);
+      tmem_ld16(tmem + lane_base + 64 * j + 32 * ch + 16 * q, r);
       tmem_ld_wait();
 #pragma unroll
       for (int e = 0; e < 16; ++e) sc[16 * q + e] = __uint_as_float(r[e]);
     }
-    const int tok0 = t_begin + i * kTcTile + 64 * half;
-    const int nvalid = min(max(t_end - tok0, 0), 64);
-    float mloc = -INFINITY;
+    // Tokens at or past the split end (only in a ragged last tile) get a score of -inf.
+    const int tok0 = t_begin + i * kTcTile + 64 * half + 32 * ch;
+    const int nvalid = t_end - tok0;
+    if (nvalid < 32) {
 #pragma unroll
-    for (int e = 0; e < 64; ++e) {
-      sc[e] = e < nvalid ? sc[e] * a.scale_log2 : -INFINITY;
-      mloc = fmaxf(mloc, sc[e]);
+      for (int e = 0; e < 32; ++e)
+        if (e >= nvalid) sc[e] = -INFINITY;
     }
-    red[j * 128 + t] = mloc;
-    named_bar_sync(1, 128);
-    const float m_tile = fmaxf(mloc, red[j * 128 + (t ^ 64)]);
+    float mloc = sc[0];
+#pragma unroll
+    for (int e = 1; e < 32; ++e) mloc = fmaxf(mloc, sc[e]);
+    mloc *= a.scale_log2;   // scale > 0, so the max commutes with the scaling
+    float* rm = red + j * 256;
+    rm[me] = mloc;
+    named_bar_sync(1, 256);
+    const float m_tile = fmaxf(fmaxf(mloc, rm[me ^ 64]), fmaxf(rm[me ^ 128], rm[me ^ 192]));
     float alpha = 1.f;
     bool need = false;
     if (m_used == -INFINITY) {
       m_used = m_tile;
       alpha = 0.f;
     } else if (m_tile > m_used + kTcRescaleThreshold) {
-      alpha = exp2f(m_used - m_tile);
+      alpha = ex2_approx(m_used - m_tile);
       m_used = m_tile;
       need = true;
     }
@@ -289,9 +354,9 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
         break;
       }
       tc_fence_after();
-      for (int q = 0; q < 16; ++q) {
+      for (int q = 0; q < 8; ++q) {
         uint32_t r[16];
-        const uint32_t addr = tmem + lane_base + 128 + 16 * q;
+        const uint32_t addr = tmem + lane_base + 128 + 128 * ch + 16 * q;
         tmem_ld16(addr, r);
         tmem_ld_wait();
 #pragma unroll
@@ -300,77 +365,79 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
       }
       tmem_st_wait();
     }
-    // P buffer j is free once PV(i-2) has read it.
-    if (i >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->p_empty[j], static_cast<uint32_t>((i - 2) >> 1) & 1u, 0x32))) {
+    // The P buffer is free once PV(i-1) has read it.  By parity this is unambiguous: s_full(i)
+    // was committed after PV(i-2), so p_empty is in phase i-1 or i.
+    if (i >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bars->p_empty, static_cast<uint32_t>(i - 1) & 1u, 0x32))) {
       ok = false;
       break;
     }
+    const float neg_m = -m_used;
     float psum = 0.f;
-    uint8_t* prow = smem + kTcOffP + j * kTcPBytes + half * kTcSlab + hl * 128;
+    uint8_t* prow = smem + kTcOffP + half * kTcSlab + hl * 128;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 4; ++u) {
       uint32_t pk[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float p0 = exp2f(sc[8 * u + 2 * e] - m_used);
-        const float p1 = exp2f(sc[8 * u + 2 * e + 1] - m_used);
+        const float p0 = ex2_approx(fmaf(sc[8 * u + 2 * e], a.scale_log2, neg_m));
+        const float p1 = ex2_approx(fmaf(sc[8 * u + 2 * e + 1], a.scale_log2, neg_m));
         psum += p0 + p1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[e] = *reinterpret_cast<uint32_t*>(&h2);
       }
-      *reinterpret_cast<uint4*>(prow + ((u ^ (hl & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      const int unit = 4 * ch + u;   // 16-byte unit (8 tokens) within the 128-byte row
+      *reinterpret_cast<uint4*>(prow + ((unit ^ (hl & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
     l_run = l_run * alpha + psum;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive_addr(lbar(&bars->p_full[j]));
+    if (lane == 0) mbar_arrive_addr(lbar(&bars->p_full));
   }
   // ---- epilogue
   if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0u, 0x33))) ok = false;
   tc_fence_after();
-  red[256 + t] = l_run;
-  named_bar_sync(1, 128);
-  const float l_tot = l_run + red[256 + (t ^ 64)];
+  float* rl = red + (n_tiles & 1) * 256;   // the maxima buffer the last tile did not use
+  rl[me] = l_run;
+  named_bar_sync(1, 256);
+  const float l_tot = (l_run + rl[me ^ 64]) + (rl[me ^ 128] + rl[me ^ 192]);
   if (!ok || *abort_flag) return;
   const int h = 64 * static_cast<int>(rank) + hl;
   const int64_t bh = static_cast<int64_t>(b) * kHeads + h;
+  const int lat0 = 256 * ch + 128 * half;
+  const uint32_t ocol = tmem + lane_base + 128 + 128 * ch;
   if (direct) {
     const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-    for (int nh = 0; nh < 2; ++nh) {
-      __nv_bfloat16* dst = a.out_lat + bh * kDLat + 256 * nh + 128 * half;
-      for (int q = 0; q < 8; ++q) {
-        uint32_t r[16];
-        tmem_ld16(tmem + lane_base + 128 + 128 * nh + 16 * q, r);
-        tmem_ld_wait();
-        uint32_t pk[8];
+    __nv_bfloat16* dst = a.out_lat + bh * kDLat + lat0;
+    for (int q = 0; q < 8; ++q) {
+      uint32_t r[16];
+      tmem_ld16(ocol + 16 * q, r);
+      tmem_ld_wait();
+      uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
-          pk[e] = *reinterpret_cast<uint32_t*>(&h2);
-        }
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * q);
-        d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      for (int e = 0; e < 8; ++e) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
+        pk[e] = *reinterpret_cast<uint32_t*>(&h2);
       }
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * q);
+      d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
-    if (half == 0 && a.lse != nullptr) a.lse[bh] = l_tot > 0.f ? (m_used + log2f(l_tot)) * kLn2 : -INFINITY;
+    if (half == 0 && ch == 0 && a.lse != nullptr) a.lse[bh] = l_tot > 0.f ? (m_used + log2f(l_tot)) * kLn2 : -INFINITY;
   } else {
     const int64_t ml = (static_cast<int64_t>(b) * a.S + split) * kHeads + h;
-    for (int nh = 0; nh < 2; ++nh) {
-      float* dst = a.ws.o + ml * kDLat + 256 * nh + 128 * half;
-      for (int q = 0; q < 8; ++q) {
-        uint32_t r[16];
-        tmem_ld16(tmem + lane_base + 128 + 128 * nh + 16 * q, r);
-        tmem_ld_wait();
-        float4* d4 = reinterpret_cast<float4*>(dst + 16 * q);
+    float* dst = a.ws.o + ml * kDLat + lat0;
+    for (int q = 0; q < 8; ++q) {
+      uint32_t r[16];
+      tmem_ld16(ocol + 16 * q, r);
+      tmem_ld_wait();
+      float4* d4 = reinterpret_cast<float4*>(dst + 16 * q);
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          d4[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
-                              __uint_as_float(r[4 * e + 3]));
-      }
+      for (int e = 0; e < 4; ++e)
+        d4[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
+                            __uint_as_float(r[4 * e + 3]));
     }
-    if (half == 0) {
+    if (half == 0 && ch == 0) {
       a.ws.m[ml] = m_used;
       a.ws.l[ml] = l_tot;
     }
@@ -379,16 +446,21 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
 
 // ------------------------------------------------------------------------------ kernel
 // grid = (2 * S, batch), clusters of 2 along x: blockIdx.x = 2 * split + rank.
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_vc,
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_q, const DecodeTcArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
   TcBars* bars = reinterpret_cast<TcBars*>(smem + kTcOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTcOffMisc);
   int* abort_flag = reinterpret_cast<int*>(smem + kTcOffMisc + 16);
-  float* red = reinterpret_cast<float*>(smem + kTcOffMisc + 64);   // [2][128] maxima + [128] sums
+  float* red = reinterpret_cast<float*>(smem + kTcOffMisc + 64);   // [2][256] tile maxima, reused for sums
 
+  // The 128-byte swizzle atoms need a 1024-byte aligned base; the layout above has no slack for
+  // realigning, so a misaligned base is reported instead of used (every CTA sees the same base).
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) set_dev_error(0x8);
+    return;
+  }
   const uint32_t rank = cluster_ctarank();
   const int split = blockIdx.x >> 1;
   const int b = blockIdx.y;
@@ -403,29 +475,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const bool direct = splits_used(L, a.S, kSplitAlign) == 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&bars->kv_full[s], 3);
-      mbar_init(&bars->kv_empty[s], 1);
+    for (int s = 0; s < kTcKSlots; ++s) {
+      mbar_init(&bars->k_full[s], 2);   // one arrival per CTA of the pair (plus the copies' bytes)
+      mbar_init(&bars->k_empty[s], 1);
     }
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(&bars->s_full[j], 1);
-      mbar_init(&bars->p_full[j], 8);
-      mbar_init(&bars->p_empty[j], 1);
+    for (int s = 0; s < kTcVSlots; ++s) {
+      mbar_init(&bars->v_full[s], 2);   // one arrival per CTA of the pair (plus the copies' bytes)
+      mbar_init(&bars->v_empty[s], 1);
     }
+    mbar_init(&bars->fix, 1);
+    mbar_init(&bars->s_full[0], 1);
+    mbar_init(&bars->s_full[1], 1);
+    mbar_init(&bars->p_full, 2 * kTcSoftmaxWarps);   // every softmax warp of both CTAs
+    mbar_init(&bars->p_empty, 1);
     mbar_init(&bars->o_ready, 1);
     mbar_init(&bars->o_final, 1);
     mbar_init(&bars->q_full, 2);
-    mbar_init(&bars->fix, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kTcMmaWarp) {
     tmem_alloc_pair(tmem_slot, 512);
     tmem_relinquish_pair();
   }
-  if (warp == 4 && (threadIdx.x & 31) == 0) {
-    tma_prefetch_desc(&tm_kc);
-    tma_prefetch_desc(&tm_vc);
+  if (warp == kTcProducerWarp && (threadIdx.x & 31) == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_q);
   }
   tc_fence_before();
@@ -433,11 +508,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
+  if (warp < kTcSoftmaxWarps) {
     tc_softmax(a, smem, bars, red, tmem, rank, b, split, t_begin, t_end, n_tiles, direct, abort_flag);
-  } else if (warp == 4) {
+  } else if (warp == kTcProducerWarp) {
     if ((threadIdx.x & 31) == 0 &&
-        !tc_producer(&tm_kc, &tm_vc, &tm_q, a, smem, bars, rank, b, t_begin, t_end, n_tiles, abort_flag))
+        !tc_producer(&tm_k, &tm_v, &tm_q, a, smem, bars, rank, b, t_begin, t_end, n_tiles, abort_flag))
       *abort_flag = 1;
   } else if (rank == 0 && (threadIdx.x & 31) == 0) {
     tc_mma(smem, bars, tmem, n_tiles, abort_flag);
@@ -447,7 +522,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   tc_fence_before();
   __syncwarp();
   cluster_sync();
-  if (warp == 5) {
+  if (warp == kTcMmaWarp) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, 512);
   }

@@ -68,6 +68,38 @@ bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
   return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 view of [rows][576] as (64-element dim-slab, row, slab index) for boxes of
+// 64 elements x 64 rows x kTcKBoxSlabs slabs, 128-byte swizzle: one box fills kTcKBoxSlabs
+// consecutive 8 KB slabs of 64 rows x 128 bytes.
+bool make_map_slabs(CUtensorMap* map, const void* base, uint64_t rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {64, rows, 9};
+  const cuuint64_t strides[2] = {mla::kDRow * 2, 128};
+  const cuuint32_t box[3] = {64, 64, mla::kTcKBoxSlabs};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 4-D bf16 view of [rows][576] as (64-element chunk, row, chunk index, latent half) for boxes of
+// 64 elements x 64 rows x 2 chunks x 2 halves (32 KB), 128-byte swizzle: the PV operand of one CTA
+// for 64 tokens, laid out [half][chunk][row][128 B].
+bool make_map_vbox(CUtensorMap* map, const void* base, uint64_t rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[4] = {64, rows, 4, 2};
+  const cuuint64_t strides[3] = {mla::kDRow * 2, 128, 512};
+  const cuuint32_t box[4] = {64, 64, 2, 2};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Validates a cache descriptor; on success fills the kernel-side view.
 mla_status check_cache(const mla_cache_desc& d, const void* cache, const int32_t* block_table, CacheView* v) {
   if (cache == nullptr || !aligned16(cache)) return MLA_ERR_INVALID_ARG;
@@ -107,7 +139,7 @@ int decode_cluster_slots() {
                            mla::kTcSmemBytes) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(192, 1, 1);
+    cfg.blockDim = dim3(mla::kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = mla::kTcSmemBytes;
     if (cudaOccupancyMaxActiveClusters(&n, mla::decode_tc_kernel, &cfg) != cudaSuccess) n = 0;
   }
@@ -232,26 +264,19 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
 int32_t mla_decode_num_splits(int32_t batch, int32_t max_seq_len, int32_t num_splits) {
   if (num_splits > 0) return num_splits > kMaxSplits ? kMaxSplits : num_splits;
   if (batch <= 0 || max_seq_len <= 0) return 1;
-  // Each (sequence, split) is one CTA pair.  Pick the split count whose pairs fill the resident
-  // pair slots best (fewest idle slots in the last wave), with at least two 128-token tiles per
-  // split; ties go to fewer splits (less partial traffic).
+  // Each (sequence, split) is one CTA pair, and every extra split costs an fp32 partial of
+  // 128 x 514 floats written and read back (about 460 cached tokens' worth of traffic).  Use the
+  // fewest splits whose pairs cover at least 80 % of the resident pair slots, keeping at least
+  // two 128-token tiles per split.
   const int slots = decode_cluster_slots();
   int s_max = (max_seq_len + 2 * mla::kTcTile - 1) / (2 * mla::kTcTile);
   if (s_max < 1) s_max = 1;
   if (s_max > kMaxSplits) s_max = kMaxSplits;
-  int best = 1;
-  double best_eff = -1.0;
-  for (int s = 1; s <= s_max; ++s) {
-    const long long units = static_cast<long long>(batch) * s;
-    const long long waves = (units + slots - 1) / slots;
-    const double eff = static_cast<double>(units) / static_cast<double>(waves * slots);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = s;
-    }
-    if (units >= 4LL * slots) break;
-  }
-  return best;
+  const long long want = (4LL * slots + 4) / 5;
+  int s = static_cast<int>((want + batch - 1) / batch);
+  if (s < 1) s = 1;
+  if (s > s_max) s = s_max;
+  return s;
 }
 
 size_t mla_decode_workspace_size(int32_t batch, int32_t max_seq_len, int32_t num_splits) {
@@ -288,15 +313,14 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
   a.ws = mla::ws_carve(workspace, batch, S);
   a.out_lat = reinterpret_cast<__nv_bfloat16*>(out_lat);
   a.lse = lse;
-  CUtensorMap tkc, tvc, tq;
-  if (!make_map_2d(&tkc, cache, mla::kDRow, desc.num_rows, mla::kDRow * 2, 64, 64) ||
-      !make_map_2d(&tvc, cache, mla::kDRow, desc.num_rows, mla::kDRow * 2, 64, 32) ||
-      !make_map_2d(&tq, q_full, mla::kDRow, static_cast<uint64_t>(batch) * mla::kHeads, mla::kDRow * 2, 64, 64))
+  CUtensorMap tk, tv, tq;
+  if (!make_map_slabs(&tk, cache, desc.num_rows) || !make_map_vbox(&tv, cache, desc.num_rows) ||
+      !make_map_slabs(&tq, q_full, static_cast<uint64_t>(batch) * mla::kHeads))
     return MLA_ERR_CUDA;
   if (cudaFuncSetAttribute(mla::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kTcSmemBytes) !=
       cudaSuccess)
     return MLA_ERR_CUDA;
-  mla::decode_tc_kernel<<<dim3(2 * S, batch), 192, mla::kTcSmemBytes, s>>>(tkc, tvc, tq, a);
+  mla::decode_tc_kernel<<<dim3(2 * S, batch), mla::kTcThreads, mla::kTcSmemBytes, s>>>(tk, tv, tq, a);
   mla_status ls = launch_status();
   if (ls != MLA_OK) return ls;
   mla::combine_kernel<<<dim3(batch, mla::kHeads / 4), 128, 0, s>>>(

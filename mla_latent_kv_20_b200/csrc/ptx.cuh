@@ -204,6 +204,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_addr(uint32_t bar_cluster_
                "r"(bytes)
                : "memory");
 }
+// Count-only arrivals (relaxed): for producers whose data is delivered by TMA complete_tx, so no
+// prior memory operation of the arriving thread needs to be ordered before the arrival.
+__device__ __forceinline__ void mbar_arrive_expect_tx_relaxed(uint32_t bar_cluster_addr, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar_cluster_addr),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_addr(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
