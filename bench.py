@@ -268,6 +268,22 @@ def run_step(st, i, ev=None):
         m.unabsorb_v(st["out_lat"], layer["w_uv"], st["out"])
 
 
+def reduce_max_over_ranks(values, world, device=None):
+    """Element-wise max of per-rank timings across the process group (the slowest rank defines
+    the job's time).  CPU tensors under gloo, CUDA tensors under nccl."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(bytes_per_rank, world, ms):
+    """Whole-job GB/s: the units every rank processed divided by the max-over-ranks time."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 def hz_bits(t):
     from mla_latent_kv_20_b200 import harness as hz
     return hz.bf16_bits(t)
@@ -343,16 +359,13 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
-    t = torch.tensor([ms, e2e_ms, dec_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms, dec_ms = t.tolist()
+    ms, e2e_ms, dec_ms = reduce_max_over_ranks([ms, e2e_ms, dec_ms], world, device=dev)
     if rank != 0:
         return
     tokens, cache_bytes, flops, dec_bytes = step_work(st["lens"])
     tokens, cache_bytes, flops = tokens * n_layers, cache_bytes * n_layers, flops * n_layers
     hbm, tc, tc_sus, peak_kind = load_peaks()
-    value = world * cache_bytes / (ms * 1e-3) / 1e9
+    value = job_throughput(cache_bytes, world, ms)
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     roofline_s = max(cache_bytes / (hbm * 1e9), flops / (tc * 1e12))
     line = {
@@ -375,7 +388,7 @@ def run_ours(args, rank, world, local_rank):
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_kind": peak_kind, "traffic": None, "avg_launch_ms": dec_ms,
                      "algorithmic_bytes_per_launch": dec_bytes},
-        "e2e": {"value": world * cache_bytes / (e2e_ms * 1e-3) / 1e9, "unit": UNIT,
+        "e2e": {"value": job_throughput(cache_bytes, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": LAUNCHES_PER_LAYER * n_layers * args.steps,
         "clocks": clocks,

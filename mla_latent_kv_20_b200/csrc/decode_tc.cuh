@@ -39,9 +39,9 @@ namespace mla {
 
 constexpr int kTcTile = 128;                 // tokens per tile
 constexpr int kTcSlab = 8192;                // 64 rows x 128 bytes
-constexpr int kTcKBoxSlabs = 3;              // dim-slabs per K TMA box
+constexpr int kTcKBoxSlabs = 9;              // dim-slabs per K TMA box (the whole 576-wide row)
 constexpr int kTcKBoxes = 9 / kTcKBoxSlabs;  // K boxes per tile
-constexpr int kTcKSlots = 3;
+constexpr int kTcKSlots = 1;
 constexpr int kTcVSlots = 2;
 constexpr int kTcVBox = 4 * kTcSlab;         // 64 tokens x 2 chunks x 2 latent halves
 constexpr int kTcQBytes = 9 * kTcSlab;
