@@ -247,6 +247,30 @@ def setup_replica(name, device):
     return st
 
 
+# DRAM bytes (read + write) of one mla_decode_attn call (decode kernel + combine kernel), from one
+# ncu capture per workload, keyed by the SHA-256 of the sources that build those kernels and
+# choose their launch shape.  A digest that no longer matches means the kernels changed since the
+# counters were taken, and the traffic is reported as null.
+TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh", "csrc/mla_lib.cu")
+MEASURED_TRAFFIC = {}   # workload -> {"bytes": int, "sha256": str, "profile": str}
+
+
+def traffic_sources_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, "mla_latent_kv_20_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload):
+    rec = MEASURED_TRAFFIC.get(workload)
+    if rec is None or rec["sha256"] != traffic_sources_digest():
+        return None
+    return rec["bytes"]
+
+
 LAUNCHES_PER_LAYER = 6   # append, absorb GEMM, q_pe rotation, decode split, combine, un-absorb GEMM
 
 
@@ -386,7 +410,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline_step_frac": roofline_s / (ms * 1e-3),
         "roofline": {"kernel": "mla_decode_attn (split-KV decode + combine)", "bound": "hbm",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_kind": peak_kind, "traffic": None, "avg_launch_ms": dec_ms,
+                     "peak_kind": peak_kind, "traffic": recorded_traffic(args.workload), "avg_launch_ms": dec_ms,
                      "algorithmic_bytes_per_launch": dec_bytes},
         "e2e": {"value": job_throughput(cache_bytes, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

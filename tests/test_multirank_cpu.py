@@ -56,3 +56,15 @@ def test_single_rank_is_identity():
     import bench
     assert bench.reduce_max_over_ranks([3.0, 4.0], 1) == [3.0, 4.0]
     assert bench.job_throughput(2e9, 1, 1.0) == pytest.approx(2000.0)
+
+
+def test_recorded_traffic_follows_kernel_sources(monkeypatch):
+    """A traffic figure is reported only while the kernel sources match the digest it was
+    recorded with."""
+    import bench
+    digest = bench.traffic_sources_digest()
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", {"w": {"bytes": 123, "sha256": digest, "profile": "p"}})
+    assert bench.recorded_traffic("w") == 123
+    assert bench.recorded_traffic("other") is None
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", {"w": {"bytes": 123, "sha256": "0" * 64, "profile": "p"}})
+    assert bench.recorded_traffic("w") is None
