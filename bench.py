@@ -274,22 +274,32 @@ def recorded_traffic(workload):
 LAUNCHES_PER_LAYER = 6   # append, absorb GEMM, q_pe rotation, decode split, combine, un-absorb GEMM
 
 
+PHASES = ("append", "absorb_q", "decode_attn", "unabsorb_v")
+
+
 def run_step(st, i, ev=None):
-    """One decode step over every layer of the workload."""
+    """One decode step over every layer of the workload.  With `ev`, events ev[layer][k] bracket
+    the phases: k and k + 1 around PHASES[k]."""
     import mla_latent_kv_20_b200 as m
     for li, layer in enumerate(st["layers"]):
         cache = layer["caches"][i % len(layer["caches"])]
         d = layer["dev"]
-        m.cache_append(d["c_new"], d["kr_new"], st["pos"], cache.data, cache.desc, seq_ids=st["seq_ids"],
-                       block_table=cache.block_table)
-        m.absorb_q(d["q_nope"], d["q_pe"], layer["w_uk"], st["q_full"], q_pos=st["pos"])
         if ev is not None:
             ev[li][0].record()
+        m.cache_append(d["c_new"], d["kr_new"], st["pos"], cache.data, cache.desc, seq_ids=st["seq_ids"],
+                       block_table=cache.block_table)
+        if ev is not None:
+            ev[li][1].record()
+        m.absorb_q(d["q_nope"], d["q_pe"], layer["w_uk"], st["q_full"], q_pos=st["pos"])
+        if ev is not None:
+            ev[li][2].record()
         m.decode_attn(st["q_full"], cache.data, cache.seq_lens, cache.desc, st["workspace"], st["out_lat"],
                       lse=st["lse"], block_table=cache.block_table, num_splits=st["splits"])
         if ev is not None:
-            ev[li][1].record()
+            ev[li][3].record()
         m.unabsorb_v(st["out_lat"], layer["w_uv"], st["out"])
+        if ev is not None:
+            ev[li][4].record()
 
 
 def reduce_max_over_ranks(values, world, device=None):
@@ -331,7 +341,7 @@ def run_ours(args, rank, world, local_rank):
         run_step(st, i)
     torch.cuda.synchronize()
     n_layers = len(st["layers"])
-    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_layers)]
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(len(PHASES) + 1)] for _ in range(n_layers)]
            for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
@@ -340,14 +350,18 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize()
     t_start.record()
+    h0 = time.perf_counter()
     for i in range(args.steps):
         run_step(st, i, evs[i])
+    host_ms = (time.perf_counter() - h0) * 1e3 / args.steps
     t_end.record()
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     ms = t_start.elapsed_time(t_end) / args.steps
-    dec_ms = sum(a.elapsed_time(b) for step in evs for a, b in step) / (args.steps * n_layers)
+    phase_ms = {p: sum(lev[k].elapsed_time(lev[k + 1]) for step in evs for lev in step) / (args.steps * n_layers)
+                for k, p in enumerate(PHASES)}
+    dec_ms = phase_ms["decode_attn"]
     assert m.get_device_error() == 0
 
     # end to end through the public API with host buffers: H2D of the step's inputs (every layer's
@@ -407,6 +421,8 @@ def run_ours(args, rank, world, local_rank):
         "tflops": world * flops / (ms * 1e-3) / 1e12,
         "tokens_per_s": world * st["B"] / (ms * 1e-3),
         "decode_layer_ms": dec_ms,
+        "phase_ms_per_layer": phase_ms,
+        "host_issue_ms_per_step": host_ms,
         "roofline_step_frac": roofline_s / (ms * 1e-3),
         "roofline": {"kernel": "mla_decode_attn (split-KV decode + combine)", "bound": "hbm",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,

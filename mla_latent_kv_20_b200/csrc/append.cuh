@@ -47,32 +47,29 @@ __device__ __forceinline__ int64_t cache_row(const CacheView& v, int seq, int t)
   return r;
 }
 
-// Rotate 4 interleaved pairs (8 values starting at element 8*chunk of the 64-wide branch).
-__device__ __forceinline__ uint4 rope8(uint4 raw, int chunk, int pos, double base) {
-  const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(&raw);
-  uint4 res;
-  __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(&res);
-#pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const int i = chunk * 4 + p;  // pair index 0..31
-    const double theta = pow(base, -2.0 * static_cast<double>(i) / static_cast<double>(kDRope));
-    double s, c;
-    sincos(static_cast<double>(pos) * theta, &s, &c);
-    const double xe = static_cast<double>(__bfloat162float(x[2 * p]));
-    const double xo = static_cast<double>(__bfloat162float(x[2 * p + 1]));
-    y[2 * p] = __double2bfloat16(xe * c - xo * s);
-    y[2 * p + 1] = __double2bfloat16(xe * s + xo * c);
-  }
-  return res;
+// Inverse frequencies base^(-2i/64) of the 32 rotation pairs, formed once on the host in fp64.
+struct RopeFreq {
+  double inv_freq[kDRope / 2];
+};
+
+// Rotate one interleaved pair (x_{2i}, x_{2i+1}) by pos * inv_freq[i]: the angle and the rotation
+// in fp64, one rounding to bf16 per output.
+__device__ __forceinline__ __nv_bfloat162 rope_pair(__nv_bfloat162 x, double c, double s) {
+  const double xe = static_cast<double>(__low2float(x));
+  const double xo = static_cast<double>(__high2float(x));
+  __nv_bfloat162 y;
+  y.x = __double2bfloat16(xe * c - xo * s);
+  y.y = __double2bfloat16(xe * s + xo * c);
+  return y;
 }
 
-// One CTA of 72 threads per new token: threads 0..63 copy the latent (16 B each), threads
-// 64..71 rotate and write the 64-wide key (4 pairs each).
-__global__ void __launch_bounds__(72) cache_append_kernel(const uint4* __restrict__ c_new,
-                                                          const uint4* __restrict__ kr_new,
+// One CTA of 96 threads per new token: threads 0..63 copy the latent (16 B each), threads
+// 64..95 rotate one pair of the 64-wide key each (one fp64 sincos per thread, all in parallel).
+__global__ void __launch_bounds__(96) cache_append_kernel(const uint4* __restrict__ c_new,
+                                                          const __nv_bfloat162* __restrict__ kr_new,
                                                           const int32_t* __restrict__ seq_ids,
                                                           const int32_t* __restrict__ pos, uint4* cache,
-                                                          CacheView v, double rope_base) {
+                                                          CacheView v, RopeFreq f) {
   const int i = blockIdx.x;
   const int seq = seq_ids ? seq_ids[i] : i;
   const int p = pos[i];
@@ -83,25 +80,42 @@ __global__ void __launch_bounds__(72) cache_append_kernel(const uint4* __restric
   }
   const int64_t row = cache_row(v, seq, p);
   if (row < 0) return;
-  uint4* dst = cache + row * (kDRow / 8);
   const int t = threadIdx.x;
   if (t < 64) {
+    uint4* dst = cache + row * (kDRow / 8);
     dst[t] = c_new[static_cast<int64_t>(i) * (kDLat / 8) + t];
   } else {
-    const int ch = t - 64;
-    dst[64 + ch] = rope8(kr_new[static_cast<int64_t>(i) * (kDRope / 8) + ch], ch, p, rope_base);
+    const int pr = t - 64;   // pair index 0..31
+    double sn, cs;
+    sincos(static_cast<double>(p) * f.inv_freq[pr], &sn, &cs);
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(cache + row * (kDRow / 8) + kDLat / 8);
+    dst[pr] = rope_pair(kr_new[static_cast<int64_t>(i) * (kDRope / 2) + pr], cs, sn);
   }
 }
 
 // q_full[b, h, 512:576] = q_pe[b, h, :] rotated at q_pos[b] (or copied when q_pos is NULL).
-// grid = batch, block = 128 x 8 threads: one 16-byte chunk of one head per thread.
+// grid = batch, block = 128 heads x 8 threads: the 32 angles of the sequence's position are formed
+// once (threads 0..31) and shared through shared memory; each thread then rotates 4 pairs of one
+// head.
 __global__ void __launch_bounds__(1024) qpe_kernel(const uint4* __restrict__ q_pe, const int32_t* __restrict__ q_pos,
-                                                   uint4* __restrict__ q_full, double rope_base) {
+                                                   uint4* __restrict__ q_full, RopeFreq f) {
+  __shared__ double cs_sn[kDRope / 2][2];
   const int b = blockIdx.x;
   const int h = threadIdx.x >> 3;
   const int ch = threadIdx.x & 7;
-  const uint4 raw = q_pe[(static_cast<int64_t>(b) * kHeads + h) * (kDRope / 8) + ch];
-  const uint4 r = q_pos ? rope8(raw, ch, q_pos[b], rope_base) : raw;
+  if (q_pos != nullptr && threadIdx.x < kDRope / 2) {
+    double sn, cs;
+    sincos(static_cast<double>(q_pos[b]) * f.inv_freq[threadIdx.x], &sn, &cs);
+    cs_sn[threadIdx.x][0] = cs;
+    cs_sn[threadIdx.x][1] = sn;
+  }
+  __syncthreads();
+  uint4 r = q_pe[(static_cast<int64_t>(b) * kHeads + h) * (kDRope / 8) + ch];
+  if (q_pos != nullptr) {
+    __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] = rope_pair(x[k], cs_sn[4 * ch + k][0], cs_sn[4 * ch + k][1]);
+  }
   q_full[(static_cast<int64_t>(b) * kHeads + h) * (kDRow / 8) + kDLat / 8 + ch] = r;
 }
 

@@ -10,7 +10,8 @@
 // B200 mapping.  The two CTAs of a cluster run "pair" MMAs (tcgen05 cta_group::2, M = 128): CTA r
 // owns heads [64r, 64r+64) (its half of the A operand: Q for QK^T, P for PV) and each CTA's TMEM
 // receives a 64-head slice of the accumulator folded over all 128 lanes, so
-//   S tile (64 heads x 128 tokens, fp32)  = 64 TMEM columns per CTA (two buffers),
+//   S tile (64 heads x 128 tokens, fp32)  = 64 TMEM columns per CTA (two buffers, and two
+//                                           partial sums over disjoint dims: 256 columns),
 //   O      (64 heads x 512 latent, fp32)  = 256 TMEM columns per CTA.
 // Per 128-token tile the B operand of QK^T is split by tokens: CTA r holds tokens [64r, 64r+64)
 // with all 576 dims, as 9 swizzled slabs of 64 dims.  The B operand of PV is split by latent
@@ -18,17 +19,19 @@
 // second read of the tile's rows that hits L2 because the pair reads them within microseconds.
 //
 // Staging.  The TMA unit of a CTA works through its tensor copies one at a time at a roughly
-// fixed cost per copy (measured: ~0.35 us for anything from 8 KB to 72 KB), so every copy is
-// large: K rows (from HBM) come as 3-D boxes of 3 dim-slabs (24 KB, 3 copies per tile) into a
-// 3-slot K ring, and V rows (the L2 re-read) as 4-D boxes of 64 tokens x both 64-wide latent
-// chunks x both latent halves (32 KB, 2 copies per tile) into a 2-slot V ring.  Separate rings let
-// the K copies of the next tile proceed while V of the current tile waits for its softmax.
+// fixed cost per copy (measured: ~0.35 us for anything from 8 KB to 72 KB from L2), so every copy
+// is large: a CTA's K rows of a tile (from HBM) come as one 3-D box of all 9 dim-slabs (72 KB),
+// and V rows (the L2 re-read) as 4-D boxes of 64 tokens x both 64-wide latent chunks x both
+// latent halves (32 KB, 2 copies per tile) into a 2-slot V ring.  K tiles a few steps ahead are
+// pulled into L2 with bulk prefetches.  Separate K and V buffers let the K copy of the next tile
+// proceed while V of the current tile waits for its softmax.
 // V rows past the split end are zeroed in shared memory before PV (rows past a sequence's end may
 // hold anything, and 0 * NaN would poison the sum).
 //
-// Warp roles (320 threads): warps 0-7 softmax / O correction / epilogue (two warps per TMEM lane
-// quadrant, each owning half of the S columns), warp 8 TMA producer, warp 9 TMEM allocation and
-// (even CTA only) MMA issue.
+// Warp roles (416 threads): warps 0-7 softmax / O correction / epilogue (two warps per TMEM lane
+// quadrant, each owning half of the S columns), warp 8 TMA producer and L2 prefetcher, and in the
+// even CTA only: warp 9 QK^T part A (warp 9 also allocates TMEM in both CTAs), warp 11 QK^T part
+// B, warps 10 and 12 PV for the two latent halves.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -39,10 +42,14 @@ namespace mla {
 
 constexpr int kTcTile = 128;                 // tokens per tile
 constexpr int kTcSlab = 8192;                // 64 rows x 128 bytes
-constexpr int kTcKBoxSlabs = 9;              // dim-slabs per K TMA box (the whole 576-wide row)
-constexpr int kTcKBoxes = 9 / kTcKBoxSlabs;  // K boxes per tile
-constexpr int kTcKSlots = 1;
+// QK^T of a tile is split along the 576 dims into two parts with their own K slot, issuing warp
+// and S accumulator (the softmax adds the two): part A = dim-slabs [0, 5), part B = [5, 9).
+constexpr int kTcKSlabsA = 5;
+constexpr int kTcKSlabsB = 4;
+__host__ __device__ constexpr int tc_part_slab0(int part) { return part ? kTcKSlabsA : 0; }
+__host__ __device__ constexpr int tc_part_slabs(int part) { return part ? kTcKSlabsB : kTcKSlabsA; }
 constexpr int kTcVSlots = 2;
+constexpr int kTcPrefetchTiles = 4;          // K tiles pulled into L2 ahead of their load
 constexpr int kTcVBox = 4 * kTcSlab;         // 64 tokens x 2 chunks x 2 latent halves
 constexpr int kTcQBytes = 9 * kTcSlab;
 constexpr int kTcPBytes = 2 * kTcSlab;       // 64 heads x 128 tokens bf16, two 64-token K chunks
@@ -50,19 +57,28 @@ constexpr float kTcRescaleThreshold = 8.0f;  // log2 units: rescale O only when 
 
 constexpr int kTcOffQ = 0;
 constexpr int kTcOffP = kTcOffQ + kTcQBytes;
-constexpr int kTcOffK = kTcOffP + kTcPBytes;
-constexpr int kTcOffV = kTcOffK + kTcKSlots * kTcKBoxSlabs * kTcSlab;
+constexpr int kTcOffK = kTcOffP + kTcPBytes;  // slot of part A, then slot of part B: 9 slabs in dim order
+constexpr int kTcOffV = kTcOffK + 9 * kTcSlab;
 constexpr int kTcOffBar = kTcOffV + kTcVSlots * kTcVBox;
 constexpr int kTcOffMisc = kTcOffBar + 256;
 constexpr int kTcSmemBytes = kTcOffMisc + 64 + 2 * 256 * 4;   // the dynamic base is 1024-aligned (checked)
 
+// TMEM columns of each CTA (512 allocated): S part A (2 buffers x 64), S part B (2 x 64), O (256).
+constexpr uint32_t kTcColSA = 0;
+constexpr uint32_t kTcColSB = 128;
+constexpr uint32_t kTcColO = 256;
+
 constexpr int kTcSoftmaxWarps = 8;
 constexpr int kTcProducerWarp = 8;
-constexpr int kTcMmaWarp = 9;
-constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 2);
+constexpr int kTcMmaWarp = 9;     // TMEM allocation (both CTAs); QK^T part A issue (even CTA)
+constexpr int kTcPvWarp = 10;     // PV issue, first latent half (even CTA)
+constexpr int kTcMmaBWarp = 11;   // QK^T part B issue (even CTA)
+constexpr int kTcPv1Warp = 12;    // PV issue, second latent half (even CTA)
+constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 5);
 
 struct DecodeTcArgs {
   CacheView v;
+  const uint8_t* cache;   // cache rows (for L2 prefetches)
   const int32_t* seq_lens;
   int S;               // splits per sequence
   float scale_log2;    // softmax_scale * log2(e)
@@ -72,16 +88,17 @@ struct DecodeTcArgs {
 };
 
 struct TcBars {
-  uint64_t k_full[kTcKSlots];    // even CTA only: both CTAs' K boxes landed (one arrival per CTA + tx)
-  uint64_t k_empty[kTcKSlots];   // both CTAs: K box consumed by the MMAs
+  uint64_t k_full[2];            // even CTA only, per QK^T part: both CTAs' K boxes landed (one arrival per CTA + tx)
+  uint64_t k_empty[2];           // both CTAs, per part: K box consumed by the MMAs
   uint64_t v_full[kTcVSlots];    // even CTA only: both CTAs' V box landed (one arrival per CTA + tx)
-  uint64_t v_empty[kTcVSlots];   // both CTAs: V box consumed
+  uint64_t v_empty[kTcVSlots];   // both CTAs: V box consumed (one commit per PV warp)
   uint64_t fix;                  // per CTA: local load of a ragged V box
-  uint64_t s_full[2];            // both: QK^T of a tile done
+  uint64_t s_full[2];            // both: QK^T of a tile done (one commit per part)
+  uint64_t s_empty[2];           // even CTA only: every softmax warp of both CTAs has read S
   uint64_t p_full;               // even CTA only: P (and corrected O) of a tile ready in both CTAs
-  uint64_t p_empty;              // both: PV of a tile done reading P
-  uint64_t o_ready;              // both: PV of a tile done writing O (one phase per tile)
-  uint64_t o_final;              // both: the last PV done (single phase, read by the epilogue)
+  uint64_t p_empty;              // both: PV of a tile done reading P (one commit per PV warp)
+  uint64_t o_ready;              // both: PV of a tile done writing O (one phase per tile, two commits)
+  uint64_t o_final;              // both: the last PV done (single phase, two commits)
   uint64_t q_full;               // even CTA only: Q of both CTAs landed
 };
 static_assert(sizeof(TcBars) <= 256, "barrier block");
@@ -126,11 +143,12 @@ __device__ __forceinline__ void tma_load_4d_local(void* dst, const CUtensorMap* 
 }
 
 // ------------------------------------------------------------------------------ TMA producer
-// Issue order K(0), K(1), V(0), K(2), V(1), ..., V(n-1): the order the MMA issuer consumes them,
-// with K one tile ahead so QK^T of tile i+1 never waits behind V of tile i.
-//  K(i): CTA r's 64 tokens [tile0 + 64r, +64) x 576 dims as kTcKBoxes boxes of kTcKBoxSlabs
-//        dim-slabs.  A half-tile past the split end is loaded from a negative row (zeros); its
-//        scores are masked anyway.
+// One warp.  Lane 0 issues the copies, in the order K(0), K(1), V(0), K(2), V(1), ..., V(n-1):
+// K one tile ahead, so QK^T of tile i+1 never waits behind V of tile i.  All lanes pull the K
+// rows of the tile kTcPrefetchTiles ahead into L2 with plain prefetches, so each K copy reads L2.
+//  K(i): CTA r's 64 tokens [tile0 + 64r, +64) x 576 dims as two boxes, one per QK^T part
+//        (5 and 4 dim-slabs).  A half-tile past the split end is loaded from a negative row
+//        (zeros); its scores are masked anyway.
 //  V(i): per 64-token half h of the tile, latent [256n + 128r, +128) for n = 0, 1 in one box,
 //        laid out [n][chunk][64 rows][128 B].
 __device__ __forceinline__ void zero_v_rows(uint8_t* box, int v) {
@@ -142,140 +160,207 @@ __device__ __forceinline__ void zero_v_rows(uint8_t* box, int v) {
     }
 }
 
-__device__ bool tc_producer(const CUtensorMap* tm_k, const CUtensorMap* tm_v, const CUtensorMap* tm_q,
-                            const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, uint32_t rank, int b, int t_begin,
-                            int t_end, int n_tiles, volatile int* abort_flag) {
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
+__device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, const CUtensorMap* tm_v,
+                            const CUtensorMap* tm_q, const DecodeTcArgs& a, uint8_t* smem, TcBars* bars,
+                            uint32_t rank, int b, int t_begin, int t_end, int n_tiles, volatile int* abort_flag) {
+  const int lane = threadIdx.x & 31;
+  const bool l0 = lane == 0;
   const bool leader = rank == 0;
-  // Q: 3 boxes of 3 dim-slabs x 64 heads.  Arrivals on the even CTA's barriers that only count
-  // (the data and its visibility come with the TMA's complete_tx) are relaxed.
-  for (int kb = 0; kb < kTcKBoxes; ++kb)
-    tma_load_3d_pair(smem + kTcOffQ + kb * kTcKBoxSlabs * kTcSlab, tm_q, lbar(&bars->q_full), 0,
-                     b * kHeads + 64 * static_cast<int>(rank), kb * kTcKBoxSlabs);
-  if (leader)
-    mbar_arrive_expect_tx_relaxed(lbar(&bars->q_full), 2u * kTcQBytes);
-  else
-    mbar_arrive_relaxed(lbar(&bars->q_full));
-  int kn = 0, vn = 0;
+  // Arrivals on the even CTA's barriers that only count (the data and its visibility come with
+  // the TMA's complete_tx) are relaxed.
+  if (l0) {
+    tma_load_3d_pair(smem + kTcOffQ, tm_q, lbar(&bars->q_full), 0, b * kHeads + 64 * static_cast<int>(rank), 0);
+    if (leader)
+      mbar_arrive_expect_tx_relaxed(lbar(&bars->q_full), 2u * kTcQBytes);
+    else
+      mbar_arrive_relaxed(lbar(&bars->q_full));
+  }
+  // Lane 0 waits; the verdict (and an abort seen meanwhile) is shared with the warp.
+  auto wait0 = [&](uint64_t* bar, uint32_t parity, uint32_t site) -> bool {
+    int ok = 1;
+    if (l0) ok = (mbar_wait(bar, parity, site) && !*abort_flag) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
+  auto prefetch_k = [&](int j) {
+    const int my0 = t_begin + j * kTcTile + 64 * static_cast<int>(rank);
+    if (j >= n_tiles || my0 >= t_end) return;
+    const int64_t row = cache_row(a.v, b, my0);
+    if (row < 0) return;
+    const int64_t nrows = a.v.num_rows - row < 64 ? a.v.num_rows - row : 64;
+    const uint8_t* base = a.cache + row * (kDRow * 2);
+    const int lines = static_cast<int>(nrows) * (kDRow * 2 / 128);
+    for (int q = lane; q < lines; q += 32) prefetch_l2(base + q * 128);
+  };
+  int vn = 0;
   uint32_t fix_phase = 0;
   auto issue_k = [&](int i) -> bool {
+    if (i > 0) prefetch_k(i + kTcPrefetchTiles);
     const int my0 = t_begin + i * kTcTile + 64 * static_cast<int>(rank);
     const int y = my0 < t_end ? tma_row(a.v, b, my0) : -kTcTile;
-    for (int kb = 0; kb < kTcKBoxes; ++kb, ++kn) {
-      const int s = kn % kTcKSlots;
-      if (kn >= kTcKSlots && !mbar_wait(&bars->k_empty[s], static_cast<uint32_t>((kn / kTcKSlots) - 1) & 1u, 0x10))
-        return false;
-      if (*abort_flag) return false;
-      tma_load_3d_pair(smem + kTcOffK + s * kTcKBoxSlabs * kTcSlab, tm_k, lbar(&bars->k_full[s]), 0, y,
-                       kb * kTcKBoxSlabs);
-      if (leader)
-        mbar_arrive_expect_tx_relaxed(lbar(&bars->k_full[s]), 2u * kTcKBoxSlabs * kTcSlab);
-      else
-        mbar_arrive_relaxed(lbar(&bars->k_full[s]));
+    for (int part = 0; part < 2; ++part) {
+      if (i >= 1 && !wait0(&bars->k_empty[part], static_cast<uint32_t>(i - 1) & 1u, 0x10 + part)) return false;
+      if (l0) {
+        tma_load_3d_pair(smem + kTcOffK + tc_part_slab0(part) * kTcSlab, part ? tm_kb : tm_ka,
+                         lbar(&bars->k_full[part]), 0, y, tc_part_slab0(part));
+        if (leader)
+          mbar_arrive_expect_tx_relaxed(lbar(&bars->k_full[part]), 2u * tc_part_slabs(part) * kTcSlab);
+        else
+          mbar_arrive_relaxed(lbar(&bars->k_full[part]));
+      }
     }
     return true;
   };
   auto issue_v = [&](int i) -> bool {
     for (int h = 0; h < 2; ++h, ++vn) {
       const int s = vn % kTcVSlots;
-      if (vn >= kTcVSlots && !mbar_wait(&bars->v_empty[s], static_cast<uint32_t>((vn / kTcVSlots) - 1) & 1u, 0x11))
+      if (vn >= kTcVSlots && !wait0(&bars->v_empty[s], static_cast<uint32_t>((vn / kTcVSlots) - 1) & 1u, 0x12))
         return false;
-      if (*abort_flag) return false;
       uint8_t* box = smem + kTcOffV + s * kTcVBox;
       const int tok0 = t_begin + i * kTcTile + 64 * h;
       const int vcount = min(max(t_end - tok0, 0), 64);
       if (vcount == 64) {
-        tma_load_4d_pair(box, tm_v, lbar(&bars->v_full[s]), 0, tma_row(a.v, b, tok0), 2 * static_cast<int>(rank), 0);
-        if (leader)
-          mbar_arrive_expect_tx_relaxed(lbar(&bars->v_full[s]), 2u * kTcVBox);
-        else
-          mbar_arrive_relaxed(lbar(&bars->v_full[s]));
+        if (l0) {
+          tma_load_4d_pair(box, tm_v, lbar(&bars->v_full[s]), 0, tma_row(a.v, b, tok0), 2 * static_cast<int>(rank), 0);
+          if (leader)
+            mbar_arrive_expect_tx_relaxed(lbar(&bars->v_full[s]), 2u * kTcVBox);
+          else
+            mbar_arrive_relaxed(lbar(&bars->v_full[s]));
+        }
       } else {
         // Ragged: load through a CTA-local barrier, zero the rows past the end, then publish with
-        // release semantics (the zeros are this thread's own shared-memory writes).
+        // release semantics (the zeros are lane 0's own shared-memory writes).
         if (vcount > 0) {
-          mbar_arrive_expect_tx(&bars->fix, kTcVBox);
-          tma_load_4d_local(box, tm_v, &bars->fix, 0, tma_row(a.v, b, tok0), 2 * static_cast<int>(rank), 0);
-          if (!mbar_wait(&bars->fix, fix_phase, 0x13)) return false;
+          if (l0) {
+            mbar_arrive_expect_tx(&bars->fix, kTcVBox);
+            tma_load_4d_local(box, tm_v, &bars->fix, 0, tma_row(a.v, b, tok0), 2 * static_cast<int>(rank), 0);
+          }
+          if (!wait0(&bars->fix, fix_phase, 0x13)) return false;
           fix_phase ^= 1u;
         }
-        zero_v_rows(box, vcount);
-        fence_proxy_async_smem();
-        if (leader)
-          mbar_arrive_expect_tx_addr(lbar(&bars->v_full[s]), 0u);
-        else
-          mbar_arrive_addr(lbar(&bars->v_full[s]));
+        if (l0) {
+          zero_v_rows(box, vcount);
+          fence_proxy_async_smem();
+          if (leader)
+            mbar_arrive_expect_tx_addr(lbar(&bars->v_full[s]), 0u);
+          else
+            mbar_arrive_addr(lbar(&bars->v_full[s]));
+        }
       }
     }
     return true;
   };
   bool ok = issue_k(0);
+  for (int j = 1; j <= kTcPrefetchTiles; ++j) prefetch_k(j);   // after K(0): it goes out first
   for (int i = 1; ok && i < n_tiles; ++i) ok = issue_k(i) && issue_v(i - 1);
   if (ok) ok = issue_v(n_tiles - 1);
   return ok;
 }
 
-// ------------------------------------------------------------------------------ MMA issuer (even CTA)
-// Order: QK(0), then for each tile i >= 1: QK(i), PV(i-1); finally PV(n-1).  QK^T of the next tile
-// thus runs on the tensor cores while the softmax warps work on the current one.
-__device__ bool tc_mma(uint8_t* smem, TcBars* bars, uint32_t tmem, int n_tiles, volatile int* abort_flag) {
+// ------------------------------------------------------------------------------ MMA issuers (even CTA)
+// A single issuing thread cannot keep the tensor pipe busy with these shapes (each tcgen05.mma
+// holds its thread for about as long as the pair takes to execute an M = 128, N = 128, K = 16
+// step), so four warps issue: QK^T part A, QK^T part B (separate S accumulators over disjoint
+// dims) and PV (two warps, one per latent half).  QK^T of tile i + 1 then runs on the tensor cores while the softmax warps work on
+// tile i and PV of tile i - 1 completes.
+
+// Advance a shared-memory descriptor by `bytes` (a multiple of 16): the start address field
+// holds address / 16 in its low 14 bits, and every operand here lies below 256 KB, so the sum
+// never carries out of the field.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// S_part(i) = Q[:, dims of part] . K(i)[:, dims of part]^T into S buffer i & 1 of the part.
+__device__ bool tc_mma_qk(uint8_t* smem, TcBars* bars, uint32_t tmem, int part, int n_tiles,
+                          volatile int* abort_flag) {
   const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-  const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
-  const uint32_t sq = smem_u32(smem + kTcOffQ);
-  const uint32_t sp = smem_u32(smem + kTcOffP);
-  const uint32_t sk = smem_u32(smem + kTcOffK);
-  const uint32_t sv = smem_u32(smem + kTcOffV);
+  const int slab0 = tc_part_slab0(part);
+  const int nslabs = tc_part_slabs(part);
+  const uint64_t dq = sdesc_sw128(smem_u32(smem + kTcOffQ + slab0 * kTcSlab), 16, 1024);
+  const uint64_t dk = sdesc_sw128(smem_u32(smem + kTcOffK + slab0 * kTcSlab), 16, 1024);
+  const uint32_t scol = tmem + (part ? kTcColSB : kTcColSA);
   if (!mbar_wait_cluster(&bars->q_full, 0, 0x20)) return false;
-  tc_fence_after();
-  int kn = 0, vn = 0;
-  auto qk = [&](int i) -> bool {
+  for (int i = 0; i < n_tiles; ++i) {
     const int j = i & 1;
-    for (int kb = 0; kb < kTcKBoxes; ++kb, ++kn) {
-      const int s = kn % kTcKSlots;
-      if (!mbar_wait_cluster(&bars->k_full[s], static_cast<uint32_t>(kn / kTcKSlots) & 1u, 0x21)) return false;
+    // S buffer j last held tile i - 2: every softmax warp of both CTAs must have read it.
+    if (i >= 2 && !mbar_wait_cluster(&bars->s_empty[j], static_cast<uint32_t>((i - 2) >> 1) & 1u, 0x24)) return false;
+    if (!mbar_wait_cluster(&bars->k_full[part], static_cast<uint32_t>(i) & 1u, 0x21)) return false;
+    tc_fence_after();
+    for (int c = 0; c < nslabs; ++c)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        umma_bf16_pair(scol + 64 * j, sdesc_add(dq, c * kTcSlab + 32 * k), sdesc_add(dk, c * kTcSlab + 32 * k),
+                       idesc_qk, (c | k) != 0 ? 1u : 0u);
+    umma_commit_pair_mc(&bars->k_empty[part], 3);
+    umma_commit_pair_mc(&bars->s_full[j], 3);
+    if (*abort_flag) return false;
+  }
+  return true;
+}
+
+// O[:, latent half nh] += P(i) . V(i)[:, half nh].  Two warps issue, one per half (separate
+// accumulators); every release below therefore counts two commits.  The first V box (tokens
+// 0..63 of the tile) is consumed first so it is released (and refilled) before the second.
+__device__ bool tc_mma_pv(uint8_t* smem, TcBars* bars, uint32_t tmem, int nh, int n_tiles, volatile int* abort_flag) {
+  const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
+  const uint64_t dp = sdesc_sw128(smem_u32(smem + kTcOffP), 16, 1024);
+  const uint64_t dv = sdesc_sw128(smem_u32(smem + kTcOffV), kTcSlab, 1024);
+  int vn = 0;
+  bool ok = true;
+  for (int i = 0; i < n_tiles && ok; ++i) {
+    if (!mbar_wait_cluster(&bars->p_full, static_cast<uint32_t>(i) & 1u, 0x22)) {
+      ok = false;
+      break;
+    }
+    for (int h = 0; h < 2 && ok; ++h, ++vn) {
+      const int vs = vn % kTcVSlots;
+      if (!mbar_wait_cluster(&bars->v_full[vs], static_cast<uint32_t>(vn / kTcVSlots) & 1u, 0x23)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < kTcKBoxSlabs; ++c)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t ad = sdesc_sw128(sq + (kb * kTcKBoxSlabs + c) * kTcSlab + 32 * k, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sk + (s * kTcKBoxSlabs + c) * kTcSlab + 32 * k, 16, 1024);
-          umma_bf16_pair(tmem + 64 * j, ad, bd, idesc_qk, (kb | c | k) != 0 ? 1u : 0u);
-        }
-      umma_commit_pair_mc(&bars->k_empty[s], 3);
-    }
-    umma_commit_pair_mc(&bars->s_full[j], 3);
-    return true;
-  };
-  auto pv = [&](int i) -> bool {
-    if (!mbar_wait_cluster(&bars->p_full, static_cast<uint32_t>(i) & 1u, 0x22)) return false;
-    int vs[2];
-    for (int h = 0; h < 2; ++h, ++vn) {
-      vs[h] = vn % kTcVSlots;
-      if (!mbar_wait_cluster(&bars->v_full[vs[h]], static_cast<uint32_t>(vn / kTcVSlots) & 1u, 0x23)) return false;
-    }
-    tc_fence_after();
-    for (int nh = 0; nh < 2; ++nh)
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {  // 16-token groups of the tile
-        const uint64_t ad = sdesc_sw128(sp + (g >> 2) * kTcSlab + 32 * (g & 3), 16, 1024);
-        const uint32_t vb = sv + vs[g >> 2] * kTcVBox + nh * 2 * kTcSlab + (g & 3) * 2048;
-        const uint64_t bd = sdesc_sw128(vb, kTcSlab, 1024);
-        umma_bf16_pair(tmem + 128 + 128 * nh, ad, bd, idesc_pv, (i > 0 || g > 0) ? 1u : 0u);
+      for (int g4 = 0; g4 < 4; ++g4) {
+        const int g = 4 * h + g4;   // 16-token group of the tile
+        umma_bf16_pair(tmem + kTcColO + 128 * nh, sdesc_add(dp, h * kTcSlab + 32 * g4),
+                       sdesc_add(dv, vs * kTcVBox + nh * 2 * kTcSlab + g4 * 2048), idesc_pv,
+                       (i > 0 || g > 0) ? 1u : 0u);
       }
-    umma_commit_pair_mc(&bars->v_empty[vs[0]], 3);
-    umma_commit_pair_mc(&bars->v_empty[vs[1]], 3);
+      umma_commit_pair_mc(&bars->v_empty[vs], 3);
+    }
+    if (!ok) break;
     umma_commit_pair_mc(&bars->p_empty, 3);
     umma_commit_pair_mc(&bars->o_ready, 3);
-    return true;
-  };
-  bool ok = qk(0);
-  for (int i = 1; ok && i < n_tiles; ++i) ok = qk(i) && pv(i - 1);
-  if (ok) ok = pv(n_tiles - 1);
+    if (*abort_flag) ok = false;
+  }
   // The epilogue cannot wait on o_ready by parity: when it starts, o_ready may still be two
   // phases short of the last one.  A dedicated single-phase barrier says "all PV done".
   umma_commit_pair_mc(&bars->o_final, 3);
-  if (!ok) *abort_flag = 1;
   return ok;
+}
+
+// Each lane holds 128 bytes (w[0..31]) of its own row r = lane of a 32-row block whose rows lie
+// row_stride bytes apart from row0.  Written through a 4 KB per-warp staging buffer (16-byte
+// chunks XOR-swizzled by row, so both passes are free of bank conflicts beyond the 4 wavefronts
+// a 512-byte access needs), each global store instruction covers four whole 128-byte row
+// segments instead of 32 scattered 16-byte pieces.
+__device__ __forceinline__ void store_rows_128b(uint8_t* stage, const uint32_t (&w)[32], uint8_t* row0,
+                                                size_t row_stride, int lane) {
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(stage + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+        make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int row = 4 * j + (lane >> 3);
+    const int c = lane & 7;
+    const uint4 v = *reinterpret_cast<const uint4*>(stage + row * 128 + ((c ^ (row & 7)) << 4));
+    *reinterpret_cast<uint4*>(row0 + row * row_stride + c * 16) = v;
+  }
 }
 
 // ------------------------------------------------------------------------------ softmax warps
@@ -311,15 +396,22 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
       break;
     }
     tc_fence_after();
+    // S = S_A + S_B (the two QK^T parts over disjoint dims).
     float sc[32];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      uint32_t r[16];
-      tmem_ld16(tmem + lane_base + 64 * j + 32 * ch + 16 * q, r);
+      uint32_t ra[16], rb[16];
+      tmem_ld16(tmem + lane_base + kTcColSA + 64 * j + 32 * ch + 16 * q, ra);
+      tmem_ld16(tmem + lane_base + kTcColSB + 64 * j + 32 * ch + 16 * q, rb);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) sc[16 * q + e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 16; ++e) sc[16 * q + e] = __uint_as_float(ra[e]) + __uint_as_float(rb[e]);
     }
+    // S is in registers (tcgen05.wait::ld above): its TMEM buffer may take tile i + 2.  The
+    // arrival orders nothing else, so it is relaxed.
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_relaxed(lbar(&bars->s_empty[j]));
     // Tokens at or past the split end (only in a ragged last tile) get a score of -inf.
     const int tok0 = t_begin + i * kTcTile + 64 * half + 32 * ch;
     const int nvalid = t_end - tok0;
@@ -348,45 +440,52 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
     }
     if (__any_sync(0xffffffffu, need)) {
       // O must hold PV(i-1) before it is scaled.  Waiting on phase i-1 by parity is unambiguous
-      // here: s_full(i) was committed after PV(i-2), so o_ready is in phase i-1 or i.
+      // here: PV(i-2) is done (tile i-1 waited for it before writing P) and PV(i) needs this
+      // tile's P, so o_ready has completed i-1 or i phases.
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_ready, static_cast<uint32_t>(i - 1) & 1u, 0x31))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      for (int q = 0; q < 8; ++q) {
-        uint32_t r[16];
-        const uint32_t addr = tmem + lane_base + 128 + 128 * ch + 16 * q;
-        tmem_ld16(addr, r);
+      for (int qb = 0; qb < 4; ++qb) {   // 2 TMEM loads in flight per wait
+        const uint32_t addr = tmem + lane_base + kTcColO + 128 * ch + 32 * qb;
+        uint32_t r[2][16];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) tmem_ld16(addr + 16 * k, r[k]);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-        tmem_st16(addr, r);
+        for (int k = 0; k < 2; ++k) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[k][e] = __float_as_uint(__uint_as_float(r[k][e]) * alpha);
+          tmem_st16(addr + 16 * k, r[k]);
+        }
       }
       tmem_st_wait();
     }
-    // The P buffer is free once PV(i-1) has read it.  By parity this is unambiguous: s_full(i)
-    // was committed after PV(i-2), so p_empty is in phase i-1 or i.
+    // P for this tile, packed to bf16 in registers before the buffer is known to be free.
+    const float neg_m = -m_used;
+    float psum = 0.f;
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float p0 = ex2_approx(fmaf(sc[2 * e], a.scale_log2, neg_m));
+      const float p1 = ex2_approx(fmaf(sc[2 * e + 1], a.scale_log2, neg_m));
+      psum += p0 + p1;
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+      pk[e] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    // The P buffer is free once PV(i-1) has read it.  By parity this is unambiguous for the
+    // same reason: p_empty has completed i-1 or i phases.
     if (i >= 1 && !__all_sync(0xffffffffu, mbar_wait(&bars->p_empty, static_cast<uint32_t>(i - 1) & 1u, 0x32))) {
       ok = false;
       break;
     }
-    const float neg_m = -m_used;
-    float psum = 0.f;
     uint8_t* prow = smem + kTcOffP + half * kTcSlab + hl * 128;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      uint32_t pk[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float p0 = ex2_approx(fmaf(sc[8 * u + 2 * e], a.scale_log2, neg_m));
-        const float p1 = ex2_approx(fmaf(sc[8 * u + 2 * e + 1], a.scale_log2, neg_m));
-        psum += p0 + p1;
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-        pk[e] = *reinterpret_cast<uint32_t*>(&h2);
-      }
       const int unit = 4 * ch + u;   // 16-byte unit (8 tokens) within the 128-byte row
-      *reinterpret_cast<uint4*>(prow + ((unit ^ (hl & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(prow + ((unit ^ (hl & 7)) << 4)) =
+          make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
     }
     l_run = l_run * alpha + psum;
     fence_proxy_async_smem();
@@ -405,37 +504,40 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
   const int h = 64 * static_cast<int>(rank) + hl;
   const int64_t bh = static_cast<int64_t>(b) * kHeads + h;
   const int lat0 = 256 * ch + 128 * half;
-  const uint32_t ocol = tmem + lane_base + 128 + 128 * ch;
+  const uint32_t ocol = tmem + lane_base + kTcColO + 128 * ch;
+  // Every MMA and copy is done (o_final), so the V buffers are free: 4 KB of staging per warp.
+  uint8_t* stage = smem + kTcOffV + warp * 4096;
   if (direct) {
     const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
     __nv_bfloat16* dst = a.out_lat + bh * kDLat + lat0;
-    for (int q = 0; q < 8; ++q) {
-      uint32_t r[16];
-      tmem_ld16(ocol + 16 * q, r);
-      tmem_ld_wait();
-      uint32_t pk[8];
+    uint8_t* row0 = reinterpret_cast<uint8_t*>(dst) - static_cast<size_t>(lane) * kDLat * 2;
+    for (int qb = 0; qb < 2; ++qb) {   // 64 latent columns (128 bytes of bf16) per pass
+      uint32_t r[4][16];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
-        pk[e] = *reinterpret_cast<uint32_t*>(&h2);
-      }
-      uint4* d4 = reinterpret_cast<uint4*>(dst + 16 * q);
-      d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      for (int k = 0; k < 4; ++k) tmem_ld16(ocol + 16 * (4 * qb + k), r[k]);
+      tmem_ld_wait();
+      uint32_t w[32];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          __nv_bfloat162 h2 =
+              __floats2bfloat162_rn(__uint_as_float(r[k][2 * e]) * inv, __uint_as_float(r[k][2 * e + 1]) * inv);
+          w[8 * k + e] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+      store_rows_128b(stage, w, row0 + 128 * qb, static_cast<size_t>(kDLat) * 2, lane);
     }
     if (half == 0 && ch == 0 && a.lse != nullptr) a.lse[bh] = l_tot > 0.f ? (m_used + log2f(l_tot)) * kLn2 : -INFINITY;
   } else {
     const int64_t ml = (static_cast<int64_t>(b) * a.S + split) * kHeads + h;
     float* dst = a.ws.o + ml * kDLat + lat0;
-    for (int q = 0; q < 8; ++q) {
-      uint32_t r[16];
-      tmem_ld16(ocol + 16 * q, r);
+    uint8_t* row0 = reinterpret_cast<uint8_t*>(dst) - static_cast<size_t>(lane) * kDLat * 4;
+    for (int qb = 0; qb < 4; ++qb) {   // 32 latent columns (128 bytes of fp32) per pass
+      uint32_t w[32];
+      tmem_ld16(ocol + 32 * qb, *reinterpret_cast<uint32_t(*)[16]>(&w[0]));
+      tmem_ld16(ocol + 32 * qb + 16, *reinterpret_cast<uint32_t(*)[16]>(&w[16]));
       tmem_ld_wait();
-      float4* d4 = reinterpret_cast<float4*>(dst + 16 * q);
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        d4[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]), __uint_as_float(r[4 * e + 2]),
-                            __uint_as_float(r[4 * e + 3]));
+      store_rows_128b(stage, w, row0 + 128 * qb, static_cast<size_t>(kDLat) * 4, lane);
     }
     if (half == 0 && ch == 0) {
       a.ws.m[ml] = m_used;
@@ -447,8 +549,9 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
 // ------------------------------------------------------------------------------ kernel
 // grid = (2 * S, batch), clusters of 2 along x: blockIdx.x = 2 * split + rank.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_q, const DecodeTcArgs a) {
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_ka, const __grid_constant__ CUtensorMap tm_kb,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
+                     const DecodeTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   TcBars* bars = reinterpret_cast<TcBars*>(smem + kTcOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTcOffMisc);
@@ -475,21 +578,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   const bool direct = splits_used(L, a.S, kSplitAlign) == 1;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcKSlots; ++s) {
-      mbar_init(&bars->k_full[s], 2);   // one arrival per CTA of the pair (plus the copies' bytes)
-      mbar_init(&bars->k_empty[s], 1);
+    for (int part = 0; part < 2; ++part) {
+      mbar_init(&bars->k_full[part], 2);   // one arrival per CTA of the pair (plus the copies' bytes)
+      mbar_init(&bars->k_empty[part], 1);
     }
     for (int s = 0; s < kTcVSlots; ++s) {
       mbar_init(&bars->v_full[s], 2);   // one arrival per CTA of the pair (plus the copies' bytes)
-      mbar_init(&bars->v_empty[s], 1);
+      mbar_init(&bars->v_empty[s], 2);   // one commit per PV warp
     }
     mbar_init(&bars->fix, 1);
-    mbar_init(&bars->s_full[0], 1);
-    mbar_init(&bars->s_full[1], 1);
+    mbar_init(&bars->s_full[0], 2);   // one commit per QK^T part
+    mbar_init(&bars->s_full[1], 2);
+    mbar_init(&bars->s_empty[0], 2 * kTcSoftmaxWarps);   // every softmax warp of both CTAs
+    mbar_init(&bars->s_empty[1], 2 * kTcSoftmaxWarps);
     mbar_init(&bars->p_full, 2 * kTcSoftmaxWarps);   // every softmax warp of both CTAs
-    mbar_init(&bars->p_empty, 1);
-    mbar_init(&bars->o_ready, 1);
-    mbar_init(&bars->o_final, 1);
+    mbar_init(&bars->p_empty, 2);   // one commit per PV warp
+    mbar_init(&bars->o_ready, 2);
+    mbar_init(&bars->o_final, 2);
     mbar_init(&bars->q_full, 2);
     *abort_flag = 0;
     fence_mbar_init();
@@ -499,7 +604,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     tmem_relinquish_pair();
   }
   if (warp == kTcProducerWarp && (threadIdx.x & 31) == 0) {
-    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_ka);
+    tma_prefetch_desc(&tm_kb);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_q);
   }
@@ -511,11 +617,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   if (warp < kTcSoftmaxWarps) {
     tc_softmax(a, smem, bars, red, tmem, rank, b, split, t_begin, t_end, n_tiles, direct, abort_flag);
   } else if (warp == kTcProducerWarp) {
-    if ((threadIdx.x & 31) == 0 &&
-        !tc_producer(&tm_k, &tm_v, &tm_q, a, smem, bars, rank, b, t_begin, t_end, n_tiles, abort_flag))
+    if (!tc_producer(&tm_ka, &tm_kb, &tm_v, &tm_q, a, smem, bars, rank, b, t_begin, t_end, n_tiles, abort_flag) &&
+        (threadIdx.x & 31) == 0)
       *abort_flag = 1;
   } else if (rank == 0 && (threadIdx.x & 31) == 0) {
-    tc_mma(smem, bars, tmem, n_tiles, abort_flag);
+    bool ok = true;
+    if (warp == kTcMmaWarp) ok = tc_mma_qk(smem, bars, tmem, 0, n_tiles, abort_flag);
+    else if (warp == kTcMmaBWarp) ok = tc_mma_qk(smem, bars, tmem, 1, n_tiles, abort_flag);
+    else if (warp == kTcPvWarp) ok = tc_mma_pv(smem, bars, tmem, 0, n_tiles, abort_flag);
+    else ok = tc_mma_pv(smem, bars, tmem, 1, n_tiles, abort_flag);
+    if (!ok) *abort_flag = 1;
   }
   __syncwarp();
   if (*reinterpret_cast<volatile int*>(abort_flag)) __nanosleep(200000);  // let stray copies land

@@ -69,14 +69,14 @@ bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
 }
 
 // 3-D bf16 view of [rows][576] as (64-element dim-slab, row, slab index) for boxes of
-// 64 elements x 64 rows x kTcKBoxSlabs slabs, 128-byte swizzle: one box fills kTcKBoxSlabs
-// consecutive 8 KB slabs of 64 rows x 128 bytes.
-bool make_map_slabs(CUtensorMap* map, const void* base, uint64_t rows) {
+// 64 elements x 64 rows x box_slabs slabs, 128-byte swizzle: one box fills box_slabs consecutive
+// 8 KB slabs of 64 rows x 128 bytes.
+bool make_map_slabs(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_slabs) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const cuuint64_t dims[3] = {64, rows, 9};
   const cuuint64_t strides[2] = {mla::kDRow * 2, 128};
-  const cuuint32_t box[3] = {64, 64, mla::kTcKBoxSlabs};
+  const cuuint32_t box[3] = {64, 64, box_slabs};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -184,6 +184,23 @@ mla_status mla_get_device_error(int32_t* code) {
   return MLA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// base^(-2i/d_R) for the 32 rotation pairs, in fp64 (the angle pos * inv_freq is formed in fp64 on
+// the device).
+mla::RopeFreq rope_freq(float rope_base) {
+  mla::RopeFreq f;
+  for (int i = 0; i < mla::kDRope / 2; ++i)
+    f.inv_freq[i] = std::pow(static_cast<double>(rope_base), -2.0 * i / static_cast<double>(mla::kDRope));
+  return f;
+}
+
+}  // namespace
+
+extern "C" {
+
 mla_status mla_cache_append(const mla_bf16* c_new, const mla_bf16* kr_new, const int32_t* seq_ids,
                             const int32_t* pos, mla_bf16* cache, const int32_t* block_table,
                             mla_cache_desc desc, int32_t n_tokens, float rope_base, void* stream) {
@@ -196,9 +213,9 @@ mla_status mla_cache_append(const mla_bf16* c_new, const mla_bf16* kr_new, const
     return MLA_ERR_INVALID_ARG;
   if (seq_ids == nullptr && n_tokens > desc.num_seqs) return MLA_ERR_INVALID_ARG;
   if (n_tokens > INT_MAX / 2) return MLA_ERR_UNSUPPORTED;
-  mla::cache_append_kernel<<<n_tokens, 72, 0, as_stream(stream)>>>(
-      reinterpret_cast<const uint4*>(c_new), reinterpret_cast<const uint4*>(kr_new), seq_ids, pos,
-      reinterpret_cast<uint4*>(cache), v, static_cast<double>(rope_base));
+  mla::cache_append_kernel<<<n_tokens, 96, 0, as_stream(stream)>>>(
+      reinterpret_cast<const uint4*>(c_new), reinterpret_cast<const __nv_bfloat162*>(kr_new), seq_ids, pos,
+      reinterpret_cast<uint4*>(cache), v, rope_freq(rope_base));
   return launch_status();
 }
 
@@ -246,7 +263,7 @@ mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int3
                                                    static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow, s);
   if (st != MLA_OK) return st;
   mla::qpe_kernel<<<batch, mla::kHeads * 8, 0, s>>>(reinterpret_cast<const uint4*>(q_pe), q_pos,
-                                                    reinterpret_cast<uint4*>(q_full), static_cast<double>(rope_base));
+                                                    reinterpret_cast<uint4*>(q_full), rope_freq(rope_base));
   return launch_status();
 }
 
@@ -313,14 +330,16 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
   a.ws = mla::ws_carve(workspace, batch, S);
   a.out_lat = reinterpret_cast<__nv_bfloat16*>(out_lat);
   a.lse = lse;
-  CUtensorMap tk, tv, tq;
-  if (!make_map_slabs(&tk, cache, desc.num_rows) || !make_map_vbox(&tv, cache, desc.num_rows) ||
-      !make_map_slabs(&tq, q_full, static_cast<uint64_t>(batch) * mla::kHeads))
+  a.cache = reinterpret_cast<const uint8_t*>(cache);
+  CUtensorMap tka, tkb, tv, tq;
+  if (!make_map_slabs(&tka, cache, desc.num_rows, mla::kTcKSlabsA) ||
+      !make_map_slabs(&tkb, cache, desc.num_rows, mla::kTcKSlabsB) || !make_map_vbox(&tv, cache, desc.num_rows) ||
+      !make_map_slabs(&tq, q_full, static_cast<uint64_t>(batch) * mla::kHeads, 9))
     return MLA_ERR_CUDA;
   if (cudaFuncSetAttribute(mla::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kTcSmemBytes) !=
       cudaSuccess)
     return MLA_ERR_CUDA;
-  mla::decode_tc_kernel<<<dim3(2 * S, batch), mla::kTcThreads, mla::kTcSmemBytes, s>>>(tk, tv, tq, a);
+  mla::decode_tc_kernel<<<dim3(2 * S, batch), mla::kTcThreads, mla::kTcSmemBytes, s>>>(tka, tkb, tv, tq, a);
   mla_status ls = launch_status();
   if (ls != MLA_OK) return ls;
   mla::combine_kernel<<<dim3(batch, mla::kHeads / 4), 128, 0, s>>>(
