@@ -109,9 +109,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------- oracle
-def time_oracle(lens, budget_tokens=1024, seed=4242):
-    """The fp64 oracle (explicit form, as it stands) on a bounded sample of the workload:
-    one sequence of the workload's first length, truncated to `budget_tokens` tokens."""
+def time_oracle(lens, budget_tokens=4096, seed=4242):
+    """The fp64 oracle (explicit form, as it stands) on one sequence of the workload's first
+    length, truncated to `budget_tokens` tokens.  Returns (tokens, seconds)."""
     import oracle
     L = int(min(int(lens[0]), budget_tokens))
     b = mi.decode_batch(seed, [L])
@@ -123,6 +123,17 @@ def time_oracle(lens, budget_tokens=1024, seed=4242):
     oracle.decode_step(*args, form="explicit")
     dt = time.perf_counter() - t0
     return L, dt
+
+
+def time_oracle_sample(lens, min_seconds=12.0, max_seqs=64):
+    """Bounded CPU baseline: sequences of the workload (first length, at most 4096 tokens each,
+    distinct seeds) through the oracle until about `min_seconds` of work.  Returns
+    (tokens, seconds, sequences)."""
+    tok, secs, n = 0, 0.0, 0
+    while n < max_seqs and (n == 0 or secs < min_seconds):
+        L, dt = time_oracle(lens, seed=4242 + n)
+        tok, secs, n = tok + L, secs + dt, n + 1
+    return tok, secs, n
 
 
 def cpu_threads():
@@ -141,8 +152,8 @@ def run_reference(args, rank, world):
     for _ in range(args.warmup):
         time_oracle(lens, budget_tokens=256)
     tok, secs = 0, 0.0
-    for _ in range(args.steps):
-        L, dt = time_oracle(lens, budget_tokens=1024)
+    for i in range(args.steps):
+        L, dt = time_oracle(lens, seed=4242 + i)
         tok += L
         secs += dt
     gbs = tok * ROW_BYTES / secs / 1e9
@@ -274,32 +285,50 @@ def recorded_traffic(workload):
 LAUNCHES_PER_LAYER = 6   # append, absorb GEMM, q_pe rotation, decode split, combine, un-absorb GEMM
 
 
-PHASES = ("append", "absorb_q", "decode_attn", "unabsorb_v")
+GRAPH_PHASES = ("append_absorb", "decode_attn", "unabsorb_v")
 
 
-def run_step(st, i, ev=None):
-    """One decode step over every layer of the workload.  With `ev`, events ev[layer][k] bracket
-    the phases: k and k + 1 around PHASES[k]."""
+def layer_phase(st, i, li, k):
+    """Phase k of GRAPH_PHASES for layer li of step i (cache copy i mod the copies)."""
     import mla_latent_kv_20_b200 as m
-    for li, layer in enumerate(st["layers"]):
-        cache = layer["caches"][i % len(layer["caches"])]
-        d = layer["dev"]
-        if ev is not None:
-            ev[li][0].record()
+    layer = st["layers"][li]
+    cache = layer["caches"][i % len(layer["caches"])]
+    d = layer["dev"]
+    if k == 0:
         m.cache_append(d["c_new"], d["kr_new"], st["pos"], cache.data, cache.desc, seq_ids=st["seq_ids"],
                        block_table=cache.block_table)
-        if ev is not None:
-            ev[li][1].record()
         m.absorb_q(d["q_nope"], d["q_pe"], layer["w_uk"], st["q_full"], q_pos=st["pos"])
-        if ev is not None:
-            ev[li][2].record()
+    elif k == 1:
         m.decode_attn(st["q_full"], cache.data, cache.seq_lens, cache.desc, st["workspace"], st["out_lat"],
                       lse=st["lse"], block_table=cache.block_table, num_splits=st["splits"])
-        if ev is not None:
-            ev[li][3].record()
+    else:
         m.unabsorb_v(st["out_lat"], layer["w_uv"], st["out"])
-        if ev is not None:
-            ev[li][4].record()
+
+
+def capture_step_graphs(st, n_rot, stream):
+    """graphs[r][li][k]: phase k of layer li on cache copy r, each captured once (the kernels'
+    arguments, tensor maps included, are fixed at capture)."""
+    import torch
+    graphs = []
+    for r in range(n_rot):
+        per_layer = []
+        for li in range(len(st["layers"])):
+            gs = []
+            for k in range(len(GRAPH_PHASES)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    layer_phase(st, r, li, k)
+                gs.append(g)
+            per_layer.append(gs)
+        graphs.append(per_layer)
+    return graphs
+
+
+def run_step(st, i):
+    """One decode step over every layer of the workload, through plain API calls."""
+    for li in range(len(st["layers"])):
+        for k in range(len(GRAPH_PHASES)):
+            layer_phase(st, i, li, k)
 
 
 def reduce_max_over_ranks(values, world, device=None):
@@ -341,7 +370,27 @@ def run_ours(args, rank, world, local_rank):
         run_step(st, i)
     torch.cuda.synchronize()
     n_layers = len(st["layers"])
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(len(PHASES) + 1)] for _ in range(n_layers)]
+    # The timed step replays CUDA graphs of the step's launches (what a serving loop does), three
+    # per layer so that events between them bracket the decode call on the device.
+    n_rot = len(st["layers"][0]["caches"])
+    cap_stream = torch.cuda.Stream()
+    graphs = capture_step_graphs(st, n_rot, cap_stream)
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+
+    def replay_step(i, ev=None):
+        for li in range(n_layers):
+            for k, g in enumerate(graphs[i % n_rot][li]):
+                if ev is not None:
+                    ev[li][k].record()
+                g.replay()
+            if ev is not None:
+                ev[li][len(GRAPH_PHASES)].record()
+
+    for i in range(args.warmup):
+        replay_step(i)
+    torch.cuda.synchronize()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(len(GRAPH_PHASES) + 1)] for _ in range(n_layers)]
            for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local_rank)
@@ -352,7 +401,7 @@ def run_ours(args, rank, world, local_rank):
     t_start.record()
     h0 = time.perf_counter()
     for i in range(args.steps):
-        run_step(st, i, evs[i])
+        replay_step(i, evs[i])
     host_ms = (time.perf_counter() - h0) * 1e3 / args.steps
     t_end.record()
     torch.cuda.synchronize()
@@ -360,9 +409,10 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop()
     ms = t_start.elapsed_time(t_end) / args.steps
     phase_ms = {p: sum(lev[k].elapsed_time(lev[k + 1]) for step in evs for lev in step) / (args.steps * n_layers)
-                for k, p in enumerate(PHASES)}
+                for k, p in enumerate(GRAPH_PHASES)}
     dec_ms = phase_ms["decode_attn"]
     assert m.get_device_error() == 0
+    del graphs
 
     # end to end through the public API with host buffers: H2D of the step's inputs (every layer's
     # new-token row and query), the step, D2H of the result, every step
@@ -423,6 +473,7 @@ def run_ours(args, rank, world, local_rank):
         "decode_layer_ms": dec_ms,
         "phase_ms_per_layer": phase_ms,
         "host_issue_ms_per_step": host_ms,
+        "timed_step": "CUDA graph replay of the step's launches (3 graphs per layer); e2e uses plain API calls",
         "roofline_step_frac": roofline_s / (ms * 1e-3),
         "roofline": {"kernel": "mla_decode_attn (split-KV decode + combine)", "bound": "hbm",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
@@ -434,12 +485,12 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     if not args.no_cpu_baseline:
-        L, dt = time_oracle(st["lens"])
+        tok, dt, nseq = time_oracle_sample(st["lens"])
         threads, cores = cpu_threads()
-        line["cpu_baseline"] = {"value": L * ROW_BYTES / dt / 1e9, "unit": UNIT, "cores": threads,
+        line["cpu_baseline"] = {"value": tok * ROW_BYTES / dt / 1e9, "unit": UNIT, "cores": threads,
                                 "kind": "oracle", "affinity_cores": cores,
-                                "sample": f"one sequence of {L} tokens, explicit fp64 form "
-                                          f"({dt:.1f} s), GB/s of cached rows processed"}
+                                "sample": f"{nseq} sequences of {tok // nseq} tokens of this workload, explicit "
+                                          f"fp64 form ({dt:.1f} s of CPU work), GB/s of cached rows processed"}
     print(json.dumps(line), flush=True)
 
 
