@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(96) cache_append_kernel(const uint4* __restric
                                                           const int32_t* __restrict__ seq_ids,
                                                           const int32_t* __restrict__ pos, uint4* cache,
                                                           CacheView v, RopeFreq f) {
+  pdl_trigger();
+  pdl_wait();
   const int i = blockIdx.x;
   const int seq = seq_ids ? seq_ids[i] : i;
   const int p = pos[i];
@@ -100,6 +102,8 @@ __global__ void __launch_bounds__(96) cache_append_kernel(const uint4* __restric
 __global__ void __launch_bounds__(1024) qpe_kernel(const uint4* __restrict__ q_pe, const int32_t* __restrict__ q_pos,
                                                    uint4* __restrict__ q_full, RopeFreq f) {
   __shared__ double cs_sn[kDRope / 2][2];
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x;
   const int h = threadIdx.x >> 3;
   const int ch = threadIdx.x & 7;

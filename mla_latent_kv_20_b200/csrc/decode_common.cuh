@@ -71,6 +71,8 @@ __global__ void __launch_bounds__(128) combine_kernel(Workspace ws, const int32_
                                                       int align, int capacity, int single_done,
                                                       __nv_bfloat16* __restrict__ out_lat,
                                                       float* __restrict__ lse) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x;
   const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;

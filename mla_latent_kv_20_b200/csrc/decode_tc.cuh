@@ -564,6 +564,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     if (threadIdx.x == 0) set_dev_error(0x8);
     return;
   }
+  // seq_lens (read next) may come from the previous kernel in the stream.
+  pdl_trigger();
+  pdl_wait();
   const uint32_t rank = cluster_ctarank();
   const int split = blockIdx.x >> 1;
   const int b = blockIdx.y;

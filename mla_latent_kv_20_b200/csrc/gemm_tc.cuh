@@ -73,6 +73,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
+  // Setup above overlaps the previous kernel; nothing global is touched before this point.
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 4 && lane == 0) {
     // ---------------- TMA producer

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/mla.h"
 #include "append.cuh"
@@ -26,9 +27,28 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-mla_status launch_status() {
-  const cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+// Launch with programmatic stream serialisation: the kernel may be scheduled while the previous
+// kernel on the stream still runs; it waits for that kernel (griddepcontrol.wait) before it
+// touches global memory, so ordering against earlier work on the stream is unchanged.
+template <typename... KArgs, typename... Args>
+mla_status launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
 }
 
 int device_sm_count() {
@@ -213,10 +233,9 @@ mla_status mla_cache_append(const mla_bf16* c_new, const mla_bf16* kr_new, const
     return MLA_ERR_INVALID_ARG;
   if (seq_ids == nullptr && n_tokens > desc.num_seqs) return MLA_ERR_INVALID_ARG;
   if (n_tokens > INT_MAX / 2) return MLA_ERR_UNSUPPORTED;
-  mla::cache_append_kernel<<<n_tokens, 96, 0, as_stream(stream)>>>(
-      reinterpret_cast<const uint4*>(c_new), reinterpret_cast<const __nv_bfloat162*>(kr_new), seq_ids, pos,
-      reinterpret_cast<uint4*>(cache), v, rope_freq(rope_base));
-  return launch_status();
+  return launch_chained(mla::cache_append_kernel, dim3(n_tokens), dim3(96), 0, as_stream(stream),
+                        reinterpret_cast<const uint4*>(c_new), reinterpret_cast<const __nv_bfloat162*>(kr_new),
+                        seq_ids, pos, reinterpret_cast<uint4*>(cache), v, rope_freq(rope_base));
 }
 
 }  // extern "C"
@@ -241,8 +260,8 @@ mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, in
       cudaSuccess)
     return MLA_ERR_CUDA;
   dim3 grid(m_total / 128, mla::kHeads, (batch + nt - 1) / nt);
-  kern<<<grid, mla::kGemmThreads, smem, stream>>>(ta, tb, out, batch, nt, out_bstride, out_hstride);
-  return launch_status();
+  return launch_chained(kern, grid, dim3(mla::kGemmThreads), smem, stream, ta, tb, out, batch, nt, out_bstride,
+                        out_hstride);
 }
 
 }  // namespace
@@ -262,9 +281,9 @@ mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int3
                                                    reinterpret_cast<__nv_bfloat16*>(q_full),
                                                    static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow, s);
   if (st != MLA_OK) return st;
-  mla::qpe_kernel<<<batch, mla::kHeads * 8, 0, s>>>(reinterpret_cast<const uint4*>(q_pe), q_pos,
-                                                    reinterpret_cast<uint4*>(q_full), rope_freq(rope_base));
-  return launch_status();
+  return launch_chained(mla::qpe_kernel, dim3(batch), dim3(mla::kHeads * 8), 0, s,
+                        reinterpret_cast<const uint4*>(q_pe), q_pos, reinterpret_cast<uint4*>(q_full),
+                        rope_freq(rope_base));
 }
 
 mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf16* out, int32_t batch,
@@ -339,13 +358,11 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
   if (cudaFuncSetAttribute(mla::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kTcSmemBytes) !=
       cudaSuccess)
     return MLA_ERR_CUDA;
-  mla::decode_tc_kernel<<<dim3(2 * S, batch), mla::kTcThreads, mla::kTcSmemBytes, s>>>(tka, tkb, tv, tq, a);
-  mla_status ls = launch_status();
+  mla_status ls = launch_chained(mla::decode_tc_kernel, dim3(2 * S, batch), dim3(mla::kTcThreads),
+                                 static_cast<size_t>(mla::kTcSmemBytes), s, tka, tkb, tv, tq, a);
   if (ls != MLA_OK) return ls;
-  mla::combine_kernel<<<dim3(batch, mla::kHeads / 4), 128, 0, s>>>(
-      a.ws, seq_lens, S, mla::kSplitAlign, capacity, /*single_done=*/1, reinterpret_cast<__nv_bfloat16*>(out_lat),
-      lse);
-  return launch_status();
+  return launch_chained(mla::combine_kernel, dim3(batch, mla::kHeads / 4), dim3(128), 0, s, a.ws, seq_lens, S,
+                        mla::kSplitAlign, capacity, /*single_done=*/1, reinterpret_cast<__nv_bfloat16*>(out_lat), lse);
 }
 
 }  // extern "C"

@@ -105,6 +105,16 @@ __device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, u
   }
 }
 
+// ---------------------------------------------------------------------------------- launch chaining
+// Kernels are launched with programmatic stream serialisation: a kernel's CTAs may start (and do
+// their setup) while the previous kernel in the stream is still running.  pdl_wait() blocks the
+// calling thread until that previous kernel has completed and its memory is visible; every
+// thread calls it before it reads or writes any global buffer (an L2 prefetch aside).
+// pdl_trigger() lets the next kernel's CTAs be scheduled as soon as every CTA of this one has
+// started.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
