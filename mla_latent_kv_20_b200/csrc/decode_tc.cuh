@@ -488,10 +488,17 @@ __device__ void tc_softmax(const DecodeTcArgs& a, uint8_t* smem, TcBars* bars, f
           make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
     }
     l_run = l_run * alpha + psum;
+    // Publish: P (generic-proxy writes) made visible to the tensor core, the O correction's
+    // tcgen05.st ordered before the thread sync, then one release of the warp's shared-memory
+    // writes (restricted to shared memory: P is all that PV reads from this thread's work)
+    // followed by a relaxed arrival on the even CTA's barrier.
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive_addr(lbar(&bars->p_full));
+    if (lane == 0) {
+      fence_release_smem_to_cluster();
+      mbar_arrive_relaxed(lbar(&bars->p_full));
+    }
   }
   // ---- epilogue
   if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0u, 0x33))) ok = false;

@@ -227,6 +227,13 @@ __device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar_cluster_addr) {
 __device__ __forceinline__ void mbar_arrive_addr(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
+// Orders this thread's prior writes to its own CTA's shared memory before its subsequent
+// cluster-scope operations (a relaxed mbarrier arrival): the release half of a release arrival,
+// restricted to shared::cta, which is far cheaper than a full cluster-scope release (that also
+// orders global memory).
+__device__ __forceinline__ void fence_release_smem_to_cluster() {
+  asm volatile("fence.release.sync_restrict::shared::cta.cluster;" ::: "memory");
+}
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core / TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
