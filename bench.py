@@ -263,7 +263,10 @@ def setup_replica(name, device):
 # choose their launch shape.  A digest that no longer matches means the kernels changed since the
 # counters were taken, and the traffic is reported as null.
 TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh", "csrc/mla_lib.cu")
-MEASURED_TRAFFIC = {}   # workload -> {"bytes": int, "sha256": str, "profile": str}
+MEASURED_TRAFFIC = {   # workload -> {"bytes": int, "sha256": str, "profile": str}
+    "b32_l4096": {"bytes": 175316992 + 3219712 + 16854528, "sha256": "40dfdc27ff37a6956f1763ac2bf2e5241927fdb419eea7d032c66f7f3be7cab9",
+                  "profile": "profiles/decode_tc_b32_l4096.md (decode + combine, ncu cache flush per kernel)"},
+}
 
 
 def traffic_sources_digest():
