@@ -8,9 +8,13 @@
 // the N operand (N = batch rounded up to 16, at most 256 per CTA):
 //     D[m, n] = sum_k Wt[m, k] * X[n, k]
 // A = Wt is MN-major in memory (the weight's output index is contiguous), B = X is K-major.
-// One CTA computes a 128 x N tile of one head: TMA streams 64-wide K slabs of A and B into a
-// ring of shared-memory stages (128-byte swizzle), one thread issues tcgen05.mma into a TMEM
-// accumulator, four warps read TMEM back and store bf16.
+// One CTA computes a 128 x N tile of one head.  Its operands arrive in few, large TMA copies (each
+// copy costs the CTA's TMA unit a roughly fixed time whatever its size): per stage of KS
+// contraction rows, one 3-D box of the weight (KS rows x both 64-wide M chunks) and one 3-D box of
+// the activation (N rows x KS/64 K slabs), 128-byte swizzled, into a ring of NSTAGE stages.  One
+// thread issues tcgen05.mma into a TMEM accumulator; four warps read TMEM back and store bf16.
+// The weight tile does not depend on earlier kernels, so it is prefetched into L2 before the
+// kernel waits for its predecessor in the stream.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -19,22 +23,26 @@
 
 namespace mla {
 
-constexpr int kGemmThreads = 192;    // warps 0-3: epilogue, warp 4: TMA producer, warp 5: MMA issuer
-constexpr int kGemmKSlab = 64;       // K per stage (one 128-byte swizzle row of bf16)
-constexpr int kGemmASlabBytes = 2 * 64 * 128;  // two 64-wide M chunks x 64 K rows x 128 B
+constexpr int kGemmThreads = 224;    // warps 0-3: epilogue, warp 4: TMA producer, warps 5-6: MMA issuers
+constexpr int kGemmIssuers = 2;      // MMA-issuing warps, each with its own accumulator (summed at the end)
+constexpr int kGemmKS = 128;         // contraction rows per stage
 
-__host__ __device__ constexpr int gemm_stage_bytes(int nt) { return kGemmASlabBytes + nt * 128; }
+// Stage bytes: weight KS x 128 (two 64-wide M chunks) + activation nt x KS, bf16.
+__host__ __device__ constexpr int gemm_stage_bytes(int nt) { return kGemmKS * 256 + nt * kGemmKS * 2; }
 
 // KTOT: contraction length (128 for absorption, 512 for un-absorption).
-// tmA: 2-D view of the weight, inner = M_total (output index), outer = heads * KTOT; box {64, 64}.
-// tmB: 2-D view of the activation, inner = heads * KTOT, outer = batch; box {64, nt}.
+// tmA: 3-D view of the weight (64-element M chunk, contraction row = h * KTOT + k, M chunk index);
+//      box {64, KS, 2}: smem [chunk][KS rows][128 B].
+// tmB: 3-D view of the activation (64-element K slab, batch row, slab index = (h * KTOT + k) / 64);
+//      box {64, nt, KS / 64}: smem [slab][nt rows][128 B].
 // out element (n, h, m) is stored at out[n * out_bstride + h * out_hstride + m].
 template <int KTOT, int NSTAGE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      __nv_bfloat16* __restrict__ out, int batch, int nt, int64_t out_bstride,
                      int out_hstride) {
-  constexpr int KSLABS = KTOT / kGemmKSlab;
+  constexpr int KSTAGES = KTOT / kGemmKS;
+  static_assert(KTOT % kGemmKS == 0, "contraction length");
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -50,14 +58,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int m0 = blockIdx.x * 128;
   const int h = blockIdx.y;
   const int n0 = blockIdx.z * nt;
-  const uint32_t tmem_cols = nt <= 32 ? 32u : (nt <= 64 ? 64u : (nt <= 128 ? 128u : 256u));
+  const uint32_t acc_cols = nt <= 32 ? 32u : (nt <= 64 ? 64u : (nt <= 128 ? 128u : 256u));
+  const uint32_t tmem_cols = kGemmIssuers * acc_cols;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], kGemmIssuers);   // one commit per issuing warp
     }
-    mbar_init(done, 1);
+    mbar_init(done, kGemmIssuers);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -68,12 +77,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    for (int ks = 0; ks < KSTAGES; ++ks) tma_prefetch_l2_3d(&tmA, 0, h * KTOT + ks * kGemmKS, m0 / 64);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
-  // Setup above overlaps the previous kernel; nothing global is touched before this point.
+  // Setup above (and the weight prefetch) overlaps the previous kernel; nothing else global is
+  // touched before this point.
   pdl_trigger();
   pdl_wait();
 
@@ -82,7 +93,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int armed[NSTAGE];
 #pragma unroll
     for (int s = 0; s < NSTAGE; ++s) armed[s] = 0;
-    for (int ks = 0; ks < KSLABS; ++ks) {
+    for (int ks = 0; ks < KSTAGES; ++ks) {
       const int s = ks % NSTAGE;
       if (ks >= NSTAGE && !mbar_wait(&empty[s], ((ks / NSTAGE) - 1) & 1)) {
         *abort_flag = 1;
@@ -90,22 +101,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (*reinterpret_cast<volatile int*>(abort_flag)) break;
       uint8_t* sa = smem + s * stage_bytes;
-      uint8_t* sb = sa + kGemmASlabBytes;
+      uint8_t* sb = sa + kGemmKS * 256;
       mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(stage_bytes));
-      const int krow = h * KTOT + ks * kGemmKSlab;
-      tma_load_2d(sa, &tmA, &full[s], m0, krow);
-      tma_load_2d(sa + 8192, &tmA, &full[s], m0 + 64, krow);
-      tma_load_2d(sb, &tmB, &full[s], krow, n0);
+      const int krow = h * KTOT + ks * kGemmKS;
+      tma_load_3d(sa, &tmA, &full[s], 0, krow, m0 / 64);
+      tma_load_3d(sb, &tmB, &full[s], 0, n0, krow / 64);
       ++armed[s];
     }
     // Drain: never leave the CTA while one of its copies is still landing.
     for (int s = 0; s < NSTAGE; ++s)
       if (armed[s] > 0) mbar_wait(&full[s], (armed[s] - 1) & 1);
-  } else if (warp == 5 && lane == 0) {
-    // ---------------- MMA issuer
+  } else if (warp >= 5 && lane == 0) {
+    // ---------------- MMA issuers: warp 5 + j takes the 16-deep K steps g with g % 2 == j into
+    // accumulator j (a single thread issues one MMA per ~125 cycles, so two halve the issue time)
+    const int j = warp - 5;
+    const uint32_t acc = tmem_d + j * acc_cols;
     const uint32_t idesc = idesc_bf16_f32(128, nt, /*a_mn_major=*/true, /*b_mn_major=*/false);
-    bool ok = true;
-    for (int ks = 0; ks < KSLABS && ok; ++ks) {
+    bool ok = true, first = true;
+    for (int ks = 0; ks < KSTAGES && ok; ++ks) {
       const int s = ks % NSTAGE;
       if (!mbar_wait(&full[s], (ks / NSTAGE) & 1)) {
         *abort_flag = 1;
@@ -114,34 +127,47 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + s * stage_bytes);
-      const uint32_t sb = sa + kGemmASlabBytes;
+      const uint32_t sb = sa + kGemmKS * 256;
 #pragma unroll
-      for (int kk = 0; kk < kGemmKSlab / 16; ++kk) {
-        // A (MN-major): 16 K rows per MMA = 2 swizzle atoms of 1024 B; M chunks 8192 B apart.
-        const uint64_t adesc = sdesc_sw128(sa + kk * 2048, 8192, 1024);
-        // B (K-major): 16 K elements = 32 B into each 128-byte row; 8-row groups 1024 B apart.
-        const uint64_t bdesc = sdesc_sw128(sb + kk * 32, 16, 1024);
-        umma_bf16_ss(tmem_d, adesc, bdesc, idesc, (ks | kk) != 0 ? 1u : 0u);
+      for (int kk = j; kk < kGemmKS / 16; kk += kGemmIssuers) {
+        // A (MN-major): 16 K rows per MMA = 2 swizzle atoms of 1024 B; M chunks KS * 128 B apart.
+        const uint64_t adesc = sdesc_sw128(sa + kk * 2048, kGemmKS * 128, 1024);
+        // B (K-major): slab kk / 4 of nt rows x 128 B; 16 K elements = 32 B into each row.
+        const uint64_t bdesc = sdesc_sw128(sb + (kk >> 2) * nt * 128 + (kk & 3) * 32, 16, 1024);
+        umma_bf16_ss(acc, adesc, bdesc, idesc, first ? 0u : 1u);
+        first = false;
       }
       umma_commit(&empty[s]);
     }
     umma_commit(done);  // also fires when nothing was issued, so the epilogue never waits forever
   } else if (warp < 4) {
-    // ---------------- epilogue: TMEM -> registers -> bf16 global
+    // ---------------- epilogue: TMEM -> registers -> bf16, staged through shared memory
+    // Warp w owns outputs m0 + 32w + [0, 32) for every n of the tile.  Lane = m in TMEM, so the
+    // warp's [n][32 m] block goes through a stage in the (now idle) operand ring: each lane writes
+    // its column, then every global store instruction covers eight whole 64-byte rows.
     const bool ok = mbar_wait(done, 0);
     tc_fence_after();
     if (ok && !*reinterpret_cast<volatile int*>(abort_flag)) {
-      const int m = m0 + warp * 32 + lane;
       const uint32_t trow = tmem_d + (static_cast<uint32_t>(warp * 32) << 16);
-      __nv_bfloat16* o = out + static_cast<int64_t>(h) * out_hstride + m;
+      __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem + warp * nt * 64);
       for (int c = 0; c < nt; c += 16) {
-        uint32_t r[16];
-        tmem_ld16(trow + c, r);
+        uint32_t r0[16], r1[16];
+        tmem_ld16(trow + c, r0);
+        tmem_ld16(trow + acc_cols + c, r1);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int n = n0 + c + i;
-          if (n < batch) o[static_cast<int64_t>(n) * out_bstride] = __float2bfloat16_rn(__uint_as_float(r[i]));
+        for (int i = 0; i < 16; ++i)
+          stage[(c + i) * 32 + lane] = __float2bfloat16_rn(__uint_as_float(r0[i]) + __uint_as_float(r1[i]));
+      }
+      __syncwarp();
+      const int q = lane & 3;   // 16-byte piece (8 outputs) of a 64-byte row
+      for (int n8 = 0; n8 < nt; n8 += 8) {
+        const int nl = n8 + (lane >> 2);
+        const int n = n0 + nl;
+        if (n < batch) {
+          const uint4 v = *reinterpret_cast<const uint4*>(stage + nl * 32 + 8 * q);
+          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * out_bstride + static_cast<int64_t>(h) * out_hstride +
+                                    m0 + warp * 32 + 8 * q) = v;
         }
       }
     }

@@ -73,18 +73,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D bf16 tensor map, 128-byte swizzle; inner is the contiguous dimension.
-bool make_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                 uint32_t box_inner, uint32_t box_outer) {
+// Generic 3-D bf16 view (dims[0] must be 64 elements = one 128-byte swizzle row), 128-byte swizzle.
+bool make_map_3d(CUtensorMap* map, const void* base, const cuuint64_t (&dims)[3], const cuuint64_t (&strides)[2],
+                 const cuuint32_t (&box)[3]) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -245,15 +242,24 @@ namespace {
 template <int KTOT, int NSTAGE>
 mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, int batch, __nv_bfloat16* out,
                             int64_t out_bstride, int out_hstride, cudaStream_t stream) {
-  // Weight viewed as [heads * KTOT rows][m_total cols]; activation as [batch rows][heads * KTOT cols].
+  // Weight viewed as [heads * KTOT rows][m_total cols]: 3-D (64-element M chunk, row, M chunk index),
+  // box {64, KS, 2}.  Activation as [batch rows][heads * KTOT cols]: 3-D (64-element K slab, batch
+  // row, slab index), box {64, nt, KS / 64}.
   const int nt = batch >= 256 ? 256 : ((batch + 15) / 16) * 16;
+  const uint64_t krows = static_cast<uint64_t>(mla::kHeads) * KTOT;
   CUtensorMap ta, tb;
-  if (!make_map_2d(&ta, weight, m_total, static_cast<uint64_t>(mla::kHeads) * KTOT,
-                   static_cast<uint64_t>(m_total) * 2, 64, 64))
-    return MLA_ERR_CUDA;
-  if (!make_map_2d(&tb, act, static_cast<uint64_t>(mla::kHeads) * KTOT, batch,
-                   static_cast<uint64_t>(mla::kHeads) * KTOT * 2, 64, nt))
-    return MLA_ERR_CUDA;
+  {
+    const cuuint64_t dims[3] = {64, krows, static_cast<cuuint64_t>(m_total / 64)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(m_total) * 2, 128};
+    const cuuint32_t box[3] = {64, mla::kGemmKS, 2};
+    if (!make_map_3d(&ta, weight, dims, strides, box)) return MLA_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(batch), krows / 64};
+    const cuuint64_t strides[2] = {krows * 2, 128};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(nt), mla::kGemmKS / 64};
+    if (!make_map_3d(&tb, act, dims, strides, box)) return MLA_ERR_CUDA;
+  }
   const size_t smem = 1024 + NSTAGE * mla::gemm_stage_bytes(nt) + (2 * NSTAGE + 1) * 8 + 16;
   auto kern = mla::proj_gemm_kernel<KTOT, NSTAGE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
@@ -277,7 +283,7 @@ mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int3
   if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(w_uk) || !aligned16(q_full)) return MLA_ERR_INVALID_ARG;
   if (q_pos != nullptr && (!(rope_base > 0.f) || !std::isfinite(rope_base))) return MLA_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
-  mla_status st = launch_proj_gemm<mla::kDHead, 2>(w_uk, mla::kDLat, q_nope, batch,
+  mla_status st = launch_proj_gemm<mla::kDHead, 1>(w_uk, mla::kDLat, q_nope, batch,
                                                    reinterpret_cast<__nv_bfloat16*>(q_full),
                                                    static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow, s);
   if (st != MLA_OK) return st;
@@ -292,7 +298,7 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
   if (batch == 0) return MLA_OK;
   if (out_lat == nullptr || w_uv == nullptr || out == nullptr) return MLA_ERR_INVALID_ARG;
   if (!aligned16(out_lat) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
-  return launch_proj_gemm<mla::kDLat, 4>(w_uv, mla::kDHead, out_lat, batch, reinterpret_cast<__nv_bfloat16*>(out),
+  return launch_proj_gemm<mla::kDLat, 2>(w_uv, mla::kDHead, out_lat, batch, reinterpret_cast<__nv_bfloat16*>(out),
                                          static_cast<int64_t>(mla::kHeads) * mla::kDHead, mla::kDHead,
                                          as_stream(stream));
 }
