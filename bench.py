@@ -244,7 +244,7 @@ def setup_replica(name, device):
         layers = [_layer_on_device(name, l, device) for l in range(n_layers)]
     last = np.asarray(lens, np.int32) - 1
     base = layers[0]["caches"][0]
-    splits = int(w.get("splits", 0))
+    splits = 0   # the auto work plan (ranges = resident CTA pairs)
     ws_bytes = m.decode_workspace_size(B, base.capacity(), splits)
     st = dict(B=B, lens=lens, w=w, layers=layers, splits=splits,
               n_splits=m.decode_num_splits(B, base.capacity(), splits),
@@ -479,7 +479,7 @@ def run_ours(args, rank, world, local_rank):
                                                      "N(0,1/512) weights)",
         "config": {"workload": args.workload, "batch": st["B"], "seq_len": int(np.max(st["lens"])),
                    "layers": n_layers, "tokens_per_layer": tokens // n_layers, "paged": bool(st["w"]["paged"]),
-                   "splits": st["n_splits"],
+                   "work_ranges": st["n_splits"],
                    "l2": "inputs larger than L2: %d cache cop%s rotated, %.0f MB each" % (
                        len(st["layers"][0]["caches"]) * n_layers, "y" if n_layers * len(st["layers"][0]["caches"]) == 1 else "ies",
                        cache_bytes / n_layers / 1e6),

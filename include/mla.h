@@ -112,35 +112,41 @@ mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int3
                         void* stream);
 
 /*
- * Number of KV splits the decode uses for this problem when num_splits == 0 (auto), or
- * num_splits itself when it is positive (clamped to [1, 1024]).  Depends only on its arguments
- * and the device's SM count.
+ * Number of work ranges P (one CTA pair each) the decode divides the batch's cached tokens into:
+ * for num_splits == 0 (auto) as many as the device keeps resident, but at most one per two
+ * 128-token tiles of batch x max_seq_len; num_splits itself when it is positive (clamped to
+ * [1, 1024]).  Depends only on its arguments and the device.
  */
 int32_t mla_decode_num_splits(int32_t batch, int32_t max_seq_len, int32_t num_splits);
 
 /*
- * Bytes of workspace mla_decode_attn needs: split partials O [batch, S, 128, 512] fp32 plus
- * (m, l) [batch, S, 128] fp32 each, with S = mla_decode_num_splits(batch, max_seq_len, num_splits).
+ * Bytes of workspace mla_decode_attn needs, with P = mla_decode_num_splits(batch, max_seq_len,
+ * num_splits): range partials O [2P, 128, 512] fp32 and (m, l) [2P, 128] fp32 each, then the
+ * per-sequence tile offsets [batch + 1] int32 (rounded up to 16 bytes).
  */
 size_t mla_decode_workspace_size(int32_t batch, int32_t max_seq_len, int32_t num_splits);
 
 /*
  * (3) Decode attention over the latent cache — [DR] §2.3/§2.4: score = scale * (q_abs.c + q_pe.k^R),
  *     the sum of the content and position channels; out_lat = softmax-weighted sum of c.
- * Split-KV flash decoding: sequence b's tokens [0, seq_lens[b]) are cut into S ranges whose
- * bounds depend only on seq_lens[b] and S; each range keeps a running max m and sum l
- * (online softmax) and writes an unnormalised partial; a combine merges the partials in
- * ascending split order:
- *     out_lat[b, h, :] = sum_s e^{m_s - M} O_s / sum_s e^{m_s - M} l_s,   M = max_s m_s
- *     lse[b, h]        = M + log(sum_s e^{m_s - M} l_s)                    (natural log)
+ * Split-KV flash decoding over balanced work ranges: every sequence is cut into 128-token tiles,
+ * the tiles of the batch are laid end to end, and P ranges take equal shares
+ * ([floor(pT/P), floor((p+1)T/P)) of the T tiles), so a range may span several sequences and a
+ * sequence several ranges.  Each part of a sequence a range covers keeps a running max m and sum
+ * l (online softmax); a sequence covered by one range is finished by the decode kernel, the
+ * others' unnormalised partials are merged by a combine in ascending range order:
+ *     out_lat[b, h, :] = sum_r e^{m_r - M} O_r / sum_r e^{m_r - M} l_r,   M = max_r m_r
+ *     lse[b, h]        = M + log(sum_r e^{m_r - M} l_r)                    (natural log)
+ * The ranges depend only on seq_lens and P.
  *   q_full   [batch, 128, 576] bf16     cache / block_table per desc     seq_lens [batch] int32
- *   softmax_scale: e.g. 1/sqrt(192)     num_splits: 0 = auto, else forced
+ *   softmax_scale: e.g. 1/sqrt(192)     num_splits: work ranges P, 0 = auto, else forced
  *   workspace: >= mla_decode_workspace_size(batch, desc.max_seq_len or capacity, num_splits) bytes,
  *              16-byte aligned, contents need not be initialised (fully overwritten)
  *   out_lat  [batch, 128, 512] bf16 (written)    lse [batch, 128] fp32 (written) or NULL
  * The result for a sequence does not depend on the cache layout: paged and contiguous caches
  * holding the same rows give bit-identical outputs.  A sequence with seq_len == 0 yields
  * out_lat = 0 and lse = -inf.  seq_len > capacity sets MLA_DEVERR_SEQLEN_RANGE and is clamped.
+ * batch must be <= 16384 (MLA_ERR_UNSUPPORTED otherwise).
  */
 mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
                            const int32_t* seq_lens, mla_cache_desc desc, int32_t batch,
@@ -153,10 +159,11 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
  * For callers that cannot obtain device memory at decode time, for example a plugin inside a
  * host engine that owns every device allocation, or a fixed-budget deployment that forbids
  * cudaMalloc after start-up.  Same arguments, result and checks as mla_decode_attn, except that
- * the split partials live in a library-owned static device buffer of MLA_NOALLOC_SCRATCH_BYTES
- * (32 MiB) that every GPU which loads the library holds until the process exits.
+ * the range partials live in a library-owned static device buffer of MLA_NOALLOC_SCRATCH_BYTES
+ * (48 MiB: room for the 2 x 74 partials of the auto plan on a 148-SM device) that every GPU which
+ * loads the library holds until the process exits.
  *   - Returns MLA_ERR_WORKSPACE, launching nothing, when mla_decode_workspace_size(batch,
- *     capacity, num_splits) exceeds MLA_NOALLOC_SCRATCH_BYTES (use fewer splits or a smaller batch).
+ *     capacity, num_splits) exceeds MLA_NOALLOC_SCRATCH_BYTES (use fewer ranges).
  *   - The first call on a device looks up the buffer's device address (once per device, with that
  *     device current); make that first call before any stream capture.
  *   - All calls share the one buffer: calls whose kernels overlap on the GPU (different streams,
@@ -164,7 +171,7 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
  *     contents; nothing in it needs to start at zero (the kernels overwrite what they read).
  *   - Calls no allocation routine (cudaMalloc, cudaFree, or a library allocator).
  */
-#define MLA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+#define MLA_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
 mla_status mla_decode_attn_noalloc(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
                                    const int32_t* seq_lens, mla_cache_desc desc, int32_t batch,
                                    float softmax_scale, int32_t num_splits, mla_bf16* out_lat, float* lse,

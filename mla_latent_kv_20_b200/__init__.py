@@ -127,14 +127,14 @@ def decode_attn(q_full, cache, seq_lens, desc: CacheDesc, workspace, out_lat, *,
                                _stream(stream)), "mla_decode_attn")
 
 
-NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
 
 
 def decode_attn_noalloc(q_full, cache, seq_lens, desc: CacheDesc, out_lat, *, lse=None, block_table=None,
                         softmax_scale: float = 1.0 / 192 ** 0.5, num_splits: int = 0, stream=None,
                         batch: int | None = None):
     """mla_decode_attn without a workspace: for callers that cannot allocate device memory at
-    decode time; split partials go to the library's static 32 MiB device buffer."""
+    decode time; range partials go to the library's static 48 MiB device buffer."""
     b = q_full.shape[0] if batch is None else batch
     _check(lib.mla_decode_attn_noalloc(_ptr(q_full), _ptr(cache), _ptr(block_table), _ptr(seq_lens), desc, b,
                                        softmax_scale, num_splits, _ptr(out_lat), _ptr(lse), _stream(stream)),

@@ -1,10 +1,24 @@
-// decode_common.cuh — split-KV plan and the cross-split combine.
+// decode_common.cuh — work plan of the split decode and the cross-range combine.
 //
 // Split-KV flash decoding (not on the pages; the standard exact identity of the softmax): the
-// tokens of a sequence are cut into S ranges; each range yields an unnormalised partial
-// (O_s = sum_t e^{s_t - m_s} c_t, m_s, l_s = sum_t e^{s_t - m_s}); the partials merge exactly.
+// tokens of a sequence are cut into ranges; each range yields an unnormalised partial
+// (O_r = sum_t e^{s_t - m_r} c_t, m_r, l_r = sum_t e^{s_t - m_r}); the partials merge exactly.
 // Scores are carried in the log2 domain (scale * log2(e) folded into one factor) so the kernels
 // use exp2; lse is converted back to the natural log at the end.
+//
+// Work plan.  Every sequence is cut into 128-token tiles (the last one ragged); T = total tiles.
+// P work ranges (one CTA pair each) share them in one of two ways:
+//  * per sequence (when every non-empty sequence has at least T / P tiles): sequence b gets
+//    r_b = floor(P tiles_b / T) >= 1 ranges that split its tiles evenly, so every range holds one
+//    piece of one sequence (pairs beyond sum r_b stay idle);
+//  * balanced (otherwise): the tiles of the batch are laid end to end (sequence b owns global
+//    tiles [off_b, off_b + tiles_b)) and range p takes [floor(p T / P), floor((p + 1) T / P));
+//    the part of each sequence a range touches is a segment.
+// A segment that covers its whole sequence is finished by the decode kernel; otherwise (in the
+// balanced plan at most the first and the last segment of a range) its partial goes to
+// workspace slot 2p (the range's first segment) or 2p + 1 (its last) and the combine merges the
+// partials of the sequence in ascending range order.  The plan depends only on the sequence
+// lengths and P, so paged and contiguous caches with equal lengths use the same ranges.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -13,42 +27,36 @@
 
 namespace mla {
 
-// Tokens per split for a sequence of length L cut into at most S ranges: ceil(L/S) rounded up
-// to `align` (the decode kernel's tile).  Depends only on L, S and align, so paged and
-// contiguous caches with the same lengths use identical ranges.
-__host__ __device__ __forceinline__ int split_chunk(int L, int S, int align) {
-  const int per = (L + S - 1) / S;
-  return ((per + align - 1) / align) * align;
-}
-__host__ __device__ __forceinline__ int splits_used(int L, int S, int align) {
-  if (L <= 0) return 0;
-  const int c = split_chunk(L, S, align);
-  return (L + c - 1) / c;
-}
-
-constexpr int kSplitAlign = 128;  // split boundaries are multiples of this many tokens
+constexpr int kTile = 128;               // tokens per tile of the work plan and of the decode kernel
+constexpr int kMaxDecodeBatch = 16384;   // sequences per decode call (the plan's prefix fits in smem)
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Workspace layout for `batch` sequences and S splits:
-//   O  [batch][S][128][512] fp32   (unnormalised partial sums of c)
-//   m  [batch][S][128]      fp32   (running max, log2 domain)
-//   l  [batch][S][128]      fp32   (running sum of exp2(s - m))
+// Workspace layout for P work ranges and `batch` sequences:
+//   O    [2P][128][512] fp32   (unnormalised partial sums of c)
+//   m    [2P][128]      fp32   (running max, log2 domain)
+//   l    [2P][128]      fp32   (running sum of exp2(s - m))
+//   plan [batch + 2]    int32  (balanced: global tile offset of each sequence, [batch] = T;
+//                               per sequence: first range of each sequence, [batch] = ranges used;
+//                               [batch + 1] = the plan kind)
 struct Workspace {
   float* o;
   float* m;
   float* l;
+  int32_t* off;
 };
-__host__ __device__ __forceinline__ Workspace ws_carve(void* base, int batch, int S) {
+__host__ __device__ __forceinline__ Workspace ws_carve(void* base, int P) {
   Workspace w;
   w.o = reinterpret_cast<float*>(base);
-  w.m = w.o + static_cast<int64_t>(batch) * S * kHeads * kDLat;
-  w.l = w.m + static_cast<int64_t>(batch) * S * kHeads;
+  w.m = w.o + static_cast<int64_t>(2 * P) * kHeads * kDLat;
+  w.l = w.m + static_cast<int64_t>(2 * P) * kHeads;
+  w.off = reinterpret_cast<int32_t*>(w.l + static_cast<int64_t>(2 * P) * kHeads);
   return w;
 }
-__host__ __device__ __forceinline__ size_t ws_bytes(int batch, int S) {
-  return static_cast<size_t>(batch) * S * kHeads * (kDLat + 2) * sizeof(float);
+__host__ __device__ __forceinline__ size_t ws_bytes(int batch, int P) {
+  const size_t partials = static_cast<size_t>(2 * P) * kHeads * (kDLat + 2) * sizeof(float);
+  return partials + ((static_cast<size_t>(batch) + 2) * sizeof(int32_t) + 15) / 16 * 16;
 }
 
 // Effective length of sequence b: seq_lens[b] clamped to [0, capacity] (error word set if it
@@ -61,34 +69,110 @@ __device__ __forceinline__ int seq_len_checked(const int32_t* seq_lens, int b, i
   }
   return L;
 }
+__host__ __device__ __forceinline__ int tiles_of(int L) { return (L + kTile - 1) / kTile; }
 
-// Combine: one warp per (b, h); lanes own 16 of the 512 latent columns.  Splits are merged in
-// ascending order.  grid = (batch, 128 / 4), block = 128.
-// Sequences whose tokens fit in one split were finalised by the decode kernel itself
-// (`single_done`); the combine only writes empty sequences (out_lat = 0, lse = -inf) and merges
-// sequences with two or more used splits.
-__global__ void __launch_bounds__(128) combine_kernel(Workspace ws, const int32_t* __restrict__ seq_lens, int S,
-                                                      int align, int capacity, int single_done,
-                                                      __nv_bfloat16* __restrict__ out_lat,
+// floor(x y / z) for x, y >= 0 and z > 0, exact; 32-bit arithmetic when x y fits.
+__host__ __device__ __forceinline__ int muldiv(int x, int y, int z) {
+  const uint64_t p = static_cast<uint64_t>(x) * static_cast<uint32_t>(y);
+  if (p <= 0xffffffffull) return static_cast<int>(static_cast<uint32_t>(p) / static_cast<uint32_t>(z));
+  return static_cast<int>(p / static_cast<uint32_t>(z));
+}
+
+// First global tile of work range p (of P) over T tiles.
+__host__ __device__ __forceinline__ int range_start(int p, int P, int T) { return muldiv(p, T, P); }
+// The (non-empty) range that holds global tile t: the last p with range_start(p) <= t.
+__host__ __device__ __forceinline__ int range_of_tile(int t, int P, int T) {
+  return static_cast<int>(((static_cast<int64_t>(t) + 1) * P + T - 1) / T) - 1;
+}
+
+constexpr int kPlanBalanced = 0;
+constexpr int kPlanPerSequence = 1;
+
+// One segment of a work range: tokens [tok_begin, tok_end) of sequence b.
+struct Segment {
+  int b;
+  int tok_begin;
+  int tok_end;
+  int n_tiles;
+  bool direct;   // covers the whole sequence: the decode kernel writes the final output
+  int slot;      // workspace slot of the partial otherwise
+};
+
+// Walks the segments of one work range in order.  Every role of a CTA walks the same sequence.
+struct SegmentCursor {
+  int b;       // next sequence to look at
+  int off;     // its tile offset (global in the balanced plan, 0 in the per-sequence plan)
+  int start;   // the range's tiles [start, end) in the same frame
+  int end;
+  int b_end;   // sequences [b, b_end) may hold segments
+  int pair;
+  bool first;
+  int len0;    // length of the first sequence b (known from the plan: no memory read on the way in)
+
+  // False only if next() will return false (true may still be followed by no segment).
+  __device__ bool may_continue() const { return b < b_end && off < end; }
+
+  __device__ bool next(const int32_t* seq_lens, int capacity, Segment& s) {
+    while (b < b_end && off < end) {
+      const int L = first ? len0 : seq_len_checked(seq_lens, b, capacity);
+      const int tiles = tiles_of(L);
+      const int t0 = (start > off ? start : off) - off;
+      const int t1 = (end < off + tiles ? end : off + tiles) - off;
+      const int cur = b;
+      off += tiles;
+      ++b;
+      if (t1 > t0) {
+        s.b = cur;
+        s.tok_begin = t0 * kTile;
+        s.tok_end = min(t1 * kTile, L);
+        s.n_tiles = t1 - t0;
+        s.direct = t0 == 0 && t1 == tiles;
+        s.slot = first ? 2 * pair : 2 * pair + 1;
+        first = false;
+        return true;
+      }
+    }
+    return false;
+  }
+};
+
+// Combine: one warp per (b, h); lanes own 16 of the 512 latent columns.  grid = (batch, 128 / 4),
+// block = 128.  Empty sequences get out_lat = 0 and lse = -inf; sequences finished by the decode
+// kernel (one segment) are skipped; the others merge their partials in ascending range order.
+__global__ void __launch_bounds__(128) combine_kernel(Workspace ws, int P, __nv_bfloat16* __restrict__ out_lat,
                                                       float* __restrict__ lse) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x;
   const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  int L = seq_lens[b];
-  L = L < 0 ? 0 : (L > capacity ? capacity : L);
-  const int n = splits_used(L, S, align);
-  if (n == 1 && single_done) return;
-  const int64_t base = static_cast<int64_t>(b) * S * kHeads;
+  const int B = gridDim.x;
+  const bool per_seq = ws.off[B + 1] == kPlanPerSequence;
+  const int T = ws.off[B];
+  const int off = ws.off[b];
+  const int span = ws.off[b + 1] - off;   // tiles (balanced) or ranges (per sequence) of b
+  __nv_bfloat16* dst = out_lat + (static_cast<int64_t>(b) * kHeads + h) * kDLat;
+  if (span == 0) {
+    for (int i = lane; i < kDLat / 8; i += 32) reinterpret_cast<uint4*>(dst)[i] = make_uint4(0, 0, 0, 0);
+    if (lse != nullptr && lane == 0) lse[static_cast<int64_t>(b) * kHeads + h] = -INFINITY;
+    return;
+  }
+  // Ranges [p0, p1] that hold pieces of b; in the per-sequence plan each holds one (slot 2p).
+  const int p0 = per_seq ? off : range_of_tile(off, P, T);
+  const int p1 = per_seq ? off + span - 1 : range_of_tile(off + span - 1, P, T);
+  if (p0 == p1) return;
+  auto slot_of = [&](int p) { return (!per_seq && range_start(p, P, T) < off) ? 2 * p + 1 : 2 * p; };
+  auto nonempty = [&](int p) { return per_seq || range_start(p, P, T) < range_start(p + 1, P, T); };
   float M = -INFINITY;
-  for (int s = 0; s < n; ++s) M = fmaxf(M, ws.m[base + static_cast<int64_t>(s) * kHeads + h]);
+  for (int p = p0; p <= p1; ++p)
+    if (nonempty(p)) M = fmaxf(M, ws.m[static_cast<int64_t>(slot_of(p)) * kHeads + h]);
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
   float den = 0.f;
-  for (int s = 0; s < n; ++s) {
-    const int64_t ml = base + static_cast<int64_t>(s) * kHeads + h;
+  for (int p = p0; p <= p1; ++p) {
+    if (!nonempty(p)) continue;
+    const int64_t ml = static_cast<int64_t>(slot_of(p)) * kHeads + h;
     const float w = exp2f(ws.m[ml] - M);
     den += w * ws.l[ml];
     const float4* o = reinterpret_cast<const float4*>(ws.o + ml * kDLat);
@@ -102,7 +186,6 @@ __global__ void __launch_bounds__(128) combine_kernel(Workspace ws, const int32_
     }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
-  __nv_bfloat16* dst = out_lat + (static_cast<int64_t>(b) * kHeads + h) * kDLat;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     __nv_bfloat162 lo = __floats2bfloat162_rn(acc[4 * i + 0] * inv, acc[4 * i + 1] * inv);

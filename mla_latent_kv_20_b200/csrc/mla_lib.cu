@@ -306,19 +306,16 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
 int32_t mla_decode_num_splits(int32_t batch, int32_t max_seq_len, int32_t num_splits) {
   if (num_splits > 0) return num_splits > kMaxSplits ? kMaxSplits : num_splits;
   if (batch <= 0 || max_seq_len <= 0) return 1;
-  // Each (sequence, split) is one CTA pair, and every extra split costs an fp32 partial of
-  // 128 x 514 floats written and read back (about 460 cached tokens' worth of traffic).  Use the
-  // fewest splits whose pairs cover at least 80 % of the resident pair slots, keeping at least
-  // two 128-token tiles per split.
+  // Work ranges = CTA pairs.  The ranges split the batch's tiles evenly, so as many ranges as pairs
+  // can be resident keep every SM busy; an upper bound on the tiles (every sequence at capacity)
+  // keeps at least two tiles per range so each pair's start-up is amortised.  The plan itself uses
+  // the true lengths on the device.
   const int slots = decode_cluster_slots();
-  int s_max = (max_seq_len + 2 * mla::kTcTile - 1) / (2 * mla::kTcTile);
-  if (s_max < 1) s_max = 1;
-  if (s_max > kMaxSplits) s_max = kMaxSplits;
-  const long long want = (4LL * slots + 4) / 5;
-  int s = static_cast<int>((want + batch - 1) / batch);
-  if (s < 1) s = 1;
-  if (s > s_max) s = s_max;
-  return s;
+  const long long tiles_max = static_cast<long long>(batch) * ((max_seq_len + mla::kTile - 1) / mla::kTile);
+  long long p = (tiles_max + 1) / 2;
+  if (p > slots) p = slots;
+  if (p > kMaxSplits) p = kMaxSplits;
+  return p < 1 ? 1 : static_cast<int32_t>(p);
 }
 
 size_t mla_decode_workspace_size(int32_t batch, int32_t max_seq_len, int32_t num_splits) {
@@ -331,7 +328,7 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
                            int32_t num_splits, void* workspace, size_t workspace_bytes, mla_bf16* out_lat,
                            float* lse, void* stream) {
   if (batch < 0 || num_splits < 0) return MLA_ERR_INVALID_ARG;
-  if (batch > kMaxBatch) return MLA_ERR_UNSUPPORTED;
+  if (batch > mla::kMaxDecodeBatch) return MLA_ERR_UNSUPPORTED;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
   CacheView v;
   const mla_status st = check_cache(desc, cache, block_table, &v);
@@ -341,8 +338,8 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
   if (q_full == nullptr || seq_lens == nullptr || out_lat == nullptr) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_full) || !aligned16(out_lat) || (lse != nullptr && !aligned16(lse))) return MLA_ERR_INVALID_ARG;
   const int capacity = cache_capacity(desc);
-  const int S = mla_decode_num_splits(batch, capacity, num_splits);
-  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < mla::ws_bytes(batch, S))
+  const int P = mla_decode_num_splits(batch, capacity, num_splits);
+  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < mla::ws_bytes(batch, P))
     return MLA_ERR_WORKSPACE;
   if (desc.num_rows >= (int64_t(1) << 31) || static_cast<int64_t>(batch) * mla::kHeads >= (int64_t(1) << 31))
     return MLA_ERR_UNSUPPORTED;
@@ -350,9 +347,11 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
   mla::DecodeTcArgs a;
   a.v = v;
   a.seq_lens = seq_lens;
-  a.S = S;
+  a.batch = batch;
+  a.capacity = capacity;
+  a.P = P;
   a.scale_log2 = softmax_scale * mla::kLog2e;
-  a.ws = mla::ws_carve(workspace, batch, S);
+  a.ws = mla::ws_carve(workspace, P);
   a.out_lat = reinterpret_cast<__nv_bfloat16*>(out_lat);
   a.lse = lse;
   a.cache = reinterpret_cast<const uint8_t*>(cache);
@@ -364,11 +363,11 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
   if (cudaFuncSetAttribute(mla::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kTcSmemBytes) !=
       cudaSuccess)
     return MLA_ERR_CUDA;
-  mla_status ls = launch_chained(mla::decode_tc_kernel, dim3(2 * S, batch), dim3(mla::kTcThreads),
+  mla_status ls = launch_chained(mla::decode_tc_kernel, dim3(2 * P), dim3(mla::kTcThreads),
                                  static_cast<size_t>(mla::kTcSmemBytes), s, tka, tkb, tv, tq, a);
   if (ls != MLA_OK) return ls;
-  return launch_chained(mla::combine_kernel, dim3(batch, mla::kHeads / 4), dim3(128), 0, s, a.ws, seq_lens, S,
-                        mla::kSplitAlign, capacity, /*single_done=*/1, reinterpret_cast<__nv_bfloat16*>(out_lat), lse);
+  return launch_chained(mla::combine_kernel, dim3(batch, mla::kHeads / 4), dim3(128), 0, s, a.ws, P,
+                        reinterpret_cast<__nv_bfloat16*>(out_lat), lse);
 }
 
 }  // extern "C"

@@ -85,7 +85,12 @@ def test_decode_validation_and_workspace(mla):
     S = lib.mla_decode_num_splits(8, 4096, 16)
     assert S == 16 and lib.mla_decode_num_splits(8, 4096, 5000) == 1024
     need = lib.mla_decode_workspace_size(8, 4096, 16)
-    assert need == 8 * 16 * 128 * (512 + 2) * 4
+    assert need == 2 * 16 * 128 * (512 + 2) * 4 + 48     # partials of 16 ranges + 9 tile offsets, 16-B rounded
+    # auto: at most one range per two 128-token tiles of batch x max_seq_len (the resident-pair
+    # bound is 74 without a device to ask)
+    assert lib.mla_decode_num_splits(1, 256, 0) == 1
+    assert lib.mla_decode_num_splits(2, 1000, 0) == 8
+    assert lib.mla_decode_num_splits(8, 4096, 0) == 74
     args = lambda ws, nbytes, scale=0.072, batch=8, splits=16, desc=d: (  # noqa: E731
         FAKE, FAKE, None, FAKE, desc, batch, scale, splits, ws, nbytes, FAKE, None, None)
     assert lib.mla_decode_attn(*args(FAKE, need - 16)) == 3           # workspace too small
@@ -94,4 +99,6 @@ def test_decode_validation_and_workspace(mla):
     assert lib.mla_decode_attn(*args(FAKE, need, batch=9)) == 1       # batch > num_seqs
     assert lib.mla_decode_attn(*args(FAKE, need, batch=0)) == 0       # empty batch is a no-op
     assert lib.mla_decode_attn(*args(FAKE, need, splits=-1)) == 1
+    big = mla.contiguous_desc(16385, 64)
+    assert lib.mla_decode_attn(*args(FAKE, 1 << 40, batch=16385, desc=big)) == 2   # batch beyond the plan's limit
     assert lib.mla_get_device_error(None) == 1

@@ -1,6 +1,6 @@
-"""Parity at the full workload sizes, in the launch configuration bench.py times (auto split count,
-or the forced 128 splits of the long-context workload), checked on sampled sequences that the
-fp64 oracle computes one by one."""
+"""Parity at the full workload sizes, in the launch configuration bench.py times (the auto work
+plan), or with 128 forced work ranges for the long-context workload (so each of its sequences is
+merged from 32 partials), checked on sampled sequences that the fp64 oracle computes one by one."""
 import numpy as np
 import pytest
 
@@ -27,7 +27,7 @@ def _run_workload(name, sample, explicit_first=True):
     qpos = torch.from_numpy(np.asarray(lens, np.int32) - 1).cuda()
     out, out_lat, lse, _ = hz.decode_step(hz.bf16_tensor(batch.q_nope), hz.bf16_tensor(batch.q_pe),
                                           hz.bf16_tensor(wts.w_uk), hz.bf16_tensor(wts.w_uv), cache,
-                                          q_pos=qpos, num_splits=int(w.get("splits", 0)))
+                                          q_pos=qpos, num_splits=int(w.get("test_ranges", 0)))
     torch.cuda.synchronize()
     assert get_device_error() == 0
     g_out = f64(hz.bf16_bits(out))
@@ -55,7 +55,7 @@ def test_b128_paged_uniform_lengths():
     _run_workload("b128_u1024_8192_paged", [int(np.argmin(lens)), int(np.argmax(lens)), 64])
 
 
-def test_b4_l131072_128_splits():
+def test_b4_l131072_128_ranges():
     _run_workload("b4_l131072", [2], explicit_first=False)
 
 

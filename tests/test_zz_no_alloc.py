@@ -2,7 +2,7 @@
 
 Some callers cannot obtain device memory while decoding: a plugin running inside a host engine
 that owns every device allocation, or a fixed-budget deployment that forbids cudaMalloc after
-start-up.  For them the library keeps the split partials in its own static 32 MiB device
+start-up.  For them the library keeps the range partials in its own static 48 MiB device
 buffer.  These tests call that entry point through the C ABI and check it against the
 workspace-taking entry point, on two calls in a row with different inputs (the shared buffer
 keeps the previous call's contents, which must not matter), and check that a problem whose
