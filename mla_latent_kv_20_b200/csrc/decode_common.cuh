@@ -71,18 +71,23 @@ __device__ __forceinline__ int seq_len_checked(const int32_t* seq_lens, int b, i
 }
 __host__ __device__ __forceinline__ int tiles_of(int L) { return (L + kTile - 1) / kTile; }
 
-// floor(x y / z) for x, y >= 0 and z > 0, exact; 32-bit arithmetic when x y fits.
+// floor(x y / z) for x, y >= 0 and z > 0, exact; 32-bit arithmetic when x y fits (the wide
+// division is out of line: it is rarely taken and its code is long).
+__host__ __device__ __noinline__ int muldiv_wide(uint64_t p, uint32_t z) { return static_cast<int>(p / z); }
 __host__ __device__ __forceinline__ int muldiv(int x, int y, int z) {
   const uint64_t p = static_cast<uint64_t>(x) * static_cast<uint32_t>(y);
   if (p <= 0xffffffffull) return static_cast<int>(static_cast<uint32_t>(p) / static_cast<uint32_t>(z));
-  return static_cast<int>(p / static_cast<uint32_t>(z));
+  return muldiv_wide(p, static_cast<uint32_t>(z));
 }
 
 // First global tile of work range p (of P) over T tiles.
 __host__ __device__ __forceinline__ int range_start(int p, int P, int T) { return muldiv(p, T, P); }
 // The (non-empty) range that holds global tile t: the last p with range_start(p) <= t.
 __host__ __device__ __forceinline__ int range_of_tile(int t, int P, int T) {
-  return static_cast<int>(((static_cast<int64_t>(t) + 1) * P + T - 1) / T) - 1;
+  // ceil((t + 1) P / T) - 1
+  const uint64_t x = static_cast<uint64_t>(t + 1) * static_cast<uint32_t>(P) + static_cast<uint32_t>(T - 1);
+  if (x <= 0xffffffffull) return static_cast<int>(static_cast<uint32_t>(x) / static_cast<uint32_t>(T)) - 1;
+  return muldiv_wide(x, static_cast<uint32_t>(T)) - 1;
 }
 
 constexpr int kPlanBalanced = 0;

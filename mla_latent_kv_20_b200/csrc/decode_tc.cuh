@@ -165,13 +165,10 @@ __device__ __forceinline__ void tma_load_4d_local(void* dst, const CUtensorMap* 
 //        (zeros); its scores are masked anyway.
 //  V(i): per 64-token half h of the tile, latent [256n + 128r, +128) for n = 0, 1 in one box,
 //        laid out [n][chunk][64 rows][128 B].
-__device__ __forceinline__ void zero_v_rows(uint8_t* box, int v) {
-  for (int q = 0; q < 4; ++q)
-    for (int row = v; row < 64; ++row) {
-      uint4* p = reinterpret_cast<uint4*>(box + q * kTcSlab + row * 128);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) p[u] = make_uint4(0, 0, 0, 0);
-    }
+__device__ __forceinline__ void zero_v_rows(uint8_t* box, int v, int lane) {
+  // each row is 4 slabs x 128 bytes: one 16-byte chunk per lane
+  uint4* p = reinterpret_cast<uint4*>(box + (lane >> 3) * kTcSlab) + (lane & 7);
+  for (int row = v; row < 64; ++row) p[row * 8] = make_uint4(0, 0, 0, 0);
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* ptr) {
@@ -221,13 +218,15 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
       const int64_t nrows = a.v.num_rows - row < 64 ? a.v.num_rows - row : 64;
       const uint8_t* base = a.cache + row * (kDRow * 2);
       const int lines = static_cast<int>(nrows) * (kDRow * 2 / 128);
+#pragma unroll 1
       for (int q = lane; q < lines; q += 32) prefetch_l2(base + q * 128);
     };
     auto issue_k = [&](int i) -> bool {
-      if (i > 0) prefetch_k(i + kTcPrefetchTiles);
+      if (i > 0) prefetch_k(i + kTcPrefetchTiles);   // before the wait: it does not depend on it
       const int gi = g + i;
       const int my0 = t_begin + i * kTcTile + 64 * static_cast<int>(rank);
       const int y = my0 < t_end ? tma_row(a.v, b, my0) : -kTcTile;
+#pragma unroll 1
       for (int part = 0; part < 2; ++part) {
         if (gi >= 1 && !wait0(&bars->k_empty[part], static_cast<uint32_t>(gi - 1) & 1u, 0x10 + part)) return false;
         if (l0) {
@@ -245,6 +244,7 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
       // The V ring doubles as the epilogue's staging buffer: the first box of a segment waits
       // until the previous segment's epilogue (in both CTAs) is done with it.
       if (i == 0 && k > 0 && !wait0(&bars->o_free, static_cast<uint32_t>(k - 1) & 1u, 0x15)) return false;
+#pragma unroll 1
       for (int h = 0; h < 2; ++h, ++vn) {
         const int s = vn % kTcVSlots;
         if (vn >= kTcVSlots && !wait0(&bars->v_empty[s], static_cast<uint32_t>((vn / kTcVSlots) - 1) & 1u, 0x12))
@@ -261,8 +261,9 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
               mbar_arrive_relaxed(lbar(&bars->v_full[s]));
           }
         } else {
-          // Ragged: load through a CTA-local barrier, zero the rows past the end, then publish with
-          // release semantics (the zeros are lane 0's own shared-memory writes).
+          // Ragged: load through a CTA-local barrier, zero the rows past the end (all lanes, after
+          // the copy has landed), then publish: each lane's proxy fence, the warp barrier, and lane
+          // 0's arrival with release semantics.
           if (vcount > 0) {
             if (l0) {
               mbar_arrive_expect_tx(&bars->fix, kTcVBox);
@@ -271,9 +272,11 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
             if (!wait0(&bars->fix, fix_phase, 0x13)) return false;
             fix_phase ^= 1u;
           }
+          __syncwarp();
+          zero_v_rows(box, vcount, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
           if (l0) {
-            zero_v_rows(box, vcount);
-            fence_proxy_async_smem();
             if (leader)
               mbar_arrive_expect_tx_addr(lbar(&bars->v_full[s]), 0u);
             else
@@ -283,10 +286,15 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
       }
       return true;
     };
-    ok = issue_k(0);
-    for (int j = 1; j <= kTcPrefetchTiles; ++j) prefetch_k(j);   // after K(0): it goes out first
-    for (int i = 1; ok && i < n_tiles; ++i) ok = issue_k(i) && issue_v(i - 1);
-    if (ok) ok = issue_v(n_tiles - 1);
+    // K(i) then V(i - 1): one call site each (the loop runs one step past the last K).  The first
+    // prefetches go out after K(0), which goes first.
+    for (int i = 0; ok && i <= n_tiles; ++i) {
+      if (i < n_tiles) ok = issue_k(i);
+      if (i == 0)
+        for (int j = 1; j <= kTcPrefetchTiles; ++j) prefetch_k(j);
+      else if (ok)
+        ok = issue_v(i - 1);
+    }
     g += n_tiles;
     ++k;
   }
@@ -307,18 +315,17 @@ __device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) { retu
 
 // S_part(g) = Q[:, dims of part] . K(g)[:, dims of part]^T into S buffer g & 1 of the part, for
 // every global tile g of the range; Q is reloaded for each segment.
-__device__ bool tc_mma_qk(uint8_t* smem, TcBars* bars, uint32_t tmem, int part, const DecodeTcArgs& a,
-                          const TcPlan& plan, int pair, volatile int* abort_flag) {
+__device__ bool tc_mma_qk(uint8_t* smem, TcBars* bars, uint32_t tmem, int part, const int32_t* seq_lens,
+                          int capacity, SegmentCursor cur, volatile int* abort_flag) {
   const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
   const int slab0 = tc_part_slab0(part);
   const int nslabs = tc_part_slabs(part);
   const uint64_t dq = sdesc_sw128(smem_u32(smem + kTcOffQ + slab0 * kTcSlab), 16, 1024);
   const uint64_t dk = sdesc_sw128(smem_u32(smem + kTcOffK + slab0 * kTcSlab), 16, 1024);
   const uint32_t scol = tmem + (part ? kTcColSB : kTcColSA);
-  SegmentCursor cur{plan.b0, plan.off0, plan.start, plan.end, plan.b_end, pair, true, plan.len0};
   Segment sg;
   int g = 0, k = 0;
-  while (cur.next(a.seq_lens, a.capacity, sg)) {
+  while (cur.next(seq_lens, capacity, sg)) {
     if (!mbar_wait_cluster(&bars->q_full, static_cast<uint32_t>(k) & 1u, 0x20)) return false;
     for (int i = 0; i < sg.n_tiles; ++i, ++g) {
       const int j = g & 1;
@@ -346,16 +353,15 @@ __device__ bool tc_mma_qk(uint8_t* smem, TcBars* bars, uint32_t tmem, int part, 
 // accumulators); every release below therefore counts two commits.  The first V box (tokens
 // 0..63 of the tile) is consumed first so it is released (and refilled) before the second.  The
 // first tile of a segment overwrites O, after the previous segment's epilogue has read it.
-__device__ bool tc_mma_pv(uint8_t* smem, TcBars* bars, uint32_t tmem, int nh, const DecodeTcArgs& a,
-                          const TcPlan& plan, int pair, volatile int* abort_flag) {
+__device__ bool tc_mma_pv(uint8_t* smem, TcBars* bars, uint32_t tmem, int nh, const int32_t* seq_lens,
+                          int capacity, SegmentCursor cur, volatile int* abort_flag) {
   const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
   const uint64_t dp = sdesc_sw128(smem_u32(smem + kTcOffP), 16, 1024);
   const uint64_t dv = sdesc_sw128(smem_u32(smem + kTcOffV), kTcSlab, 1024);
-  SegmentCursor cur{plan.b0, plan.off0, plan.start, plan.end, plan.b_end, pair, true, plan.len0};
   Segment sg;
   int g = 0, k = 0, vn = 0;
   bool ok = true;
-  while (ok && cur.next(a.seq_lens, a.capacity, sg)) {
+  while (ok && cur.next(seq_lens, capacity, sg)) {
     if (k > 0 && !mbar_wait_cluster(&bars->o_free, static_cast<uint32_t>(k - 1) & 1u, 0x25)) {
       ok = false;
       break;
@@ -658,105 +664,107 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
 }
 
 // ------------------------------------------------------------------------------ work plan
-// Block-wide exclusive prefix sum of one int per thread (every thread of the CTA calls it);
-// scratch holds at least 33 ints and is free again on return.
-__device__ void block_scan(int v, int* scratch, int& excl, int& total) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int incl = v;
+// One warp computes the plan; every CTA computes it for itself (it only reads seq_lens), and the
+// even CTA of range 0 also writes the table the combine reads.  Lane l walks the contiguous chunk
+// of sequences [l per, (l + 1) per): three passes over it (tile totals and the smallest sequence;
+// per-chunk sums of the prefix counts; the prefix itself, the table and this pair's piece), with
+// one warp reduction or scan between passes.  Every lane returns the same plan.
+__device__ __forceinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacity, int B, int P, int32_t* table,
+                                               int pair, bool write_table) {
+  const int lane = threadIdx.x & 31;
+  const int per = (B + 31) / 32;
+  const int lo = min(B, lane * per), hi = min(B, lo + per);
+  // pass 1: total tiles T and the smallest non-empty sequence (and the largest)
+  int sum = 0, mn = INT_MAX, mx = 0;
+  for (int bb = lo; bb < hi; ++bb) {
+    const int t = tiles_of(seq_len_checked(seq_lens, bb, capacity));
+    sum += t;
+    mx = max(mx, t);
+    if (t > 0) mn = min(mn, t);
+  }
+  const int T = __reduce_add_sync(0xffffffffu, sum);
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  const bool per_seq = T > 0 && static_cast<int64_t>(mn) * P >= T;
+  if (per_seq && mx == mn && static_cast<int64_t>(mn) * B == T) {
+    // Every sequence has the same tile count t (the usual case): r_b = floor(P t / (B t)) =
+    // floor(P / B) for all b, so the prefix is b r and no scan is needed.  Same plan as below.
+    const int t = mn;
+    const int r = min(P / B, t);
+    if (write_table) {
+      for (int bb = lo; bb < hi; ++bb) table[bb] = bb * r;
+      if (lane == 0) {
+        table[B] = B * r;
+        table[B + 1] = kPlanPerSequence;
+      }
+    }
+    TcPlan pl;
+    pl.start = pl.end = 0;
+    pl.b0 = pl.off0 = pl.b_end = pl.len0 = 0;
+    const int b0 = pair / r, jj = pair - b0 * r;
+    if (b0 < B) {
+      pl.b0 = b0;
+      pl.len0 = seq_len_checked(seq_lens, b0, capacity);
+      pl.start = muldiv(jj, t, r);
+      pl.end = muldiv(jj + 1, t, r);
+      pl.b_end = b0 + 1;
+    }
+    return pl;
+  }
+  // what each sequence contributes to the prefix: its tiles, or (per sequence) its ranges
+  // r_b = floor(P tiles_b / T), which the condition makes >= 1 and which is at most tiles_b
+  auto count_of = [&](int t) -> int {
+    if (!per_seq || t == 0) return t;
+    const int r = muldiv(P, t, T);
+    return r < t ? r : t;
+  };
+  // pass 2: this lane's share of the prefix
+  int csum = sum;
+  if (per_seq) {
+    csum = 0;
+    for (int bb = lo; bb < hi; ++bb) csum += count_of(tiles_of(seq_len_checked(seq_lens, bb, capacity)));
+  }
+  int incl = csum;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const int u = __shfl_up_sync(0xffffffffu, incl, d);
     if (lane >= d) incl += u;
   }
-  if (lane == 31) scratch[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    const int x = lane < nw ? scratch[lane] : 0;
-    int inc = x;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, inc, d);
-      if (lane >= d) inc += u;
-    }
-    if (lane < nw) scratch[lane] = inc - x;
-    if (lane == 31) scratch[32] = inc;
-  }
-  __syncthreads();
-  excl = scratch[w] + incl - v;
-  total = scratch[32];
-  __syncthreads();
-}
-
-// Warp-level inclusive prefix sum.
-__device__ __forceinline__ int warp_incl_scan(int v) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, v, d);
-    if (lane >= d) v += u;
-  }
-  return v;
-}
-
-// The plan of tc_make_plan computed by one warp with shuffles only (batches of up to
-// kWarpPlanMax sequences, the common case), returned to every lane: the warp that computes it
-// (the producer) needs no CTA barrier to start its copies.  Same results as the block-wide version.
-constexpr int kWarpPlanMax = 1024;
-__device__ TcPlan tc_make_plan_warp(const DecodeTcArgs& a, int pair, bool write_table) {
-  const int lane = threadIdx.x & 31;
-  const int B = a.batch;
-  const int P = a.P;
-  // pass 1: total tiles T and the smallest non-empty sequence
-  int T = 0, mn = INT_MAX;
-  for (int c = 0; c < B; c += 32) {
-    const int bb = c + lane;
-    const int t = bb < B ? tiles_of(seq_len_checked(a.seq_lens, bb, a.capacity)) : 0;
-    if (t > 0) mn = min(mn, t);
-    T += __reduce_add_sync(0xffffffffu, t);
-  }
-  mn = __reduce_min_sync(0xffffffffu, mn);
-  const bool per_seq = T > 0 && static_cast<int64_t>(mn) * P >= T;
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  // pass 3: the prefix of each sequence, the table, and the piece of this pair
   const int start_g = T > 0 ? range_start(pair, P, T) : 0;   // the balanced plan's range
   const int end_g = T > 0 ? range_start(pair + 1, P, T) : 0;
   TcPlan pl;
   pl.start = pl.end = 0;
   pl.b0 = pl.off0 = pl.b_end = pl.len0 = 0;
-  // pass 2: prefix (of tiles, or of ranges per sequence) and this pair's piece
-  int run = 0;   // prefix before this chunk
-  for (int c = 0; c < B; c += 32) {
-    const int bb = c + lane;
-    const int L = bb < B ? seq_len_checked(a.seq_lens, bb, a.capacity) : 0;
+  int run = incl - csum;
+  for (int bb = lo; bb < hi; ++bb) {
+    const int L = seq_len_checked(seq_lens, bb, capacity);
     const int t = tiles_of(L);
-    int v = t;
-    if (per_seq && t > 0) {
-      v = muldiv(P, t, T);   // r_b >= 1 by the condition
-      v = v < t ? v : t;
-    }
-    const int incl = warp_incl_scan(v);
-    const int excl = run + incl - v;
-    if (bb < B && write_table) a.ws.off[bb] = excl;
+    const int v = count_of(t);
+    if (write_table) table[bb] = run;
     if (per_seq) {
-      if (v > 0 && excl <= pair && pair < excl + v) {
-        const int jj = pair - excl;
+      if (v > 0 && run <= pair && pair < run + v) {
+        const int jj = pair - run;
         pl.b0 = bb;
         pl.len0 = L;
         pl.start = muldiv(jj, t, v);
         pl.end = muldiv(jj + 1, t, v);
         pl.b_end = bb + 1;
       }
-    } else if (t > 0 && start_g < end_g && excl <= start_g && start_g < excl + t) {
+    } else if (t > 0 && start_g < end_g && run <= start_g && start_g < run + t) {
       pl.b0 = bb;
       pl.len0 = L;
-      pl.off0 = excl;
+      pl.off0 = run;
       pl.start = start_g;
       pl.end = end_g;
       pl.b_end = B;
     }
-    run = __shfl_sync(0xffffffffu, excl + v, 31);
+    run += v;
   }
   if (write_table && lane == 0) {
-    a.ws.off[B] = run;
-    a.ws.off[B + 1] = per_seq ? kPlanPerSequence : kPlanBalanced;
+    table[B] = total;
+    table[B + 1] = per_seq ? kPlanPerSequence : kPlanBalanced;
   }
   // the lane that found the piece (at most one) hands it to the warp; otherwise the pair is idle
   const unsigned found = __ballot_sync(0xffffffffu, pl.end > pl.start);
@@ -769,93 +777,6 @@ __device__ TcPlan tc_make_plan_warp(const DecodeTcArgs& a, int pair, bool write_
   r.b_end = __shfl_sync(0xffffffffu, pl.b_end, src);
   r.len0 = __shfl_sync(0xffffffffu, pl.len0, src);
   return r;
-}
-
-// Every thread of the CTA: tile counts of all sequences (into `tiles`, at least `batch` ints of
-// shared memory), the plan kind, this pair's range and the sequence it starts in.  The even CTA
-// of range 0 also writes the plan table the combine reads.
-__device__ void tc_make_plan(const DecodeTcArgs& a, int pair, bool write_table, int* tiles, int* scratch,
-                             TcPlan* plan) {
-  const int tid = threadIdx.x;
-  const int nthr = blockDim.x;
-  const int B = a.batch;
-  const int per = (B + nthr - 1) / nthr;
-  const int lo = min(B, tid * per), hi = min(B, lo + per);
-  int sum = 0, mn = INT_MAX;
-  for (int bb = lo; bb < hi; ++bb) {
-    const int t = tiles_of(seq_len_checked(a.seq_lens, bb, a.capacity));
-    tiles[bb] = t;
-    sum += t;
-    if (t > 0) mn = min(mn, t);
-  }
-  int excl, T;
-  block_scan(sum, scratch, excl, T);
-  // smallest non-empty sequence (in tiles)
-#pragma unroll
-  for (int d = 16; d > 0; d >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, d));
-  if ((tid & 31) == 0) scratch[tid >> 5] = mn;
-  if (tid == 0) {
-    plan->start = plan->end = 0;   // an idle pair unless a thread below finds its range
-    plan->b0 = plan->off0 = 0;
-    plan->b_end = 0;
-    plan->len0 = 0;
-  }
-  __syncthreads();
-  for (int i = 0; i < (nthr >> 5); ++i) mn = min(mn, scratch[i]);
-  __syncthreads();
-  const bool per_seq = T > 0 && static_cast<int64_t>(mn) * a.P >= T;
-  if (per_seq) {
-    // r_b = floor(P tiles_b / T) ranges for sequence b (>= 1 by the condition, <= tiles_b)
-    auto ranges_of = [&](int t) -> int {
-      if (t == 0) return 0;
-      const int r = static_cast<int>((static_cast<int64_t>(a.P) * t) / T);
-      return r < t ? r : t;
-    };
-    int rsum = 0;
-    for (int bb = lo; bb < hi; ++bb) rsum += ranges_of(tiles[bb]);
-    int rexcl, R;
-    block_scan(rsum, scratch, rexcl, R);
-    int r0 = rexcl;
-    for (int bb = lo; bb < hi; ++bb) {
-      const int t = tiles[bb], r = ranges_of(t);
-      if (write_table) a.ws.off[bb] = r0;
-      if (r0 <= pair && pair < r0 + r) {
-        const int j = pair - r0;
-        plan->b0 = bb;
-        plan->len0 = seq_len_checked(a.seq_lens, bb, a.capacity);
-        plan->off0 = 0;
-        plan->start = static_cast<int>((static_cast<int64_t>(j) * t) / r);
-        plan->end = static_cast<int>((static_cast<int64_t>(j + 1) * t) / r);
-        plan->b_end = bb + 1;
-      }
-      r0 += r;
-    }
-    if (write_table && tid == 0) {
-      a.ws.off[B] = R;
-      a.ws.off[B + 1] = kPlanPerSequence;
-    }
-  } else {
-    const int start = T > 0 ? range_start(pair, a.P, T) : 0;
-    const int end = T > 0 ? range_start(pair + 1, a.P, T) : 0;
-    int off = excl;   // global tile offset of sequence lo
-    for (int bb = lo; bb < hi; ++bb) {
-      if (write_table) a.ws.off[bb] = off;
-      if (start < end && off <= start && start < off + tiles[bb]) {
-        plan->b0 = bb;
-        plan->len0 = seq_len_checked(a.seq_lens, bb, a.capacity);
-        plan->off0 = off;
-        plan->start = start;
-        plan->end = end;
-        plan->b_end = B;
-      }
-      off += tiles[bb];
-    }
-    if (write_table && tid == 0) {
-      a.ws.off[B] = T;
-      a.ws.off[B + 1] = kPlanBalanced;
-    }
-  }
-  __syncthreads();
 }
 
 // ------------------------------------------------------------------------------ kernel
@@ -922,22 +843,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   cluster_arrive_release();
   // seq_lens (read by the plan) may come from the previous kernel.
   pdl_wait();
-  if (a.batch <= kWarpPlanMax) {
-    // The producer warp computes the plan and hands it to the other warps through named barrier 2
-    // (it only arrives, so its first copies need not wait for them).
-    if (warp == kTcProducerWarp) {
-      const TcPlan w = tc_make_plan_warp(a, pair, pair == 0 && rank == 0);
-      if ((threadIdx.x & 31) == 0) *plan = w;
-      __syncwarp();
-      named_bar_arrive(2, kTcThreads);
-    } else {
-      named_bar_sync(2, kTcThreads);
-    }
+  // The producer warp computes the plan and hands it to the other warps through named barrier 2
+  // (it only arrives, so its first copies need not wait for them).
+  if (warp == kTcProducerWarp) {
+    const TcPlan w = tc_make_plan(a.seq_lens, a.capacity, a.batch, a.P, a.ws.off, pair, pair == 0 && rank == 0);
+    if ((threadIdx.x & 31) == 0) *plan = w;
+    __syncwarp();
+    named_bar_arrive(2, kTcThreads);
   } else {
-    // The block-wide plan uses the V ring (idle until the first V copy) for the tile counts and
-    // the exchange buffer for its scans; it ends with a CTA barrier.
-    tc_make_plan(a, pair, pair == 0 && rank == 0, reinterpret_cast<int*>(smem + kTcOffV), reinterpret_cast<int*>(red),
-                 plan);
+    named_bar_sync(2, kTcThreads);
   }
   cluster_wait_acquire();
   tc_fence_after();
@@ -955,10 +869,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
       *abort_flag = 1;
   } else if (rank == 0 && (threadIdx.x & 31) == 0) {
     bool ok = true;
-    if (warp == kTcMmaWarp) ok = tc_mma_qk(smem, bars, tmem, 0, a, pl, pair, abort_flag);
-    else if (warp == kTcMmaBWarp) ok = tc_mma_qk(smem, bars, tmem, 1, a, pl, pair, abort_flag);
-    else if (warp == kTcPvWarp) ok = tc_mma_pv(smem, bars, tmem, 0, a, pl, pair, abort_flag);
-    else ok = tc_mma_pv(smem, bars, tmem, 1, a, pl, pair, abort_flag);
+    // One out-of-line copy of each issuer serves both of its warps (part / latent half as argument).
+    const SegmentCursor cur{pl.b0, pl.off0, pl.start, pl.end, pl.b_end, pair, true, pl.len0};
+    if (warp == kTcMmaWarp || warp == kTcMmaBWarp)
+      ok = tc_mma_qk(smem, bars, tmem, warp == kTcMmaWarp ? 0 : 1, a.seq_lens, a.capacity, cur, abort_flag);
+    else
+      ok = tc_mma_pv(smem, bars, tmem, warp == kTcPvWarp ? 0 : 1, a.seq_lens, a.capacity, cur, abort_flag);
     if (!ok) *abort_flag = 1;
   }
   __syncwarp();
