@@ -1,9 +1,10 @@
-// decode_tc.cuh — split-KV MLA decode on the tcgen05 tensor cores, one CTA pair per
-// (sequence, split).
+// decode_tc.cuh — split-KV MLA decode on the tcgen05 tensor cores, one CTA pair per work range
+// of 128-token tiles (the plan in decode_common.cuh: a range is one piece of one sequence, or a
+// run of tiles that crosses sequences; each sequence piece it meets is a segment).
 //
 // What it computes (《DeepSeek-V2》深度解读报告 §2.3 Absorption, §2.4 Decoupled RoPE): for every
 // head h the score of cached token t is  s = scale * q_full[h] . row_t  over the 576-wide row
-// [c (512) | RoPE(k^R) (64)] (content plus position channel), an online softmax over the split's
+// [c (512) | RoPE(k^R) (64)] (content plus position channel), an online softmax over the segment's
 // tokens, and  O[h] = sum_t e^{s - m} c_t  over the 512-wide latent.  Every latent row is read from
 // HBM once and shared by all 128 heads, which is what makes QK^T and PV dense contractions.
 //
@@ -22,14 +23,19 @@
 // fixed cost per copy (measured: ~0.35 us for anything from 8 KB to 72 KB from L2), so every copy
 // is large: a CTA's K rows of a tile (from HBM) come as one 3-D box of all 9 dim-slabs (72 KB),
 // and V rows (the L2 re-read) as 4-D boxes of 64 tokens x both 64-wide latent chunks x both
-// latent halves (32 KB, 2 copies per tile) into a 2-slot V ring.  K tiles a few steps ahead are
-// pulled into L2 with bulk prefetches.  Separate K and V buffers let the K copy of the next tile
-// proceed while V of the current tile waits for its softmax.
-// V rows past the split end are zeroed in shared memory before PV (rows past a sequence's end may
-// hold anything, and 0 * NaN would poison the sum).
+// latent halves (32 KB, 2 copies per tile) into a 2-slot V ring.  Separate K and V buffers let
+// the K copy of the next tile proceed while V of the current tile waits for its softmax.
+// V rows past the segment end are zeroed in shared memory before PV (rows past a sequence's end
+// may hold anything, and 0 * NaN would poison the sum).
+//
+// Segments.  Every role walks the same segments of its range with a SegmentCursor.  A new
+// segment loads its sequence's Q (once both QK^T parts are done with the previous Q), restarts
+// the softmax state, overwrites O with its first PV (after the previous segment's epilogue has
+// read O and released the V ring it stages through), and ends with an epilogue that writes either
+// the final output (a segment covering its whole sequence) or an fp32 partial for the combine.
 //
 // Warp roles (416 threads): warps 0-7 softmax / O correction / epilogue (two warps per TMEM lane
-// quadrant, each owning half of the S columns), warp 8 TMA producer and L2 prefetcher, and in the
+// quadrant, each owning half of the S columns), warp 8 work plan and TMA producer, and in the
 // even CTA only: warp 9 QK^T part A (warp 9 also allocates TMEM in both CTAs), warp 11 QK^T part
 // B, warps 10 and 12 PV for the two latent halves.
 #pragma once
@@ -51,7 +57,6 @@ constexpr int kTcKSlabsB = 4;
 __host__ __device__ constexpr int tc_part_slab0(int part) { return part ? kTcKSlabsA : 0; }
 __host__ __device__ constexpr int tc_part_slabs(int part) { return part ? kTcKSlabsB : kTcKSlabsA; }
 constexpr int kTcVSlots = 2;
-constexpr int kTcPrefetchTiles = 4;          // K tiles pulled into L2 ahead of their load
 constexpr int kTcVBox = 4 * kTcSlab;         // 64 tokens x 2 chunks x 2 latent halves
 constexpr int kTcQBytes = 9 * kTcSlab;
 constexpr int kTcPBytes = 2 * kTcSlab;       // 64 heads x 128 tokens bf16, two 64-token K chunks
@@ -80,7 +85,6 @@ constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 5);
 
 struct DecodeTcArgs {
   CacheView v;
-  const uint8_t* cache;   // cache rows (for L2 prefetches)
   const int32_t* seq_lens;
   int batch;
   int capacity;        // tokens a sequence can hold (lengths are clamped to it)
@@ -158,8 +162,9 @@ __device__ __forceinline__ void tma_load_4d_local(void* dst, const CUtensorMap* 
 
 // ------------------------------------------------------------------------------ TMA producer
 // One warp.  Lane 0 issues the copies, in the order K(0), K(1), V(0), K(2), V(1), ..., V(n-1):
-// K one tile ahead, so QK^T of tile i+1 never waits behind V of tile i.  All lanes pull the K
-// rows of the tile kTcPrefetchTiles ahead into L2 with plain prefetches, so each K copy reads L2.
+// K one tile ahead, so QK^T of tile i+1 never waits behind V of tile i.  (Pulling later K tiles
+// into L2 ahead of their copies with plain prefetches measured no faster and adds code to the
+// per-tile loop, so the K copies read HBM directly.)
 //  K(i): CTA r's 64 tokens [tile0 + 64r, +64) x 576 dims as two boxes, one per QK^T part
 //        (5 and 4 dim-slabs).  A half-tile past the split end is loaded from a negative row
 //        (zeros); its scores are masked anyway.
@@ -171,8 +176,33 @@ __device__ __forceinline__ void zero_v_rows(uint8_t* box, int v, int lane) {
   for (int row = v; row < 64; ++row) p[row * 8] = make_uint4(0, 0, 0, 0);
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* ptr) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+// A V box that reaches past the segment end: loaded through a CTA-local barrier (if any row is
+// valid), the rows past the end zeroed by all lanes after the copy has landed, then published:
+// each lane's proxy fence, the warp barrier, and lane 0's arrival with release semantics on the
+// even CTA's v_full.  Out of line: it runs at most twice per segment.  False if a wait failed.
+__device__ __noinline__ bool tc_load_ragged_v(uint8_t* box, const CUtensorMap* tm_v, uint64_t* fix, uint32_t fix_phase,
+                                              int row, int rank, int vcount, uint32_t vfull, volatile int* abort_flag) {
+  const int lane = threadIdx.x & 31;
+  if (vcount > 0) {
+    int ok = 1;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(fix, kTcVBox);
+      tma_load_4d_local(box, tm_v, fix, 0, row, 2 * rank, 0);
+      ok = (mbar_wait(fix, fix_phase, 0x13) && !*abort_flag) ? 1 : 0;
+    }
+    if (__shfl_sync(0xffffffffu, ok, 0) == 0) return false;
+  }
+  __syncwarp();
+  zero_v_rows(box, vcount, lane);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    if (rank == 0)
+      mbar_arrive_expect_tx_addr(vfull, 0u);
+    else
+      mbar_arrive_addr(vfull);
+  }
+  return true;
 }
 
 __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, const CUtensorMap* tm_v,
@@ -210,19 +240,7 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
       else
         mbar_arrive_relaxed(lbar(&bars->q_full));
     }
-    auto prefetch_k = [&](int j) {
-      const int my0 = t_begin + j * kTcTile + 64 * static_cast<int>(rank);
-      if (j >= n_tiles || my0 >= t_end) return;
-      const int64_t row = cache_row(a.v, b, my0);
-      if (row < 0) return;
-      const int64_t nrows = a.v.num_rows - row < 64 ? a.v.num_rows - row : 64;
-      const uint8_t* base = a.cache + row * (kDRow * 2);
-      const int lines = static_cast<int>(nrows) * (kDRow * 2 / 128);
-#pragma unroll 1
-      for (int q = lane; q < lines; q += 32) prefetch_l2(base + q * 128);
-    };
     auto issue_k = [&](int i) -> bool {
-      if (i > 0) prefetch_k(i + kTcPrefetchTiles);   // before the wait: it does not depend on it
       const int gi = g + i;
       const int my0 = t_begin + i * kTcTile + 64 * static_cast<int>(rank);
       const int y = my0 < t_end ? tma_row(a.v, b, my0) : -kTcTile;
@@ -261,39 +279,18 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
               mbar_arrive_relaxed(lbar(&bars->v_full[s]));
           }
         } else {
-          // Ragged: load through a CTA-local barrier, zero the rows past the end (all lanes, after
-          // the copy has landed), then publish: each lane's proxy fence, the warp barrier, and lane
-          // 0's arrival with release semantics.
-          if (vcount > 0) {
-            if (l0) {
-              mbar_arrive_expect_tx(&bars->fix, kTcVBox);
-              tma_load_4d_local(box, tm_v, &bars->fix, 0, tma_row(a.v, b, tok0), 2 * static_cast<int>(rank), 0);
-            }
-            if (!wait0(&bars->fix, fix_phase, 0x13)) return false;
-            fix_phase ^= 1u;
-          }
-          __syncwarp();
-          zero_v_rows(box, vcount, lane);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (l0) {
-            if (leader)
-              mbar_arrive_expect_tx_addr(lbar(&bars->v_full[s]), 0u);
-            else
-              mbar_arrive_addr(lbar(&bars->v_full[s]));
-          }
+          if (!tc_load_ragged_v(box, tm_v, &bars->fix, fix_phase, vcount > 0 ? tma_row(a.v, b, tok0) : 0,
+                                static_cast<int>(rank), vcount, lbar(&bars->v_full[s]), abort_flag))
+            return false;
+          if (vcount > 0) fix_phase ^= 1u;
         }
       }
       return true;
     };
-    // K(i) then V(i - 1): one call site each (the loop runs one step past the last K).  The first
-    // prefetches go out after K(0), which goes first.
+    // K(i) then V(i - 1): one call site each (the loop runs one step past the last K).
     for (int i = 0; ok && i <= n_tiles; ++i) {
       if (i < n_tiles) ok = issue_k(i);
-      if (i == 0)
-        for (int j = 1; j <= kTcPrefetchTiles; ++j) prefetch_k(j);
-      else if (ok)
-        ok = issue_v(i - 1);
+      if (i > 0 && ok) ok = issue_v(i - 1);
     }
     g += n_tiles;
     ++k;
@@ -492,6 +489,24 @@ __device__ __noinline__ void tc_write_segment(bool direct, void* row, float* m_o
   }
 }
 
+// O row slice *= alpha (128 fp32 columns of this thread's TMEM lane from addr).  Out of line: the
+// lazy rescale runs on few tiles, and the per-tile loop stays compact.
+__device__ __noinline__ void tc_rescale_o(uint32_t addr, float alpha) {
+  for (int qb = 0; qb < 4; ++qb, addr += 32) {   // 2 TMEM loads in flight per wait
+    uint32_t r[2][16];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) tmem_ld16(addr + 16 * k, r[k]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) r[k][e] = __float_as_uint(__uint_as_float(r[k][e]) * alpha);
+      tmem_st16(addr + 16 * k, r[k]);
+    }
+  }
+  tmem_st_wait();
+}
+
 __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, uint8_t* smem, TcBars* bars,
                            float* red, uint32_t tmem, uint32_t rank, volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5;
@@ -570,20 +585,7 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
         break;
       }
       tc_fence_after();
-      for (int qb = 0; qb < 4; ++qb) {   // 2 TMEM loads in flight per wait
-        const uint32_t addr = tmem + lane_base + kTcColO + 128 * ch + 32 * qb;
-        uint32_t r[2][16];
-#pragma unroll
-        for (int k = 0; k < 2; ++k) tmem_ld16(addr + 16 * k, r[k]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) r[k][e] = __float_as_uint(__uint_as_float(r[k][e]) * alpha);
-          tmem_st16(addr + 16 * k, r[k]);
-        }
-      }
-      tmem_st_wait();
+      tc_rescale_o(tmem + lane_base + kTcColO + 128 * ch, alpha);
     }
     // P for this tile, packed to bf16 in registers before the buffer is known to be free.
     const float neg_m = -m_used;
@@ -669,13 +671,14 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
 // of sequences [l per, (l + 1) per): three passes over it (tile totals and the smallest sequence;
 // per-chunk sums of the prefix counts; the prefix itself, the table and this pair's piece), with
 // one warp reduction or scan between passes.  Every lane returns the same plan.
-__device__ __forceinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacity, int B, int P, int32_t* table,
+__device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacity, int B, int P, int32_t* table,
                                                int pair, bool write_table) {
   const int lane = threadIdx.x & 31;
   const int per = (B + 31) / 32;
   const int lo = min(B, lane * per), hi = min(B, lo + per);
   // pass 1: total tiles T and the smallest non-empty sequence (and the largest)
   int sum = 0, mn = INT_MAX, mx = 0;
+  #pragma unroll 1
   for (int bb = lo; bb < hi; ++bb) {
     const int t = tiles_of(seq_len_checked(seq_lens, bb, capacity));
     sum += t;
@@ -692,6 +695,7 @@ __device__ __forceinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capa
     const int t = mn;
     const int r = min(P / B, t);
     if (write_table) {
+      #pragma unroll 1
       for (int bb = lo; bb < hi; ++bb) table[bb] = bb * r;
       if (lane == 0) {
         table[B] = B * r;
@@ -722,6 +726,7 @@ __device__ __forceinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capa
   int csum = sum;
   if (per_seq) {
     csum = 0;
+    #pragma unroll 1
     for (int bb = lo; bb < hi; ++bb) csum += count_of(tiles_of(seq_len_checked(seq_lens, bb, capacity)));
   }
   int incl = csum;
@@ -738,6 +743,7 @@ __device__ __forceinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capa
   pl.start = pl.end = 0;
   pl.b0 = pl.off0 = pl.b_end = pl.len0 = 0;
   int run = incl - csum;
+  #pragma unroll 1
   for (int bb = lo; bb < hi; ++bb) {
     const int L = seq_len_checked(seq_lens, bb, capacity);
     const int t = tiles_of(L);
