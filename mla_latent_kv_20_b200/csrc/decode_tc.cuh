@@ -54,9 +54,10 @@ constexpr int kTcSlab = 8192;                // 64 rows x 128 bytes
 // and S accumulator (the softmax adds the two): part A = dim-slabs [0, 5), part B = [5, 9).
 constexpr int kTcKSlabsA = 5;
 constexpr int kTcKSlabsB = 4;
+static_assert(kTcKSlabsB <= kTcKSlabsA, "the QK^T issue loop is unrolled to part A's slab count");
 __host__ __device__ constexpr int tc_part_slab0(int part) { return part ? kTcKSlabsA : 0; }
 __host__ __device__ constexpr int tc_part_slabs(int part) { return part ? kTcKSlabsB : kTcKSlabsA; }
-constexpr int kTcVSlots = 2;
+constexpr int kTcVSlots = 2;                 // one slot per 64-token half of a tile (the PV issuer relies on it)
 constexpr int kTcVBox = 4 * kTcSlab;         // 64 tokens x 2 chunks x 2 latent halves
 constexpr int kTcQBytes = 9 * kTcSlab;
 constexpr int kTcPBytes = 2 * kTcSlab;       // 64 heads x 128 tokens bf16, two 64-token K chunks
@@ -331,11 +332,15 @@ __device__ bool tc_mma_qk(uint8_t* smem, TcBars* bars, uint32_t tmem, int part, 
         return false;
       if (!mbar_wait_cluster(&bars->k_full[part], static_cast<uint32_t>(g) & 1u, 0x21)) return false;
       tc_fence_after();
-      for (int c = 0; c < nslabs; ++c)
+      // Fully unrolled (the issue rate of this thread bounds the tensor pipe here): every
+      // descriptor is a constant offset from the part's base.
+#pragma unroll
+      for (int c = 0; c < kTcKSlabsA; ++c)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16_pair(scol + 64 * j, sdesc_add(dq, c * kTcSlab + 32 * kk), sdesc_add(dk, c * kTcSlab + 32 * kk),
-                         idesc_qk, (c | kk) != 0 ? 1u : 0u);
+          if (c < nslabs)
+            umma_bf16_pair(scol + 64 * j, sdesc_add(dq, c * kTcSlab + 32 * kk), sdesc_add(dk, c * kTcSlab + 32 * kk),
+                           idesc_qk, (c | kk) != 0 ? 1u : 0u);
       umma_commit_pair_mc(&bars->k_empty[part], 3);
       umma_commit_pair_mc(&bars->s_full[j], 3);
       if (*abort_flag) return false;
@@ -354,9 +359,10 @@ __device__ bool tc_mma_pv(uint8_t* smem, TcBars* bars, uint32_t tmem, int nh, co
                           int capacity, SegmentCursor cur, volatile int* abort_flag) {
   const uint32_t idesc_pv = idesc_bf16_f32(128, 256, false, true);
   const uint64_t dp = sdesc_sw128(smem_u32(smem + kTcOffP), 16, 1024);
-  const uint64_t dv = sdesc_sw128(smem_u32(smem + kTcOffV), kTcSlab, 1024);
+  const uint64_t dv = sdesc_sw128(smem_u32(smem + kTcOffV + nh * 2 * kTcSlab), kTcSlab, 1024);
+  const uint32_t ocol = tmem + kTcColO + 128 * nh;
   Segment sg;
-  int g = 0, k = 0, vn = 0;
+  int g = 0, k = 0;
   bool ok = true;
   while (ok && cur.next(seq_lens, capacity, sg)) {
     if (k > 0 && !mbar_wait_cluster(&bars->o_free, static_cast<uint32_t>(k - 1) & 1u, 0x25)) {
@@ -368,20 +374,21 @@ __device__ bool tc_mma_pv(uint8_t* smem, TcBars* bars, uint32_t tmem, int nh, co
         ok = false;
         break;
       }
-      for (int h = 0; h < 2 && ok; ++h, ++vn) {
-        const int vs = vn % kTcVSlots;
-        if (!mbar_wait_cluster(&bars->v_full[vs], static_cast<uint32_t>(vn / kTcVSlots) & 1u, 0x23)) {
+      // V box 2g + h sits in slot h of the 2-slot ring, in its (g + 1)-th fill.
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int vs = h;
+        if (!mbar_wait_cluster(&bars->v_full[vs], static_cast<uint32_t>(g) & 1u, 0x23)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint64_t pb = sdesc_add(dp, h * kTcSlab);
+        const uint64_t vb = sdesc_add(dv, vs * kTcVBox);
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          const int gt = 4 * h + g4;   // 16-token group of the tile
-          umma_bf16_pair(tmem + kTcColO + 128 * nh, sdesc_add(dp, h * kTcSlab + 32 * g4),
-                         sdesc_add(dv, vs * kTcVBox + nh * 2 * kTcSlab + g4 * 2048), idesc_pv,
-                         (i > 0 || gt > 0) ? 1u : 0u);
-        }
+        for (int g4 = 0; g4 < 4; ++g4)   // 16-token groups; the segment's first MMA overwrites O
+          umma_bf16_pair(ocol, sdesc_add(pb, 32 * g4), sdesc_add(vb, g4 * 2048), idesc_pv,
+                         (i > 0 || h > 0 || g4 > 0) ? 1u : 0u);
         umma_commit_pair_mc(&bars->v_empty[vs], 3);
       }
       if (!ok) break;
