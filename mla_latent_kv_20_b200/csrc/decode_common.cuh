@@ -142,9 +142,10 @@ struct SegmentCursor {
 };
 
 // Combine: one warp per (b, h); lanes own 16 of the 512 latent columns.  grid = (batch, 128 / 4),
-// block = 128.  Empty sequences get out_lat = 0 and lse = -inf; sequences finished by the decode
-// kernel (one segment) are skipped; the others merge their partials in ascending range order.
-__global__ void __launch_bounds__(128) combine_kernel(Workspace ws, int P, __nv_bfloat16* __restrict__ out_lat,
+// block = 128, at most 64 registers a thread (8 blocks per SM: a 32-sequence batch is one wave).
+// Empty sequences get out_lat = 0 and lse = -inf; sequences finished by the decode kernel (one
+// segment) are skipped; the others merge their partials in ascending range order.
+__global__ void __launch_bounds__(128, 8) combine_kernel(Workspace ws, int P, __nv_bfloat16* __restrict__ out_lat,
                                                       float* __restrict__ lse) {
   pdl_trigger();
   pdl_wait();
@@ -168,27 +169,47 @@ __global__ void __launch_bounds__(128) combine_kernel(Workspace ws, int P, __nv_
   if (p0 == p1) return;
   auto slot_of = [&](int p) { return (!per_seq && range_start(p, P, T) < off) ? 2 * p + 1 : 2 * p; };
   auto nonempty = [&](int p) { return per_seq || range_start(p, P, T) < range_start(p + 1, P, T); };
-  float M = -INFINITY;
-  for (int p = p0; p <= p1; ++p)
-    if (nonempty(p)) M = fmaxf(M, ws.m[static_cast<int64_t>(slot_of(p)) * kHeads + h]);
+  // Online merge in ascending range order: after each range, (M, den, acc) hold the merge of the
+  // ranges so far relative to M.  Two ranges are fetched per step so their loads overlap (every
+  // partial's m is finite: a non-empty range holds at least one valid token of b).
+  float M = -INFINITY, den = 0.f;
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  float den = 0.f;
-  for (int p = p0; p <= p1; ++p) {
-    if (!nonempty(p)) continue;
+  auto fetch = [&](int p, float& m, float& l, float4 (&o)[4]) -> bool {
+    if (p > p1 || !nonempty(p)) return false;
     const int64_t ml = static_cast<int64_t>(slot_of(p)) * kHeads + h;
-    const float w = exp2f(ws.m[ml] - M);
-    den += w * ws.l[ml];
-    const float4* o = reinterpret_cast<const float4*>(ws.o + ml * kDLat);
+    m = ws.m[ml];
+    l = ws.l[ml];
+    const float4* src = reinterpret_cast<const float4*>(ws.o + ml * kDLat);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = src[lane + 32 * i];
+    return true;
+  };
+  auto merge = [&](float m, float l, const float4 (&o)[4]) {
+    const float Mn = fmaxf(M, m);
+    const float sa = M == -INFINITY ? 0.f : exp2f(M - Mn);
+    const float w = exp2f(m - Mn);
+    den = den * sa + w * l;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const float4 v = o[lane + 32 * i];
-      acc[4 * i + 0] += w * v.x;
-      acc[4 * i + 1] += w * v.y;
-      acc[4 * i + 2] += w * v.z;
-      acc[4 * i + 3] += w * v.w;
+      acc[4 * i + 0] = acc[4 * i + 0] * sa + w * o[i].x;
+      acc[4 * i + 1] = acc[4 * i + 1] * sa + w * o[i].y;
+      acc[4 * i + 2] = acc[4 * i + 2] * sa + w * o[i].z;
+      acc[4 * i + 3] = acc[4 * i + 3] * sa + w * o[i].w;
     }
+    M = Mn;
+  };
+  constexpr int kStep = 2;
+  for (int p = p0; p <= p1; p += kStep) {
+    float m[kStep], l[kStep];
+    float4 o[kStep][4];
+    bool has[kStep];
+#pragma unroll
+    for (int u = 0; u < kStep; ++u) has[u] = fetch(p + u, m[u], l[u], o[u]);
+#pragma unroll
+    for (int u = 0; u < kStep; ++u)
+      if (has[u]) merge(m[u], l[u], o[u]);
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
