@@ -64,48 +64,66 @@ def step_work(lens):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling while the timed region runs."""
+    """nvidia-smi clock/throttle sampling (every 50 ms) in a background reader that stamps each
+    sample with the host's monotonic clock, so samples can be kept for a time window."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.rows = []   # (monotonic time, sm MHz, max MHz, active reasons)
+        self.reader = None
 
     def start(self):
+        import threading
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+
+        def read():
+            for line in self.proc.stdout:
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm, mx = float(f[1]), float(f[2])
+                except ValueError:
+                    continue
+                act = {n for n, v in zip(self.NAMES, f[5:9]) if v.lower().startswith("active")}
+                self.rows.append((time.monotonic(), sm, mx, act))
+
+        self.reader = threading.Thread(target=read, daemon=True)
+        self.reader.start()
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.reader is not None:
+            self.reader.join(timeout=5)
+
+    def summary(self, t0, t1):
+        """Median SM clock, max clock and the union of active reasons of the samples in [t0, t1]."""
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = [r for r in self.rows if t0 <= r[0] <= t1]
+        reasons = set()
+        for r in rows:
+            reasons |= r[3]
+        return {"sm_mhz": statistics.median(r[1] for r in rows) if rows else None,
+                "sm_max_mhz": max(r[2] for r in rows) if rows else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
 
 
 # ------------------------------------------------------------------------------------- oracle
@@ -264,7 +282,7 @@ def setup_replica(name, device):
 # counters were taken, and the traffic is reported as null.
 TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh", "csrc/mla_lib.cu")
 MEASURED_TRAFFIC = {   # workload -> {"bytes": int, "sha256": str, "profile": str}
-    "b32_l4096": {"bytes": 175316992 + 3219712 + 16854528, "sha256": "40dfdc27ff37a6956f1763ac2bf2e5241927fdb419eea7d032c66f7f3be7cab9",
+    "b32_l4096": {"bytes": 155790848 + 3274240 + 16858368, "sha256": "7a9681871d95b005e56d815da9f61c91bf47bc802c05f4e9f83d047fe5b5dabc",
                   "profile": "profiles/decode_tc_b32_l4096.md (decode + combine, ncu cache flush per kernel)"},
 }
 
@@ -284,6 +302,8 @@ def recorded_traffic(workload):
         return None
     return rec["bytes"]
 
+
+CLOCK_WINDOW_S = 1.0     # clock-sampling replay window when the timed region is too short to sample
 
 LAUNCHES_PER_LAYER = 6   # append, absorb GEMM, q_pe rotation, decode split, combine, un-absorb GEMM
 
@@ -405,6 +425,7 @@ def run_ours(args, rank, world, local_rank):
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
+    m0 = time.monotonic()
     t_start.record()
     h0 = time.perf_counter()
     for i in range(args.steps):
@@ -412,9 +433,25 @@ def run_ours(args, rank, world, local_rank):
     host_ms = (time.perf_counter() - h0) * 1e3 / args.steps
     t_end.record()
     torch.cuda.synchronize()
+    m1 = time.monotonic()
     barrier()
-    clocks = sampler.stop()
     ms = t_start.elapsed_time(t_end) / args.steps
+    clocks = sampler.summary(m0, m1)
+    clocks["window"] = "timed region (%.1f ms)" % ((m1 - m0) * 1e3)
+    if clocks["samples"] < 5:
+        # The timed region is shorter than the sampler's resolution: the same step graphs replay
+        # for another ~CLOCK_WINDOW_S seconds right after it, untimed, and the clocks of that window
+        # stand for the load of the timed region.
+        n_win = max(1, int(CLOCK_WINDOW_S / max(ms * 1e-3, 1e-6)))
+        w0 = time.monotonic()
+        for i in range(n_win):
+            step_graphs[i % n_rot].replay()
+        torch.cuda.synchronize()
+        w1 = time.monotonic()
+        clocks = sampler.summary(w0, w1)
+        clocks["window"] = ("%d replays of the timed step right after the timed region (%.2f s; the timed "
+                            "region itself lasted %.1f ms)" % (n_win, w1 - w0, (m1 - m0) * 1e3))
+    sampler.stop()
     # per-phase timing loop
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(len(GRAPH_PHASES) + 1)] for _ in range(n_layers)]
            for _ in range(args.steps)]

@@ -122,16 +122,19 @@ int32_t mla_decode_num_splits(int32_t batch, int32_t max_seq_len, int32_t num_sp
 /*
  * Bytes of workspace mla_decode_attn needs, with P = mla_decode_num_splits(batch, max_seq_len,
  * num_splits): range partials O [2P, 128, 512] fp32 and (m, l) [2P, 128] fp32 each, then the
- * per-sequence tile offsets [batch + 1] int32 (rounded up to 16 bytes).
+ * plan table [batch + 2] int32 (per sequence its first global tile or first range, the total,
+ * the plan kind; rounded up to 16 bytes).
  */
 size_t mla_decode_workspace_size(int32_t batch, int32_t max_seq_len, int32_t num_splits);
 
 /*
  * (3) Decode attention over the latent cache — [DR] §2.3/§2.4: score = scale * (q_abs.c + q_pe.k^R),
  *     the sum of the content and position channels; out_lat = softmax-weighted sum of c.
- * Split-KV flash decoding over balanced work ranges: every sequence is cut into 128-token tiles,
- * the tiles of the batch are laid end to end, and P ranges take equal shares
- * ([floor(pT/P), floor((p+1)T/P)) of the T tiles), so a range may span several sequences and a
+ * Split-KV flash decoding over P work ranges of 128-token tiles (T tiles in the batch, the last
+ * tile of a sequence ragged), planned on the device from seq_lens: when every non-empty sequence
+ * has at least T/P tiles, sequence b gets floor(P tiles_b / T) ranges that split its tiles evenly
+ * (per-sequence plan); otherwise the tiles of the batch are laid end to end and range p takes
+ * [floor(pT/P), floor((p+1)T/P)) (balanced plan), so a range may span several sequences and a
  * sequence several ranges.  Each part of a sequence a range covers keeps a running max m and sum
  * l (online softmax); a sequence covered by one range is finished by the decode kernel, the
  * others' unnormalised partials are merged by a combine in ascending range order:
