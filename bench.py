@@ -305,7 +305,7 @@ def recorded_traffic(workload):
 
 CLOCK_WINDOW_S = 1.0     # clock-sampling replay window when the timed region is too short to sample
 
-LAUNCHES_PER_LAYER = 6   # append, absorb GEMM, q_pe rotation, decode split, combine, un-absorb GEMM
+LAUNCHES_PER_LAYER = 5   # append, absorb GEMM (with the q_pe rotation), decode ranges, combine, un-absorb GEMM
 
 
 GRAPH_PHASES = ("append_absorb", "decode_attn", "unabsorb_v")

@@ -95,32 +95,4 @@ __global__ void __launch_bounds__(96) cache_append_kernel(const uint4* __restric
   }
 }
 
-// q_full[b, h, 512:576] = q_pe[b, h, :] rotated at q_pos[b] (or copied when q_pos is NULL).
-// grid = batch, block = 128 heads x 8 threads: the 32 angles of the sequence's position are formed
-// once (threads 0..31) and shared through shared memory; each thread then rotates 4 pairs of one
-// head.
-__global__ void __launch_bounds__(1024) qpe_kernel(const uint4* __restrict__ q_pe, const int32_t* __restrict__ q_pos,
-                                                   uint4* __restrict__ q_full, RopeFreq f) {
-  __shared__ double cs_sn[kDRope / 2][2];
-  pdl_trigger();
-  pdl_wait();
-  const int b = blockIdx.x;
-  const int h = threadIdx.x >> 3;
-  const int ch = threadIdx.x & 7;
-  if (q_pos != nullptr && threadIdx.x < kDRope / 2) {
-    double sn, cs;
-    sincos(static_cast<double>(q_pos[b]) * f.inv_freq[threadIdx.x], &sn, &cs);
-    cs_sn[threadIdx.x][0] = cs;
-    cs_sn[threadIdx.x][1] = sn;
-  }
-  __syncthreads();
-  uint4 r = q_pe[(static_cast<int64_t>(b) * kHeads + h) * (kDRope / 8) + ch];
-  if (q_pos != nullptr) {
-    __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(&r);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) x[k] = rope_pair(x[k], cs_sn[4 * ch + k][0], cs_sn[4 * ch + k][1]);
-  }
-  q_full[(static_cast<int64_t>(b) * kHeads + h) * (kDRow / 8) + kDLat / 8 + ch] = r;
-}
-
 }  // namespace mla

@@ -19,6 +19,7 @@
 
 #include <cuda_bf16.h>
 
+#include "append.cuh"
 #include "ptx.cuh"
 
 namespace mla {
@@ -36,11 +37,15 @@ __host__ __device__ constexpr int gemm_stage_bytes(int nt) { return kGemmKS * 25
 // tmB: 3-D view of the activation (64-element K slab, batch row, slab index = (h * KTOT + k) / 64);
 //      box {64, nt, KS / 64}: smem [slab][nt rows][128 B].
 // out element (n, h, m) is stored at out[n * out_bstride + h * out_hstride + m].
+// Query side only (qpe != nullptr, KTOT = d_h): the CTAs of M tile 0 also fill the RoPE part of the
+// query rows of their head and batch tile, out[n, h, 512:576] = q_pe[n, h, :] rotated at
+// q_pos[n] (or copied when q_pos is null), with their epilogue warps while the MMAs run.
 template <int KTOT, int NSTAGE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      __nv_bfloat16* __restrict__ out, int batch, int nt, int64_t out_bstride,
-                     int out_hstride) {
+                     int out_hstride, const uint4* __restrict__ qpe, const int32_t* __restrict__ q_pos,
+                     const RopeFreq rope) {
   constexpr int KSTAGES = KTOT / kGemmKS;
   static_assert(KTOT % kGemmKS == 0, "contraction length");
   extern __shared__ uint8_t smem_raw[];
@@ -145,6 +150,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // Warp w owns outputs m0 + 32w + [0, 32) for every n of the tile.  Lane = m in TMEM, so the
     // warp's [n][32 m] block goes through a stage in the (now idle) operand ring: each lane writes
     // its column, then every global store instruction covers eight whole 64-byte rows.
+    if (qpe != nullptr && blockIdx.x == 0) {
+      // 8 uint4 (64 bf16) per query row; rows n0 .. n0 + nt - 1 of head h.  Angle and rotation in
+      // fp64, one rounding per output (the same arithmetic as the cache append's RoPE).
+      const int rows = min(nt, batch - n0);
+      for (int idx = threadIdx.x; idx < rows * 8; idx += 128) {
+        const int n = n0 + (idx >> 3);
+        const int ch = idx & 7;
+        const int64_t row = static_cast<int64_t>(n) * kHeads + h;
+        uint4 r = qpe[row * (kDRope / 8) + ch];
+        if (q_pos != nullptr) {
+          const double pos = static_cast<double>(q_pos[n]);
+          __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            double sn, cs;
+            sincos(pos * rope.inv_freq[4 * ch + k], &sn, &cs);
+            x[k] = rope_pair(x[k], cs, sn);
+          }
+        }
+        reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * out_bstride + static_cast<int64_t>(h) * out_hstride)[kDLat / 8 + ch] = r;
+      }
+    }
     const bool ok = mbar_wait(done, 0);
     tc_fence_after();
     if (ok && !*reinterpret_cast<volatile int*>(abort_flag)) {

@@ -241,7 +241,8 @@ namespace {
 
 template <int KTOT, int NSTAGE>
 mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, int batch, __nv_bfloat16* out,
-                            int64_t out_bstride, int out_hstride, cudaStream_t stream) {
+                            int64_t out_bstride, int out_hstride, cudaStream_t stream, const void* qpe = nullptr,
+                            const int32_t* q_pos = nullptr, float rope_base = 10000.f) {
   // Weight viewed as [heads * KTOT rows][m_total cols]: 3-D (64-element M chunk, row, M chunk index),
   // box {64, KS, 2}.  Activation as [batch rows][heads * KTOT cols]: 3-D (64-element K slab, batch
   // row, slab index), box {64, nt, KS / 64}.
@@ -267,7 +268,7 @@ mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, in
     return MLA_ERR_CUDA;
   dim3 grid(m_total / 128, mla::kHeads, (batch + nt - 1) / nt);
   return launch_chained(kern, grid, dim3(mla::kGemmThreads), smem, stream, ta, tb, out, batch, nt, out_bstride,
-                        out_hstride);
+                        out_hstride, reinterpret_cast<const uint4*>(qpe), q_pos, rope_freq(rope_base));
 }
 
 }  // namespace
@@ -283,13 +284,11 @@ mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int3
   if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(w_uk) || !aligned16(q_full)) return MLA_ERR_INVALID_ARG;
   if (q_pos != nullptr && (!(rope_base > 0.f) || !std::isfinite(rope_base))) return MLA_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
-  mla_status st = launch_proj_gemm<mla::kDHead, 1>(w_uk, mla::kDLat, q_nope, batch,
-                                                   reinterpret_cast<__nv_bfloat16*>(q_full),
-                                                   static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow, s);
-  if (st != MLA_OK) return st;
-  return launch_chained(mla::qpe_kernel, dim3(batch), dim3(mla::kHeads * 8), 0, s,
-                        reinterpret_cast<const uint4*>(q_pe), q_pos, reinterpret_cast<uint4*>(q_full),
-                        rope_freq(rope_base));
+  // One launch: the W_UK GEMM fills q_full[:, :, 0:512] and its M-tile-0 CTAs rotate q_pe into
+  // q_full[:, :, 512:576].
+  return launch_proj_gemm<mla::kDHead, 1>(w_uk, mla::kDLat, q_nope, batch, reinterpret_cast<__nv_bfloat16*>(q_full),
+                                          static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow, s, q_pe, q_pos,
+                                          rope_base);
 }
 
 mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf16* out, int32_t batch,
