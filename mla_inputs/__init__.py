@@ -24,6 +24,8 @@ D_HEAD = 128      # d_h: per-head width of q_nope and of the output
 D_LATENT = 512    # d_c: width of the cached latent c^KV
 D_ROPE = 64       # d_R: width of the shared decoupled-RoPE key k^R
 D_ROW = D_LATENT + D_ROPE
+D_HIDDEN = 5120   # d: model width ([DR] §3.3), input of the down-projections
+DOWN_W_STD = 0.006   # initialisation std of the weights ([DR] §3.3)
 PAGE = 64
 W_STD = 1.0 / math.sqrt(512.0)
 
@@ -75,6 +77,25 @@ def layer_weights(seed: int, n_heads: int = N_HEADS, d_head: int = D_HEAD,
     w_uk = _normal_bf16(rng, (n_heads, d_head, d_latent), W_STD)
     w_uv = _normal_bf16(rng, (n_heads, d_latent, d_head), W_STD)
     return LayerWeights(w_uk, w_uv)
+
+
+@dataclasses.dataclass
+class DownProjection:
+    """Inputs of the fused down-projection + append: new tokens' hidden states and the weights
+    that map them to the cached latent and RoPE key (recipe: hidden 5120 and the initialisation
+    std 0.006 of [DR] §3.3; hidden states N(0, 1))."""
+    h: np.ndarray        # [n, d] bf16 bits
+    w_dkv: np.ndarray    # [d_c, d] bf16 bits: c^KV = W_D^KV h
+    w_kr: np.ndarray     # [d_R, d] bf16 bits: k^R (before RoPE) = W^KR h
+
+
+def down_projection(seed: int, n_tokens: int, d_hidden: int = D_HIDDEN, d_latent: int = D_LATENT,
+                    d_rope: int = D_ROPE) -> DownProjection:
+    rng = np.random.Generator(np.random.PCG64(seed))
+    w_dkv = _normal_bf16(rng, (d_latent, d_hidden), DOWN_W_STD)
+    w_kr = _normal_bf16(rng, (d_rope, d_hidden), DOWN_W_STD)
+    h = _normal_bf16(rng, (n_tokens, d_hidden), 1.0)
+    return DownProjection(h, w_dkv, w_kr)
 
 
 def decode_batch(seed: int, seq_lens, n_heads: int = N_HEADS, d_head: int = D_HEAD,

@@ -21,7 +21,10 @@ Readings where the pages are silent (each one is listed in the design doc):
     formula; this is the original RoPE definition);
   * W_UK is laid out [head, d_h, d_c] (k^C_j = sum_k W_UK[h,j,k] c_k) and W_UV is laid out
     [head, d_c, d_h] (v^C_j = sum_k W_UV[h,k,j] c_k);
-  * the new token is appended before attention, so the query attends to itself.
+  * the new token is appended before attention, so the query attends to itself;
+  * the down-projections are laid out [out, in] (W_D^KV [d_c, d], W^KR [d_R, d]) and k^R is the
+    plain linear projection W^KR h_t (the pages draw the branch h_t -> k^R without naming its
+    matrix), rotated by RoPE before it is cached.
 
 Pins: every function here is checked by ``tests/test_oracle_pins.py`` against values that
 do not come from this file (closed forms, library routines, brute-force scalar loops,
@@ -76,6 +79,19 @@ def apply_rope(x: np.ndarray, pos, base: float = ROPE_BASE) -> np.ndarray:
 def cache_rows(c: np.ndarray, kr_raw: np.ndarray, pos, base: float = ROPE_BASE) -> np.ndarray:
     """The cached row of a token: [c^KV | RoPE(k^R, pos)], width d_c + d_R ([DR] §2.4)."""
     return np.concatenate([np.asarray(c, dtype=np.float64), apply_rope(kr_raw, pos, base)], axis=-1)
+
+
+def project_rows(h: np.ndarray, w_dkv: np.ndarray, w_kr: np.ndarray, pos, base: float = ROPE_BASE) -> np.ndarray:
+    """Cached rows straight from the hidden states ([DR] §2.2: c^KV = W_D^KV h; §3.1: k^R is the
+    shared 64-wide projection of h on the RoPE branch; §2.4: RoPE applies to that branch only).
+
+    h: [n, d]; w_dkv: [d_c, d] and w_kr: [d_R, d] (output index first, as a linear layer maps
+    d inputs to d_c or d_R outputs); pos: [n].  Returns [n, d_c + d_R]: [W_D^KV h | RoPE(W^KR h)].
+    """
+    h = np.asarray(h, dtype=np.float64)
+    c = h @ np.asarray(w_dkv, dtype=np.float64).T       # [n, d_c]
+    kr_raw = h @ np.asarray(w_kr, dtype=np.float64).T   # [n, d_R]
+    return cache_rows(c, kr_raw, pos, base)
 
 
 # ----------------------------------------------------------------------------------------

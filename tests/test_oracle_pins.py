@@ -324,3 +324,69 @@ def test_pins_catch_planted_absorb_mistakes():
         return np.einsum("hj,hjk->hk", qn, w_uk[::-1])          # heads swapped
 
     assert _fails(check_absorb_unabsorb, uk_wrong_index, oracle.unabsorb_v)
+
+
+# ------------------------------------------------------------------ down-projection + append
+def bf_project_rows(h, w_dkv, w_kr, pos, base=oracle.ROPE_BASE):
+    """[W_D^KV h | RoPE(W^KR h)] by scalar loops: the rotation of each pair written out with
+    math.cos / math.sin of pos * base^(-2i/d_R)."""
+    n, d = h.shape
+    dc, dr = w_dkv.shape[0], w_kr.shape[0]
+    rows = []
+    for t in range(n):
+        c = [sum(float(w_dkv[j, k]) * float(h[t, k]) for k in range(d)) for j in range(dc)]
+        kr = [sum(float(w_kr[j, k]) * float(h[t, k]) for k in range(d)) for j in range(dr)]
+        rot = []
+        for i in range(dr // 2):
+            a = float(pos[t]) * float(base) ** (-2.0 * i / dr)
+            x, y = kr[2 * i], kr[2 * i + 1]
+            rot += [x * math.cos(a) - y * math.sin(a), x * math.sin(a) + y * math.cos(a)]
+        rows.append(c + rot)
+    return np.array(rows)
+
+
+def check_project_rows(project_rows):
+    rng = np.random.default_rng(11)
+    h = rng.standard_normal((3, 7))
+    w_dkv = rng.standard_normal((5, 7))
+    w_kr = rng.standard_normal((4, 7))
+    pos = np.array([0, 3, 1000])
+    got = project_rows(h, w_dkv, w_kr, pos)
+    assert got.shape == (3, 9)
+    assert np.allclose(got, bf_project_rows(h, w_dkv, w_kr, pos), rtol=1e-12, atol=1e-12)
+    # Selection weights reduce it to the plain append of (c, k^R) = parts of h.
+    c = rng.standard_normal((2, 4))
+    kr = rng.standard_normal((2, 2))
+    hsel = np.concatenate([c, kr, rng.standard_normal((2, 3))], axis=1)       # d = 9
+    sel_c = np.eye(4, 9)
+    sel_k = np.eye(2, 9, k=4)
+    p2 = np.array([5, 77])
+    assert np.allclose(project_rows(hsel, sel_c, sel_k, p2), oracle.cache_rows(c, kr, p2), rtol=0, atol=1e-14)
+    # Linear in h at fixed positions.
+    h2 = rng.standard_normal((3, 7))
+    lhs = project_rows(2.0 * h - 0.5 * h2, w_dkv, w_kr, pos)
+    rhs = 2.0 * project_rows(h, w_dkv, w_kr, pos) - 0.5 * project_rows(h2, w_dkv, w_kr, pos)
+    assert np.allclose(lhs, rhs, rtol=1e-12, atol=1e-12)
+
+
+def test_project_rows_pins():
+    check_project_rows(oracle.project_rows)
+
+
+def test_pins_catch_planted_projection_mistakes():
+    def parts_swapped(h, w_dkv, w_kr, pos, base=oracle.ROPE_BASE):
+        r = oracle.project_rows(h, w_dkv, w_kr, pos, base)
+        dc = w_dkv.shape[0]
+        return np.concatenate([r[:, dc:], r[:, :dc]], axis=1)
+
+    def rope_on_latent(h, w_dkv, w_kr, pos, base=oracle.ROPE_BASE):
+        r = oracle.project_rows(h, w_dkv, w_kr, pos, base)
+        dc = w_dkv.shape[0] - w_dkv.shape[0] % 2
+        r[:, :dc] = oracle.apply_rope(r[:, :dc], pos, base)
+        return r
+
+    def unrotated_key(h, w_dkv, w_kr, pos, base=oracle.ROPE_BASE):
+        return oracle.project_rows(h, w_dkv, w_kr, np.zeros_like(np.asarray(pos)), base)
+
+    for bad in (parts_swapped, rope_on_latent, unrotated_key):
+        assert _fails(check_project_rows, bad), bad.__name__
