@@ -100,6 +100,26 @@ mla_status mla_cache_append(const mla_bf16* c_new, const mla_bf16* kr_new, const
                             mla_cache_desc desc, int32_t n_tokens, float rope_base, void* stream);
 
 /*
+ * (1') Down-projection + cache append — [DR] §2.2 (c^KV = W_D^KV h_t), §3.1 (k^R, the shared
+ *      64-wide key of the RoPE branch, is projected from h_t too; c^KV and k^R are the only cached
+ *      objects), §2.4 (RoPE on that branch only), §3.3 (model width d = 5120).
+ * For each new token i in [0, n_tokens):
+ *     row = [ W_D^KV h[i] (512) | RoPE(W^KR h[i], pos[i]) (64) ]  written to the slot of
+ *     (seq = seq_ids ? seq_ids[i] : i, token position pos[i])
+ * i.e. the row mla_cache_append writes for c_new = W_D^KV h, kr_new = W^KR h, without the
+ * round trip through memory.  Products in fp32 (exact for bf16), sums over d in fp32; the latent is
+ * rounded once to bf16, the key rotated in fp64 from its fp32 sum and rounded once to bf16.
+ *   h      [n_tokens, 5120] bf16          w_dkv [512, 5120] bf16 (output index first)
+ *   w_kr   [64, 5120] bf16                seq_ids [n_tokens] int32 or NULL    pos [n_tokens] int32
+ *   cache  per desc (written)             block_table per desc or NULL
+ * n_tokens == 0 is a no-op; n_tokens must be <= 65536.  Device checks as mla_cache_append.
+ */
+mla_status mla_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const mla_bf16* w_kr,
+                              const int32_t* seq_ids, const int32_t* pos, mla_bf16* cache,
+                              const int32_t* block_table, mla_cache_desc desc, int32_t n_tokens,
+                              float rope_base, void* stream);
+
+/*
  * (2) Query absorption — [DR] §2.3 (q.(W_UK c) = (q W_UK).c by associativity).
  *     q_full[b, h, 0:512]   = sum_j q_nope[b, h, j] * W_UK[h, j, :]        (tcgen05, fp32 accumulate)
  *     q_full[b, h, 512:576] = q_pe[b, h, :], rotated at q_pos[b] if q_pos != NULL

@@ -51,6 +51,7 @@ def _load():
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "mla_version": (I32, []),
         "mla_cache_append": (ctypes.c_int, [P, P, P, P, P, P, CacheDesc, I32, F32, P]),
+        "mla_project_append": (ctypes.c_int, [P, P, P, P, P, P, P, CacheDesc, I32, F32, P]),
         "mla_absorb_q": (ctypes.c_int, [P, P, P, P, P, I32, F32, P]),
         "mla_decode_num_splits": (I32, [I32, I32, I32]),
         "mla_decode_workspace_size": (SZ, [I32, I32, I32]),
@@ -100,6 +101,13 @@ def cache_append(c_new, kr_new, pos, cache, desc: CacheDesc, *, seq_ids=None, bl
     n = c_new.shape[0] if n_tokens is None else n_tokens
     _check(lib.mla_cache_append(_ptr(c_new), _ptr(kr_new), _ptr(seq_ids), _ptr(pos), _ptr(cache),
                                 _ptr(block_table), desc, n, rope_base, _stream(stream)), "mla_cache_append")
+
+
+def project_append(h, w_dkv, w_kr, pos, cache, desc: CacheDesc, *, seq_ids=None, block_table=None,
+                   rope_base: float = 10000.0, stream=None, n_tokens: int | None = None):
+    n = h.shape[0] if n_tokens is None else n_tokens
+    _check(lib.mla_project_append(_ptr(h), _ptr(w_dkv), _ptr(w_kr), _ptr(seq_ids), _ptr(pos), _ptr(cache),
+                                  _ptr(block_table), desc, n, rope_base, _stream(stream)), "mla_project_append")
 
 
 def absorb_q(q_nope, q_pe, w_uk, q_full, *, q_pos=None, rope_base: float = 10000.0, stream=None,

@@ -37,9 +37,10 @@ __host__ __device__ constexpr int gemm_stage_bytes(int nt) { return kGemmKS * 25
 // tmB: 3-D view of the activation (64-element K slab, batch row, slab index = (h * KTOT + k) / 64);
 //      box {64, nt, KS / 64}: smem [slab][nt rows][128 B].
 // out element (n, h, m) is stored at out[n * out_bstride + h * out_hstride + m].
-// Query side only (qpe != nullptr, KTOT = d_h): the CTAs of M tile 0 also fill the RoPE part of the
-// query rows of their head and batch tile, out[n, h, 512:576] = q_pe[n, h, :] rotated at
-// q_pos[n] (or copied when q_pos is null), with their epilogue warps while the MMAs run.
+// Query side only (qpe != nullptr, KTOT = d_h): the epilogue warps also fill the RoPE part of the
+// query rows, out[n, h, 512:576] = q_pe[n, h, :] rotated at q_pos[n] (or copied when q_pos is
+// null), while the MMAs run: CTA c (linear index) takes rows n = c, c + #CTAs, ... for all 128
+// heads, so each row's 32 angles are formed once.
 template <int KTOT, int NSTAGE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -150,26 +151,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // Warp w owns outputs m0 + 32w + [0, 32) for every n of the tile.  Lane = m in TMEM, so the
     // warp's [n][32 m] block goes through a stage in the (now idle) operand ring: each lane writes
     // its column, then every global store instruction covers eight whole 64-byte rows.
-    if (qpe != nullptr && blockIdx.x == 0) {
-      // 8 uint4 (64 bf16) per query row; rows n0 .. n0 + nt - 1 of head h.  Angle and rotation in
-      // fp64, one rounding per output (the same arithmetic as the cache append's RoPE).
-      const int rows = min(nt, batch - n0);
-      for (int idx = threadIdx.x; idx < rows * 8; idx += 128) {
-        const int n = n0 + (idx >> 3);
-        const int ch = idx & 7;
-        const int64_t row = static_cast<int64_t>(n) * kHeads + h;
-        uint4 r = qpe[row * (kDRope / 8) + ch];
-        if (q_pos != nullptr) {
-          const double pos = static_cast<double>(q_pos[n]);
-          __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(&r);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            double sn, cs;
-            sincos(pos * rope.inv_freq[4 * ch + k], &sn, &cs);
-            x[k] = rope_pair(x[k], cs, sn);
-          }
+    if (qpe != nullptr) {
+      // Angle and rotation in fp64, one rounding per output (the same arithmetic as the cache
+      // append's RoPE).  cs_sn: this row's 32 (cos, sin) pairs, formed by threads 0..31.
+      double* cs_sn = reinterpret_cast<double*>(tmem_slot + 4);
+      const int ncta = gridDim.x * gridDim.y * gridDim.z;
+      const int c = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+      for (int n = c; n < batch; n += ncta) {
+        if (q_pos != nullptr && threadIdx.x < kDRope / 2) {
+          double sn, cs;
+          sincos(static_cast<double>(q_pos[n]) * rope.inv_freq[threadIdx.x], &sn, &cs);
+          cs_sn[2 * threadIdx.x] = cs;
+          cs_sn[2 * threadIdx.x + 1] = sn;
         }
-        reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * out_bstride + static_cast<int64_t>(h) * out_hstride)[kDLat / 8 + ch] = r;
+        named_bar_sync(1, 128);
+        for (int idx = threadIdx.x; idx < kHeads * (kDRope / 8); idx += 128) {   // (head, 16-byte chunk)
+          const int hh = idx >> 3;
+          const int ch = idx & 7;
+          const int64_t row = static_cast<int64_t>(n) * kHeads + hh;
+          uint4 r = qpe[row * (kDRope / 8) + ch];
+          if (q_pos != nullptr) {
+            __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) x[k] = rope_pair(x[k], cs_sn[2 * (4 * ch + k)], cs_sn[2 * (4 * ch + k) + 1]);
+          }
+          reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * out_bstride +
+                                   static_cast<int64_t>(hh) * out_hstride)[kDLat / 8 + ch] = r;
+        }
+        named_bar_sync(1, 128);   // the table is read before the next row overwrites it
       }
     }
     const bool ok = mbar_wait(done, 0);

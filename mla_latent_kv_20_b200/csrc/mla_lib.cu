@@ -16,6 +16,7 @@
 #include "append.cuh"
 #include "decode_common.cuh"
 #include "decode_tc.cuh"
+#include "down_proj.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 
@@ -235,6 +236,43 @@ mla_status mla_cache_append(const mla_bf16* c_new, const mla_bf16* kr_new, const
                         seq_ids, pos, reinterpret_cast<uint4*>(cache), v, rope_freq(rope_base));
 }
 
+
+mla_status mla_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const mla_bf16* w_kr,
+                              const int32_t* seq_ids, const int32_t* pos, mla_bf16* cache,
+                              const int32_t* block_table, mla_cache_desc desc, int32_t n_tokens, float rope_base,
+                              void* stream) {
+  if (n_tokens < 0 || !(rope_base > 0.f) || !std::isfinite(rope_base)) return MLA_ERR_INVALID_ARG;
+  CacheView v;
+  const mla_status st = check_cache(desc, cache, block_table, &v);
+  if (st != MLA_OK) return st;
+  if (n_tokens == 0) return MLA_OK;
+  if (h == nullptr || w_dkv == nullptr || w_kr == nullptr || pos == nullptr) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_dkv) || !aligned16(w_kr)) return MLA_ERR_INVALID_ARG;
+  if (seq_ids == nullptr && n_tokens > desc.num_seqs) return MLA_ERR_INVALID_ARG;
+  if (n_tokens > kMaxBatch) return MLA_ERR_UNSUPPORTED;
+  // 3-D views (64-column chunk, row, chunk index) of the row-major [rows][5120] matrices.
+  CUtensorMap tw, tk, th;
+  {
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDHidden) * 2, 128};
+    const cuuint64_t dw[3] = {64, static_cast<cuuint64_t>(mla::kDLat), mla::kDHidden / 64};
+    const cuuint64_t dk[3] = {64, static_cast<cuuint64_t>(mla::kDRope), mla::kDHidden / 64};
+    const cuuint64_t dh[3] = {64, static_cast<cuuint64_t>(n_tokens), mla::kDHidden / 64};
+    const cuuint32_t bw[3] = {64, 128, 2};
+    const cuuint32_t bk[3] = {64, static_cast<cuuint32_t>(mla::kDRope), 2};
+    const cuuint32_t bh[3] = {64, static_cast<cuuint32_t>(mla::kDpNt), 2};
+    if (!make_map_3d(&tw, w_dkv, dw, strides, bw) || !make_map_3d(&tk, w_kr, dk, strides, bk) ||
+        !make_map_3d(&th, h, dh, strides, bh))
+      return MLA_ERR_CUDA;
+  }
+  if (cudaFuncSetAttribute(mla::down_proj_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           mla::kDpSmemBytes) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  const dim3 grid(mla::kDpSplit, mla::kDpMTiles, (n_tokens + mla::kDpNt - 1) / mla::kDpNt);
+  return launch_chained(mla::down_proj_append_kernel, grid, dim3(mla::kDpThreads),
+                        static_cast<size_t>(mla::kDpSmemBytes), as_stream(stream), tw, tk, th, seq_ids, pos,
+                        reinterpret_cast<__nv_bfloat16*>(cache), v, n_tokens, rope_freq(rope_base));
+}
+
 }  // extern "C"
 
 namespace {
@@ -261,7 +299,8 @@ mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, in
     const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(nt), mla::kGemmKS / 64};
     if (!make_map_3d(&tb, act, dims, strides, box)) return MLA_ERR_CUDA;
   }
-  const size_t smem = 1024 + NSTAGE * mla::gemm_stage_bytes(nt) + (2 * NSTAGE + 1) * 8 + 16;
+  // ring, barriers, TMEM slot and flag, then the 32 (cos, sin) pairs of the q_pe rotation
+  const size_t smem = 1024 + NSTAGE * mla::gemm_stage_bytes(nt) + (2 * NSTAGE + 1) * 8 + 16 + 32 * 16;
   auto kern = mla::proj_gemm_kernel<KTOT, NSTAGE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
