@@ -52,6 +52,32 @@ mla_status launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   return MLA_OK;
 }
 
+// As launch_chained, with the cluster shape set at launch (cluster_x CTAs along x).
+template <typename... KArgs, typename... Args>
+mla_status launch_chained_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                  unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -215,6 +241,33 @@ mla::RopeFreq rope_freq(float rope_base) {
   return f;
 }
 
+// One down-projection + append launch with K split over SPLIT-CTA clusters.
+template <int SPLIT>
+mla_status launch_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const mla_bf16* w_kr,
+                                 const int32_t* seq_ids, const int32_t* pos, mla_bf16* cache, const CacheView& v,
+                                 int32_t n_tokens, float rope_base, void* stream) {
+  using Sh = mla::DpShape<SPLIT>;
+  // 3-D views (64-column chunk, row, chunk index) of the row-major [rows][5120] matrices.
+  CUtensorMap tw, tk, th;
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDHidden) * 2, 128};
+  const cuuint64_t dw[3] = {64, static_cast<cuuint64_t>(mla::kDLat), mla::kDHidden / 64};
+  const cuuint64_t dk[3] = {64, static_cast<cuuint64_t>(mla::kDRope), mla::kDHidden / 64};
+  const cuuint64_t dh[3] = {64, static_cast<cuuint64_t>(n_tokens), mla::kDHidden / 64};
+  const cuuint32_t bw[3] = {64, 128, static_cast<cuuint32_t>(Sh::kChunks)};
+  const cuuint32_t bk[3] = {64, static_cast<cuuint32_t>(mla::kDRope), static_cast<cuuint32_t>(Sh::kChunks)};
+  const cuuint32_t bh[3] = {64, static_cast<cuuint32_t>(mla::kDpNt), static_cast<cuuint32_t>(Sh::kChunks)};
+  if (!make_map_3d(&tw, w_dkv, dw, strides, bw) || !make_map_3d(&tk, w_kr, dk, strides, bk) ||
+      !make_map_3d(&th, h, dh, strides, bh))
+    return MLA_ERR_CUDA;
+  auto kern = mla::down_proj_append_kernel<SPLIT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmemBytes) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  const dim3 grid(SPLIT, mla::kDpMTiles, (n_tokens + mla::kDpNt - 1) / mla::kDpNt);
+  return launch_chained_cluster(kern, grid, dim3(mla::kDpThreads), static_cast<size_t>(Sh::kSmemBytes),
+                                as_stream(stream), SPLIT, tw, tk, th, seq_ids, pos,
+                                reinterpret_cast<__nv_bfloat16*>(cache), v, n_tokens, rope_freq(rope_base));
+}
+
 }  // namespace
 
 extern "C" {
@@ -250,27 +303,35 @@ mla_status mla_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const ml
   if (!aligned16(h) || !aligned16(w_dkv) || !aligned16(w_kr)) return MLA_ERR_INVALID_ARG;
   if (seq_ids == nullptr && n_tokens > desc.num_seqs) return MLA_ERR_INVALID_ARG;
   if (n_tokens > kMaxBatch) return MLA_ERR_UNSUPPORTED;
-  // 3-D views (64-column chunk, row, chunk index) of the row-major [rows][5120] matrices.
-  CUtensorMap tw, tk, th;
-  {
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDHidden) * 2, 128};
-    const cuuint64_t dw[3] = {64, static_cast<cuuint64_t>(mla::kDLat), mla::kDHidden / 64};
-    const cuuint64_t dk[3] = {64, static_cast<cuuint64_t>(mla::kDRope), mla::kDHidden / 64};
-    const cuuint64_t dh[3] = {64, static_cast<cuuint64_t>(n_tokens), mla::kDHidden / 64};
-    const cuuint32_t bw[3] = {64, 128, 2};
-    const cuuint32_t bk[3] = {64, static_cast<cuuint32_t>(mla::kDRope), 2};
-    const cuuint32_t bh[3] = {64, static_cast<cuuint32_t>(mla::kDpNt), 2};
-    if (!make_map_3d(&tw, w_dkv, dw, strides, bw) || !make_map_3d(&tk, w_kr, dk, strides, bk) ||
-        !make_map_3d(&th, h, dh, strides, bh))
-      return MLA_ERR_CUDA;
-  }
-  if (cudaFuncSetAttribute(mla::down_proj_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           mla::kDpSmemBytes) != cudaSuccess)
-    return MLA_ERR_CUDA;
-  const dim3 grid(mla::kDpSplit, mla::kDpMTiles, (n_tokens + mla::kDpNt - 1) / mla::kDpNt);
-  return launch_chained(mla::down_proj_append_kernel, grid, dim3(mla::kDpThreads),
-                        static_cast<size_t>(mla::kDpSmemBytes), as_stream(stream), tw, tk, th, seq_ids, pos,
-                        reinterpret_cast<__nv_bfloat16*>(cache), v, n_tokens, rope_freq(rope_base));
+  // K split over 16-CTA clusters where the device places them, else over 8-CTA clusters.
+  static const int split = [] {
+    auto k16 = mla::down_proj_append_kernel<16>;
+    if (cudaFuncSetAttribute(k16, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+        cudaFuncSetAttribute(k16, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::DpShape<16>::kSmemBytes) !=
+            cudaSuccess) {
+      (void)cudaGetLastError();
+      return 8;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1, 1);
+    cfg.blockDim = dim3(mla::kDpThreads);
+    cfg.dynamicSmemBytes = mla::DpShape<16>::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k16, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    return n >= 1 ? 16 : 8;
+  }();
+  return split == 16 ? launch_project_append<16>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream)
+                     : launch_project_append<8>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream);
 }
 
 }  // extern "C"
