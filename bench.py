@@ -354,6 +354,48 @@ def capture_step_graphs(st, n_rot, stream):
     return steps, phases
 
 
+def measure_project_append(st, steps, warmup):
+    """The next scope row built beside the step: mla_project_append (down-projection of the new
+    tokens' hidden states + cache append) for the step's B new tokens.  Each call reads its 5.9 MB
+    of weights from HBM (L2 flushed before every call, the way a multi-layer step meets them);
+    timed per call with CUDA events.  Runs after the step's own measurements (it rewrites the new
+    tokens' rows of cache copy 0)."""
+    import torch
+    import mla_latent_kv_20_b200 as m
+    from mla_latent_kv_20_b200 import harness as hz
+    B = st["B"]
+    d = mi.down_projection(9001, B)
+    h, wd, wk = hz.bf16_tensor(d.h), hz.bf16_tensor(d.w_dkv), hz.bf16_tensor(d.w_kr)
+    cache = st["layers"][0]["caches"][0]
+    # evict L2 by reading a buffer twice its size (a read leaves no dirty lines to write back
+    # while the timed call runs)
+    flush = torch.ones(64 << 20, dtype=torch.int32, device="cuda")
+
+    def call():
+        m.project_append(h, wd, wk, st["pos"], cache.data, cache.desc, seq_ids=st["seq_ids"],
+                         block_table=cache.block_table)
+
+    for _ in range(max(warmup, 1)):
+        call()
+    torch.cuda.synchronize()
+    n = min(max(steps, 1), 200)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for e0, e1 in ev:
+        flush.max()
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+    ms = sorted(e0.elapsed_time(e1) for e0, e1 in ev)[n // 2]
+    nbytes = 576 * mi.D_HIDDEN * 2 + B * mi.D_HIDDEN * 2 + B * 576 * 2
+    hbm = load_peaks()[0]
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": "down_proj_append_kernel", "tokens": B, "us_per_call": ms * 1e3, "bound": "hbm",
+            "algorithmic_bytes_per_launch": nbytes, "achieved": gbs, "peak": hbm, "unit": "GB/s",
+            "frac": gbs / hbm, "l2": "evicted before each call by reading 256 MB (median of %d calls)" % n}
+
+
 def run_step(st, i):
     """One decode step over every layer of the workload, through plain API calls."""
     for li in range(len(st["layers"])):
@@ -500,6 +542,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
+    next_rows = {"project_append": measure_project_append(st, args.steps, args.warmup)}
     ms, e2e_ms, dec_ms = reduce_max_over_ranks([ms, e2e_ms, dec_ms], world, device=dev)
     if rank != 0:
         return
@@ -537,6 +580,7 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": LAUNCHES_PER_LAYER * n_layers * args.steps,
         "clocks": clocks,
+        "next_rows": next_rows,
     }
     if not args.no_cpu_baseline:
         tok, dt, nseq = time_oracle_sample(st["lens"])
