@@ -98,6 +98,12 @@ def down_projection(seed: int, n_tokens: int, d_hidden: int = D_HIDDEN, d_latent
     return DownProjection(h, w_dkv, w_kr)
 
 
+def output_weight(seed: int, d_hidden: int = D_HIDDEN, n_heads: int = N_HEADS, d_head: int = D_HEAD) -> np.ndarray:
+    """W_O [d, H * d_h] bf16 bits ~ N(0, 0.006^2) ([DR] §3.3 initialisation std)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return _normal_bf16(rng, (d_hidden, n_heads * d_head), DOWN_W_STD)
+
+
 def decode_batch(seed: int, seq_lens, n_heads: int = N_HEADS, d_head: int = D_HEAD,
                  d_latent: int = D_LATENT, d_rope: int = D_ROPE) -> DecodeBatch:
     rng = np.random.Generator(np.random.PCG64(seed))

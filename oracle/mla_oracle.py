@@ -22,6 +22,9 @@ Readings where the pages are silent (each one is listed in the design doc):
   * W_UK is laid out [head, d_h, d_c] (k^C_j = sum_k W_UK[h,j,k] c_k) and W_UV is laid out
     [head, d_c, d_h] (v^C_j = sum_k W_UV[h,k,j] c_k);
   * the new token is appended before attention, so the query attends to itself;
+  * W_O is laid out [d, H d_h] and applied after the un-absorb to the head-major concatenation of
+    the heads' outputs (folding W_U^V into W_O ahead of time would need H x d_c x d weights, four
+    times the bytes of the two-step form, so the two projections stay separate);
   * the down-projections are laid out [out, in] (W_D^KV [d_c, d], W^KR [d_R, d]) and k^R is the
     plain linear projection W^KR h_t (the pages draw the branch h_t -> k^R without naming its
     matrix), rotated by RoPE before it is cached.
@@ -156,6 +159,17 @@ def absorb_q(q_nope: np.ndarray, w_uk: np.ndarray) -> np.ndarray:
 def unabsorb_v(out_lat: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
     """out[..., h, j] = sum_k out_lat[..., h, k] W_UV[h, k, j]   ([..., H, d_c] -> [..., H, d_h])."""
     return np.einsum("...hk,hkj->...hj", np.asarray(out_lat, np.float64), np.asarray(w_uv, np.float64), optimize=True)
+
+
+def output_proj(out: np.ndarray, w_o: np.ndarray) -> np.ndarray:
+    """The attention block's output projection after the un-absorb ([DR] §2.3: W_U^V belongs with
+    the output projection W_O): y[b] = W_O [concat_h out[b, h]], heads concatenated head-major.
+
+    out: [B, H, d_h]; w_o: [d, H * d_h] (output index first).  Returns [B, d].
+    """
+    out = np.asarray(out, dtype=np.float64)
+    B = out.shape[0]
+    return out.reshape(B, -1) @ np.asarray(w_o, dtype=np.float64).T
 
 
 def q_full(q_abs: np.ndarray, q_pe: np.ndarray) -> np.ndarray:

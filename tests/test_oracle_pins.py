@@ -390,3 +390,35 @@ def test_pins_catch_planted_projection_mistakes():
 
     for bad in (parts_swapped, rope_on_latent, unrotated_key):
         assert _fails(check_project_rows, bad), bad.__name__
+
+
+# ------------------------------------------------------------------ output projection
+def check_output_proj(output_proj):
+    rng = np.random.default_rng(12)
+    out = rng.standard_normal((3, 2, 3))          # B = 3, H = 2, d_h = 3
+    w_o = rng.standard_normal((4, 6))             # d = 4, H d_h = 6
+    got = output_proj(out, w_o)
+    assert got.shape == (3, 4)
+    # scalar loops over heads and head dims: y[b][i] = sum_h sum_j W_O[i][h*3 + j] out[b][h][j]
+    bf = [[sum(float(w_o[i, h * 3 + j]) * float(out[b, h, j]) for h in range(2) for j in range(3))
+           for i in range(4)] for b in range(3)]
+    assert np.allclose(got, np.array(bf), rtol=1e-12, atol=1e-12)
+    # one-hot weights pick single (head, dim) entries
+    sel = np.zeros((4, 6))
+    sel[0, 5] = sel[1, 0] = sel[2, 3] = sel[3, 1] = 1.0
+    assert np.array_equal(output_proj(out, sel), np.stack([out[:, 1, 2], out[:, 0, 0], out[:, 1, 0], out[:, 0, 1]], 1))
+
+
+def test_output_proj_pins():
+    check_output_proj(oracle.output_proj)
+
+
+def test_pins_catch_planted_output_proj_mistakes():
+    def dim_major_concat(out, w_o):
+        return np.asarray(out, np.float64).transpose(0, 2, 1).reshape(out.shape[0], -1) @ np.asarray(w_o).T
+
+    def heads_reversed(out, w_o):
+        return oracle.output_proj(np.asarray(out)[:, ::-1, :], w_o)
+
+    for bad in (dim_major_concat, heads_reversed):
+        assert _fails(check_output_proj, bad), bad.__name__
