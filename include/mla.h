@@ -212,6 +212,16 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
                           int32_t batch, void* stream);
 
 /*
+ * (6) Output projection — [DR] §2.3 (W_U^V belongs with the output projection W_O), §3.3 (model
+ *     width d = 5120):  y[b] = W_O [ out[b, 0, :] | ... | out[b, 127, :] ]   (5120 <- 16384)
+ * on the heads' outputs of mla_unabsorb_v, concatenated head-major.  Products in fp32 (exact for
+ * bf16), sums over the 16384 inputs in fp32, one bf16 rounding of y.
+ *   out [batch, 128, 128] bf16     w_o [5120, 16384] bf16 (output index first)     y [batch, 5120] bf16
+ * batch == 0 is a no-op; batch must be <= 65536.
+ */
+mla_status mla_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y, int32_t batch, void* stream);
+
+/*
  * Read and clear the sticky device error word of the current device: bits 0..7 are MLA_DEVERR_*
  * flags; when MLA_DEVERR_WAIT_TIMEOUT is set, bits 8..15 hold the id of the first pipeline wait
  * that gave up (a diagnostic for locating a protocol error).  Synchronises the device.

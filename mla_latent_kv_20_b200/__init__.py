@@ -52,6 +52,7 @@ def _load():
         "mla_version": (I32, []),
         "mla_cache_append": (ctypes.c_int, [P, P, P, P, P, P, CacheDesc, I32, F32, P]),
         "mla_project_append": (ctypes.c_int, [P, P, P, P, P, P, P, CacheDesc, I32, F32, P]),
+        "mla_output_proj": (ctypes.c_int, [P, P, P, I32, P]),
         "mla_absorb_q": (ctypes.c_int, [P, P, P, P, P, I32, F32, P]),
         "mla_decode_num_splits": (I32, [I32, I32, I32]),
         "mla_decode_workspace_size": (SZ, [I32, I32, I32]),
@@ -108,6 +109,11 @@ def project_append(h, w_dkv, w_kr, pos, cache, desc: CacheDesc, *, seq_ids=None,
     n = h.shape[0] if n_tokens is None else n_tokens
     _check(lib.mla_project_append(_ptr(h), _ptr(w_dkv), _ptr(w_kr), _ptr(seq_ids), _ptr(pos), _ptr(cache),
                                   _ptr(block_table), desc, n, rope_base, _stream(stream)), "mla_project_append")
+
+
+def output_proj(out, w_o, y, *, stream=None, batch: int | None = None):
+    b = out.shape[0] if batch is None else batch
+    _check(lib.mla_output_proj(_ptr(out), _ptr(w_o), _ptr(y), b, _stream(stream)), "mla_output_proj")
 
 
 def absorb_q(q_nope, q_pe, w_uk, q_full, *, q_pos=None, rope_base: float = 10000.0, stream=None,

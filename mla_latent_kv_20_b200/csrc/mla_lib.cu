@@ -17,6 +17,7 @@
 #include "decode_common.cuh"
 #include "decode_tc.cuh"
 #include "down_proj.cuh"
+#include "out_proj.cuh"
 #include "gemm_tc.cuh"
 #include "ptx.cuh"
 
@@ -241,6 +242,52 @@ mla::RopeFreq rope_freq(float rope_base) {
   return f;
 }
 
+// Whether the device places 16-CTA clusters of `kernel` (non-portable size) with this block size
+// and dynamic shared memory; sets the attributes the launch needs.
+template <typename K>
+bool cluster16_ok(K kernel, int threads, int smem) {
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(16, 1, 1);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 16;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  return n >= 1;
+}
+
+// One output-projection launch with K split over SPLIT-CTA clusters.
+template <int SPLIT>
+mla_status launch_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y, int32_t batch, void* stream) {
+  CUtensorMap tw, tx;
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kOpIn) * 2, 128};
+  const cuuint64_t dw[3] = {64, static_cast<cuuint64_t>(mla::kOpOut), mla::kOpIn / 64};
+  const cuuint64_t dx[3] = {64, static_cast<cuuint64_t>(batch), mla::kOpIn / 64};
+  const cuuint32_t bw[3] = {64, 128, static_cast<cuuint32_t>(mla::kOpKS / 64)};
+  const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(mla::kOpNt), static_cast<cuuint32_t>(mla::kOpKS / 64)};
+  if (!make_map_3d(&tw, w_o, dw, strides, bw) || !make_map_3d(&tx, out, dx, strides, bx)) return MLA_ERR_CUDA;
+  auto kern = mla::out_proj_kernel<SPLIT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kOpSmemBytes) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  const dim3 grid(SPLIT, mla::kOpMTiles, (batch + mla::kOpNt - 1) / mla::kOpNt);
+  return launch_chained_cluster(kern, grid, dim3(mla::kOpThreads), static_cast<size_t>(mla::kOpSmemBytes),
+                                as_stream(stream), SPLIT, tw, tx, reinterpret_cast<__nv_bfloat16*>(y), batch);
+}
+
 // One down-projection + append launch with K split over SPLIT-CTA clusters.
 template <int SPLIT>
 mla_status launch_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const mla_bf16* w_kr,
@@ -304,34 +351,20 @@ mla_status mla_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const ml
   if (seq_ids == nullptr && n_tokens > desc.num_seqs) return MLA_ERR_INVALID_ARG;
   if (n_tokens > kMaxBatch) return MLA_ERR_UNSUPPORTED;
   // K split over 16-CTA clusters where the device places them, else over 8-CTA clusters.
-  static const int split = [] {
-    auto k16 = mla::down_proj_append_kernel<16>;
-    if (cudaFuncSetAttribute(k16, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
-        cudaFuncSetAttribute(k16, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::DpShape<16>::kSmemBytes) !=
-            cudaSuccess) {
-      (void)cudaGetLastError();
-      return 8;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(16, 1, 1);
-    cfg.blockDim = dim3(mla::kDpThreads);
-    cfg.dynamicSmemBytes = mla::DpShape<16>::kSmemBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 16;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k16, &cfg) != cudaSuccess) {
-      (void)cudaGetLastError();
-      n = 0;
-    }
-    return n >= 1 ? 16 : 8;
-  }();
+  static const int split = cluster16_ok(mla::down_proj_append_kernel<16>, mla::kDpThreads,
+                                        mla::DpShape<16>::kSmemBytes) ? 16 : 8;
   return split == 16 ? launch_project_append<16>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream)
                      : launch_project_append<8>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream);
+}
+
+mla_status mla_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y, int32_t batch, void* stream) {
+  if (batch < 0 || batch > kMaxBatch) return batch < 0 ? MLA_ERR_INVALID_ARG : MLA_ERR_UNSUPPORTED;
+  if (batch == 0) return MLA_OK;
+  if (out == nullptr || w_o == nullptr || y == nullptr) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(w_o) || !aligned16(y)) return MLA_ERR_INVALID_ARG;
+  // 8-CTA clusters: twice as many clusters are resident at once as with 16 (measured 57 vs 72 us
+  // per call on 32 sequences with the weight coming from HBM).
+  return launch_output_proj<8>(out, w_o, y, batch, stream);
 }
 
 }  // extern "C"
