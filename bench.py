@@ -396,6 +396,43 @@ def measure_project_append(st, steps, warmup):
             "frac": gbs / hbm, "l2": "evicted before each call by reading 256 MB (median of %d calls)" % n}
 
 
+def measure_output_proj(st, steps, warmup):
+    """The next scope row built after the step: mla_output_proj (W_O over the step's un-absorbed
+    head outputs, y [B, 5120]).  The 168 MB weight (seeded on the device) is larger than L2, so
+    every call streams it from HBM; timed per call with CUDA events (median)."""
+    import torch
+    import mla_latent_kv_20_b200 as m
+    B = st["B"]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(9002)
+    w_o = (torch.randn((mi.D_HIDDEN, mi.N_HEADS * mi.D_HEAD), device="cuda", generator=gen) *
+           mi.DOWN_W_STD).to(torch.bfloat16)
+    y = torch.empty((B, mi.D_HIDDEN), dtype=torch.bfloat16, device="cuda")
+
+    def call():
+        m.output_proj(st["out"], w_o, y)
+
+    for _ in range(max(warmup, 1)):
+        call()
+    torch.cuda.synchronize()
+    n = min(max(steps, 1), 200)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for e0, e1 in ev:
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+    ms = sorted(e0.elapsed_time(e1) for e0, e1 in ev)[n // 2]
+    nbytes = mi.D_HIDDEN * mi.N_HEADS * mi.D_HEAD * 2 + B * mi.N_HEADS * mi.D_HEAD * 2 + B * mi.D_HIDDEN * 2
+    hbm = load_peaks()[0]
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del w_o
+    return {"kernel": "out_proj_kernel", "sequences": B, "us_per_call": ms * 1e3, "bound": "hbm",
+            "algorithmic_bytes_per_launch": nbytes, "achieved": gbs, "peak": hbm, "unit": "GB/s",
+            "frac": gbs / hbm, "l2": "weight (168 MB) larger than L2 (median of %d back-to-back calls)" % n}
+
+
 def run_step(st, i):
     """One decode step over every layer of the workload, through plain API calls."""
     for li in range(len(st["layers"])):
@@ -542,7 +579,8 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
-    next_rows = {"project_append": measure_project_append(st, args.steps, args.warmup)}
+    next_rows = {"project_append": measure_project_append(st, args.steps, args.warmup),
+                 "output_proj": measure_output_proj(st, args.steps, args.warmup)}
     ms, e2e_ms, dec_ms = reduce_max_over_ranks([ms, e2e_ms, dec_ms], world, device=dev)
     if rank != 0:
         return
