@@ -305,7 +305,7 @@ def recorded_traffic(workload):
 
 CLOCK_WINDOW_S = 1.0     # clock-sampling replay window when the timed region is too short to sample
 
-LAUNCHES_PER_LAYER = 5   # append, absorb GEMM (with the q_pe rotation), decode ranges, combine, un-absorb GEMM
+LAUNCHES_PER_LAYER = 4   # append + absorb GEMM (with the q_pe rotation), decode ranges, combine, un-absorb GEMM
 
 
 GRAPH_PHASES = ("append_absorb", "decode_attn", "unabsorb_v")
@@ -318,9 +318,10 @@ def layer_phase(st, i, li, k):
     cache = layer["caches"][i % len(layer["caches"])]
     d = layer["dev"]
     if k == 0:
-        m.cache_append(d["c_new"], d["kr_new"], st["pos"], cache.data, cache.desc, seq_ids=st["seq_ids"],
-                       block_table=cache.block_table)
-        m.absorb_q(d["q_nope"], d["q_pe"], layer["w_uk"], st["q_full"], q_pos=st["pos"])
+        # append the new tokens' rows and absorb their queries in one launch
+        m.append_absorb(d["c_new"], d["kr_new"], st["pos"], cache.data, cache.desc, d["q_nope"], d["q_pe"],
+                        layer["w_uk"], st["q_full"], seq_ids=st["seq_ids"], block_table=cache.block_table,
+                        q_pos=st["pos"])
     elif k == 1:
         m.decode_attn(st["q_full"], cache.data, cache.seq_lens, cache.desc, st["workspace"], st["out_lat"],
                       lse=st["lse"], block_table=cache.block_table, num_splits=st["splits"])

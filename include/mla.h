@@ -132,6 +132,19 @@ mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int3
                         void* stream);
 
 /*
+ * (1)+(2) in one launch: the cache append of n_tokens new tokens (exactly mla_cache_append's rows
+ * and device checks) and the query absorption of batch queries (exactly mla_absorb_q's q_full),
+ * for a decode step that appends the new tokens' rows and absorbs their queries together: one
+ * kernel instead of two in the step's chain.  Arguments as in those two calls; n_tokens == 0 skips
+ * the append, batch == 0 the absorption.
+ */
+mla_status mla_append_absorb(const mla_bf16* c_new, const mla_bf16* kr_new, const int32_t* seq_ids,
+                             const int32_t* pos, mla_bf16* cache, const int32_t* block_table,
+                             mla_cache_desc desc, int32_t n_tokens, const mla_bf16* q_nope,
+                             const mla_bf16* q_pe, const int32_t* q_pos, const mla_bf16* w_uk,
+                             mla_bf16* q_full, int32_t batch, float rope_base, void* stream);
+
+/*
  * Number of work ranges P (one CTA pair each) the decode divides the batch's cached tokens into:
  * for num_splits == 0 (auto) as many as the device keeps resident, but at most one per two
  * 128-token tiles of batch x max_seq_len; num_splits itself when it is positive (clamped to

@@ -53,6 +53,7 @@ def _load():
         "mla_cache_append": (ctypes.c_int, [P, P, P, P, P, P, CacheDesc, I32, F32, P]),
         "mla_project_append": (ctypes.c_int, [P, P, P, P, P, P, P, CacheDesc, I32, F32, P]),
         "mla_output_proj": (ctypes.c_int, [P, P, P, I32, P]),
+        "mla_append_absorb": (ctypes.c_int, [P, P, P, P, P, P, CacheDesc, I32, P, P, P, P, P, I32, F32, P]),
         "mla_absorb_q": (ctypes.c_int, [P, P, P, P, P, I32, F32, P]),
         "mla_decode_num_splits": (I32, [I32, I32, I32]),
         "mla_decode_workspace_size": (SZ, [I32, I32, I32]),
@@ -109,6 +110,14 @@ def project_append(h, w_dkv, w_kr, pos, cache, desc: CacheDesc, *, seq_ids=None,
     n = h.shape[0] if n_tokens is None else n_tokens
     _check(lib.mla_project_append(_ptr(h), _ptr(w_dkv), _ptr(w_kr), _ptr(seq_ids), _ptr(pos), _ptr(cache),
                                   _ptr(block_table), desc, n, rope_base, _stream(stream)), "mla_project_append")
+
+
+def append_absorb(c_new, kr_new, pos, cache, desc: CacheDesc, q_nope, q_pe, w_uk, q_full, *, seq_ids=None,
+                  block_table=None, q_pos=None, rope_base: float = 10000.0, stream=None):
+    """mla_cache_append and mla_absorb_q in one launch."""
+    _check(lib.mla_append_absorb(_ptr(c_new), _ptr(kr_new), _ptr(seq_ids), _ptr(pos), _ptr(cache), _ptr(block_table),
+                                 desc, c_new.shape[0], _ptr(q_nope), _ptr(q_pe), _ptr(q_pos), _ptr(w_uk), _ptr(q_full),
+                                 q_nope.shape[0], rope_base, _stream(stream)), "mla_append_absorb")
 
 
 def output_proj(out, w_o, y, *, stream=None, batch: int | None = None):

@@ -31,6 +31,18 @@ constexpr int kGemmKS = 128;         // contraction rows per stage
 // Stage bytes: weight KS x 128 (two 64-wide M chunks) + activation nt x KS, bf16.
 __host__ __device__ constexpr int gemm_stage_bytes(int nt) { return kGemmKS * 256 + nt * kGemmKS * 2; }
 
+// New tokens' cache rows written by the query-side launch (cache == nullptr: none): the rows of
+// mla_cache_append, row = [c_new[i] | RoPE(kr_new[i], pos[i])] at (seq_ids ? seq_ids[i] : i, pos[i]).
+struct AppendJob {
+  const uint4* c_new;              // [n_tokens, 512] bf16
+  const __nv_bfloat162* kr_new;    // [n_tokens, 64] bf16, before RoPE
+  const int32_t* seq_ids;          // [n_tokens] or null
+  const int32_t* pos;              // [n_tokens]
+  uint4* cache;
+  CacheView v;
+  int n_tokens;
+};
+
 // KTOT: contraction length (128 for absorption, 512 for un-absorption).
 // tmA: 3-D view of the weight (64-element M chunk, contraction row = h * KTOT + k, M chunk index);
 //      box {64, KS, 2}: smem [chunk][KS rows][128 B].
@@ -39,14 +51,15 @@ __host__ __device__ constexpr int gemm_stage_bytes(int nt) { return kGemmKS * 25
 // out element (n, h, m) is stored at out[n * out_bstride + h * out_hstride + m].
 // Query side only (qpe != nullptr, KTOT = d_h): the epilogue warps also fill the RoPE part of the
 // query rows, out[n, h, 512:576] = q_pe[n, h, :] rotated at q_pos[n] (or copied when q_pos is
-// null), while the MMAs run: CTA c (linear index) takes rows n = c, c + #CTAs, ... for all 128
-// heads, so each row's 32 angles are formed once.
+// null), and write the new tokens' cache rows of `app` (if any), while the MMAs run: CTA c (linear
+// index) takes rows n = c, c + #CTAs, ... (for all 128 heads, so each row's 32 angles are formed
+// once).
 template <int KTOT, int NSTAGE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      __nv_bfloat16* __restrict__ out, int batch, int nt, int64_t out_bstride,
                      int out_hstride, const uint4* __restrict__ qpe, const int32_t* __restrict__ q_pos,
-                     const RopeFreq rope) {
+                     const RopeFreq rope, const AppendJob app) {
   constexpr int KSTAGES = KTOT / kGemmKS;
   static_assert(KTOT % kGemmKS == 0, "contraction length");
   extern __shared__ uint8_t smem_raw[];
@@ -151,13 +164,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // Warp w owns outputs m0 + 32w + [0, 32) for every n of the tile.  Lane = m in TMEM, so the
     // warp's [n][32 m] block goes through a stage in the (now idle) operand ring: each lane writes
     // its column, then every global store instruction covers eight whole 64-byte rows.
-    if (qpe != nullptr) {
+    const int nrows = max(qpe != nullptr ? batch : 0, app.cache != nullptr ? app.n_tokens : 0);
+    {
       // Angle and rotation in fp64, one rounding per output (the same arithmetic as the cache
-      // append's RoPE).  cs_sn: this row's 32 (cos, sin) pairs, formed by threads 0..31.
+      // append's RoPE).  cs_sn: a query row's 32 (cos, sin) pairs, formed by threads 0..31.
       double* cs_sn = reinterpret_cast<double*>(tmem_slot + 4);
       const int ncta = gridDim.x * gridDim.y * gridDim.z;
       const int c = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-      for (int n = c; n < batch; n += ncta) {
+      for (int n = c; n < nrows; n += ncta) {
+        if (app.cache != nullptr && n < app.n_tokens) {
+          // new token n: threads 0..63 copy the latent (16 B each), 64..95 rotate one key pair each
+          const int seq = app.seq_ids ? app.seq_ids[n] : n;
+          const int p = app.pos[n];
+          const int capacity = app.v.page_size == 0 ? app.v.max_seq_len : app.v.max_blocks * kPage;
+          if (p < 0 || p >= capacity || seq < 0 || seq >= app.v.num_seqs) {
+            if (threadIdx.x == 0) set_dev_error(0x1);
+          } else if (threadIdx.x < 96) {
+            const int64_t crow = cache_row(app.v, seq, p);
+            if (crow >= 0) {
+              const int t = threadIdx.x;
+              if (t < 64) {
+                app.cache[crow * (kDRow / 8) + t] = app.c_new[static_cast<int64_t>(n) * (kDLat / 8) + t];
+              } else {
+                const int pr = t - 64;
+                double sn, cs;
+                sincos(static_cast<double>(p) * rope.inv_freq[pr], &sn, &cs);
+                reinterpret_cast<__nv_bfloat162*>(app.cache + crow * (kDRow / 8) + kDLat / 8)[pr] =
+                    rope_pair(app.kr_new[static_cast<int64_t>(n) * (kDRope / 2) + pr], cs, sn);
+              }
+            }
+          }
+        }
+        if (qpe == nullptr || n >= batch) continue;   // uniform across the 128 threads
         if (q_pos != nullptr && threadIdx.x < kDRope / 2) {
           double sn, cs;
           sincos(static_cast<double>(q_pos[n]) * rope.inv_freq[threadIdx.x], &sn, &cs);

@@ -374,7 +374,8 @@ namespace {
 template <int KTOT, int NSTAGE>
 mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, int batch, __nv_bfloat16* out,
                             int64_t out_bstride, int out_hstride, cudaStream_t stream, const void* qpe = nullptr,
-                            const int32_t* q_pos = nullptr, float rope_base = 10000.f) {
+                            const int32_t* q_pos = nullptr, float rope_base = 10000.f,
+                            const mla::AppendJob* app = nullptr) {
   // Weight viewed as [heads * KTOT rows][m_total cols]: 3-D (64-element M chunk, row, M chunk index),
   // box {64, KS, 2}.  Activation as [batch rows][heads * KTOT cols]: 3-D (64-element K slab, batch
   // row, slab index), box {64, nt, KS / 64}.
@@ -401,7 +402,8 @@ mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, in
     return MLA_ERR_CUDA;
   dim3 grid(m_total / 128, mla::kHeads, (batch + nt - 1) / nt);
   return launch_chained(kern, grid, dim3(mla::kGemmThreads), smem, stream, ta, tb, out, batch, nt, out_bstride,
-                        out_hstride, reinterpret_cast<const uint4*>(qpe), q_pos, rope_freq(rope_base));
+                        out_hstride, reinterpret_cast<const uint4*>(qpe), q_pos, rope_freq(rope_base),
+                        app != nullptr ? *app : mla::AppendJob{nullptr, nullptr, nullptr, nullptr, nullptr, {}, 0});
 }
 
 }  // namespace
@@ -422,6 +424,34 @@ mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int3
   return launch_proj_gemm<mla::kDHead, 1>(w_uk, mla::kDLat, q_nope, batch, reinterpret_cast<__nv_bfloat16*>(q_full),
                                           static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow, s, q_pe, q_pos,
                                           rope_base);
+}
+
+mla_status mla_append_absorb(const mla_bf16* c_new, const mla_bf16* kr_new, const int32_t* seq_ids,
+                             const int32_t* pos, mla_bf16* cache, const int32_t* block_table, mla_cache_desc desc,
+                             int32_t n_tokens, const mla_bf16* q_nope, const mla_bf16* q_pe, const int32_t* q_pos,
+                             const mla_bf16* w_uk, mla_bf16* q_full, int32_t batch, float rope_base, void* stream) {
+  // the checks of mla_cache_append ...
+  if (n_tokens < 0 || !(rope_base > 0.f) || !std::isfinite(rope_base)) return MLA_ERR_INVALID_ARG;
+  CacheView v;
+  const mla_status st = check_cache(desc, cache, block_table, &v);
+  if (st != MLA_OK) return st;
+  if (n_tokens > 0) {
+    if (c_new == nullptr || kr_new == nullptr || pos == nullptr || !aligned16(c_new) || !aligned16(kr_new))
+      return MLA_ERR_INVALID_ARG;
+    if (seq_ids == nullptr && n_tokens > desc.num_seqs) return MLA_ERR_INVALID_ARG;
+    if (n_tokens > kMaxBatch) return MLA_ERR_UNSUPPORTED;
+  }
+  // ... and of mla_absorb_q
+  if (batch < 0 || batch > kMaxBatch) return batch < 0 ? MLA_ERR_INVALID_ARG : MLA_ERR_UNSUPPORTED;
+  if (batch == 0) return n_tokens == 0 ? MLA_OK : mla_cache_append(c_new, kr_new, seq_ids, pos, cache, block_table,
+                                                                    desc, n_tokens, rope_base, stream);
+  if (q_nope == nullptr || q_pe == nullptr || w_uk == nullptr || q_full == nullptr) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(w_uk) || !aligned16(q_full)) return MLA_ERR_INVALID_ARG;
+  const mla::AppendJob app{reinterpret_cast<const uint4*>(c_new), reinterpret_cast<const __nv_bfloat162*>(kr_new),
+                           seq_ids, pos, reinterpret_cast<uint4*>(cache), v, n_tokens};
+  return launch_proj_gemm<mla::kDHead, 1>(w_uk, mla::kDLat, q_nope, batch, reinterpret_cast<__nv_bfloat16*>(q_full),
+                                          static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow,
+                                          as_stream(stream), q_pe, q_pos, rope_base, &app);
 }
 
 mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf16* out, int32_t batch,

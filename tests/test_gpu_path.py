@@ -221,3 +221,36 @@ def test_full_step_vs_explicit_oracle(env, lens, paged):
                              f64(w.w_uk), f64(w.w_uv), SCALE, q_pos=qpos, form="explicit")
     assert_full_path(f64(hz.bf16_bits(out)), ref["out"])
     assert np.abs(lse.cpu().numpy() - ref["lse"]).max() <= 5e-3
+
+
+# ----------------------------------------------------------------------------- fused append + absorb
+@pytest.mark.parametrize("paged,n_tokens,batch", [(False, 4, 4), (True, 4, 4), (False, 7, 3), (True, 2, 33)])
+def test_append_absorb_equals_separate_calls(env, paged, n_tokens, batch):
+    """mla_append_absorb writes exactly the rows of mla_cache_append and the q_full of mla_absorb_q."""
+    m, hz, torch = env
+    lens = [5, 64, 65, 300]
+    table, nblk = mi.block_permutation(301, lens) if paged else (None, 0)
+    c1 = hz.Cache(lens, paged, table, nblk)
+    c2 = hz.Cache(lens, paged, table, nblk)
+    rng = np.random.default_rng(302 + n_tokens)
+    seq = rng.integers(0, len(lens), n_tokens).astype(np.int32)
+    pos = np.array([rng.integers(0, lens[s]) for s in seq], dtype=np.int32)
+    _, keep = np.unique(seq.astype(np.int64) * 100000 + pos, return_index=True)
+    seq, pos = seq[np.sort(keep)], pos[np.sort(keep)]
+    b = mi.decode_batch(303, [1] * batch)
+    w = mi.layer_weights(304)
+    c_new = hz.bf16_tensor(mi.f64_to_bf16(rng.standard_normal((len(seq), 512))))
+    kr_new = hz.bf16_tensor(mi.f64_to_bf16(rng.standard_normal((len(seq), 64))))
+    t_seq, t_pos = torch.from_numpy(seq).cuda(), torch.from_numpy(pos).cuda()
+    q_pos = torch.from_numpy(rng.integers(0, 131072, batch).astype(np.int32)).cuda()
+    qn, qp, wuk = hz.bf16_tensor(b.q_nope), hz.bf16_tensor(b.q_pe), hz.bf16_tensor(w.w_uk)
+    qf1 = torch.empty((batch, 128, 576), dtype=torch.bfloat16, device="cuda")
+    qf2 = torch.empty_like(qf1)
+    m.cache_append(c_new, kr_new, t_pos, c1.data, c1.desc, seq_ids=t_seq, block_table=c1.block_table)
+    m.absorb_q(qn, qp, wuk, qf1, q_pos=q_pos)
+    m.append_absorb(c_new, kr_new, t_pos, c2.data, c2.desc, qn, qp, wuk, qf2, seq_ids=t_seq,
+                    block_table=c2.block_table, q_pos=q_pos)
+    torch.cuda.synchronize()
+    _clear(m)
+    assert torch.equal(c1.data, c2.data)
+    assert torch.equal(qf1, qf2)
