@@ -235,6 +235,17 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
 mla_status mla_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y, int32_t batch, void* stream);
 
 /*
+ * Self-test of the bounded waits every pipeline of this library uses (the pages have no
+ * counterpart; this is failure detection without a fault): launches one CTA that waits on a
+ * barrier nothing arrives on, with the wait loop of the pipelines and a limit of limit_us
+ * (1 .. 2,000,000).  The wait must give up: result[0] = 1 if it completed (a broken wait),
+ * 0 if it gave up; result[1] = microseconds waited.  Giving up sets MLA_DEVERR_WAIT_TIMEOUT with
+ * wait site 0x7F (read and clear it with mla_get_device_error); the context stays usable.
+ *   result: device int32[2] (written)
+ */
+mla_status mla_selftest_wait_timeout(uint32_t limit_us, int32_t* result, void* stream);
+
+/*
  * Read and clear the sticky device error word of the current device: bits 0..7 are MLA_DEVERR_*
  * flags; when MLA_DEVERR_WAIT_TIMEOUT is set, bits 8..15 hold the id of the first pipeline wait
  * that gave up (a diagnostic for locating a protocol error).  Synchronises the device.

@@ -54,6 +54,7 @@ def _load():
         "mla_project_append": (ctypes.c_int, [P, P, P, P, P, P, P, CacheDesc, I32, F32, P]),
         "mla_output_proj": (ctypes.c_int, [P, P, P, I32, P]),
         "mla_append_absorb": (ctypes.c_int, [P, P, P, P, P, P, CacheDesc, I32, P, P, P, P, P, I32, F32, P]),
+        "mla_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, P, P]),
         "mla_absorb_q": (ctypes.c_int, [P, P, P, P, P, I32, F32, P]),
         "mla_decode_num_splits": (I32, [I32, I32, I32]),
         "mla_decode_workspace_size": (SZ, [I32, I32, I32]),
@@ -118,6 +119,11 @@ def append_absorb(c_new, kr_new, pos, cache, desc: CacheDesc, q_nope, q_pe, w_uk
     _check(lib.mla_append_absorb(_ptr(c_new), _ptr(kr_new), _ptr(seq_ids), _ptr(pos), _ptr(cache), _ptr(block_table),
                                  desc, c_new.shape[0], _ptr(q_nope), _ptr(q_pe), _ptr(q_pos), _ptr(w_uk), _ptr(q_full),
                                  q_nope.shape[0], rope_base, _stream(stream)), "mla_append_absorb")
+
+
+def selftest_wait_timeout(limit_us: int, result, *, stream=None):
+    """Run the bounded-wait self-test; result is a device int32[2] tensor (see mla.h)."""
+    _check(lib.mla_selftest_wait_timeout(limit_us, _ptr(result), _stream(stream)), "mla_selftest_wait_timeout")
 
 
 def output_proj(out, w_o, y, *, stream=None, batch: int | None = None):

@@ -199,6 +199,25 @@ constexpr int kMaxSplits = 1024;
 
 }  // namespace
 
+namespace mla {
+// Self-test of the bounded wait: one thread waits on a barrier nothing arrives on, which must give
+// up after limit_ns (setting the wait-timeout error with site 0x7F) and return normally.
+__global__ void selftest_wait_kernel(uint64_t limit_ns, int32_t* result) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    const bool completed = mbar_wait_for(&bar, 0, 0x7F, limit_ns);
+    result[0] = completed ? 1 : 0;
+    result[1] = static_cast<int32_t>((globaltimer_ns() - t0) / 1000);
+  }
+}
+}  // namespace mla
+
 extern "C" {
 
 const char* mla_status_string(mla_status s) {
@@ -355,6 +374,12 @@ mla_status mla_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const ml
                                         mla::DpShape<16>::kSmemBytes) ? 16 : 8;
   return split == 16 ? launch_project_append<16>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream)
                      : launch_project_append<8>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream);
+}
+
+mla_status mla_selftest_wait_timeout(uint32_t limit_us, int32_t* result, void* stream) {
+  if (result == nullptr || limit_us == 0 || limit_us > 2000000u) return MLA_ERR_INVALID_ARG;
+  mla::selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(static_cast<uint64_t>(limit_us) * 1000ull, result);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 mla_status mla_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y, int32_t batch, void* stream) {

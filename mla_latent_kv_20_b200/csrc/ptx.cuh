@@ -80,17 +80,22 @@ __device__ __forceinline__ void wait_timed_out(uint32_t site) {
   set_dev_error(0x8);
   atomicCAS(&g_mla_dev_error_site, 0, static_cast<int>(site));
 }
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t site = 1) {
+// The loop of every bounded CTA-scope wait, with the limit as an argument (the pipelines use
+// kWaitLimitNs through mbar_wait; the library's wait self-test uses a short limit).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t site, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(a, parity)) return true;
-    if ((it & 255u) == 255u && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 255u) == 255u && globaltimer_ns() - t0 > limit_ns) {
       wait_timed_out(site);
       return false;
     }
   }
+}
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t site = 1) {
+  return mbar_wait_for(bar, parity, site, kWaitLimitNs);
 }
 __device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t site = 1) {
   const uint32_t a = smem_u32(bar);

@@ -102,3 +102,15 @@ def test_decode_validation_and_workspace(mla):
     big = mla.contiguous_desc(16385, 64)
     assert lib.mla_decode_attn(*args(FAKE, 1 << 40, batch=16385, desc=big)) == 2   # batch beyond the plan's limit
     assert lib.mla_get_device_error(None) == 1
+
+
+def test_wait_selftest_validates_arguments(mla):
+    """Host-side checks of the bounded-wait self-test (no launch, no GPU needed)."""
+    import ctypes
+    lib = ctypes.CDLL(mla.LIB_PATH)
+    lib.mla_selftest_wait_timeout.restype = ctypes.c_int
+    lib.mla_selftest_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p]
+    bogus = ctypes.c_void_p(16)
+    assert lib.mla_selftest_wait_timeout(0, bogus, None) == 1           # MLA_ERR_INVALID_ARG
+    assert lib.mla_selftest_wait_timeout(2000001, bogus, None) == 1
+    assert lib.mla_selftest_wait_timeout(1000, None, None) == 1
