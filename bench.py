@@ -282,7 +282,7 @@ def setup_replica(name, device):
 # counters were taken, and the traffic is reported as null.
 TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh", "csrc/mla_lib.cu")
 MEASURED_TRAFFIC = {   # workload -> {"bytes": int, "sha256": str, "profile": str}
-    "b32_l4096": {"bytes": 155814656 + 4873472 + 16858624, "sha256": "10213514962ef0690644c6ead6b2ef45653667666f4e4296c3e601a7a1f8a2c0",
+    "b32_l4096": {"bytes": 155796480 + 3692032 + 16858368, "sha256": "c207dcc53529bbe15f8b1ae24d8d9d575d0a93708359ee0a790fee19e32dac5c",
                   "profile": "profiles/decode_tc_b32_l4096.md (decode + combine, ncu cache flush per kernel)"},
 }
 
