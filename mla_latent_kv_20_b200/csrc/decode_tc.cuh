@@ -94,6 +94,7 @@ struct DecodeTcArgs {
   Workspace ws;
   __nv_bfloat16* out_lat;
   float* lse;
+  const uint8_t* cache;   // the cache buffer (L2 prefetch addresses)
 };
 
 // This CTA pair's work range, computed once per CTA at entry (the cursor's starting state).
@@ -427,6 +428,26 @@ __device__ __forceinline__ void store_rows_128b(uint8_t* stage, const uint32_t (
 }
 
 // ------------------------------------------------------------------------------ softmax warps
+// L2 prefetch of the K rows the producer will copy kTcPfDist tiles later.  A K copy is issued only
+// once QK^T has released the slot it refills (a single K slot per part), so its HBM latency sits
+// on the critical loop; with the rows already in L2 it shrinks to the L2 latency.  The softmax
+// warps issue the prefetches (plain prefetch.global.L2, not the TMA unit, which serialises its
+// copies): this CTA's 64 rows of the tile are one contiguous 72 KB run (a 64-token page, or 64
+// consecutive rows of a contiguous cache), 576 lines over 256 threads, once per tile.
+constexpr int kTcPfDist = 2;
+__device__ __forceinline__ void tc_prefetch_tile(const DecodeTcArgs& a, int b, int tok0, int t_end) {
+  if (tok0 >= t_end) return;
+  const int64_t r = cache_row(a.v, b, tok0);
+  if (r < 0) return;
+  // rows of one page (paged) and of the buffer only
+  int n = min(64, t_end - tok0);
+  if (a.v.page_size != 0) n = min(n, kPage - tok0 % kPage);
+  if (a.v.num_rows - r < n) n = static_cast<int>(a.v.num_rows - r);
+  const uint8_t* base = a.cache + r * (kDRow * 2);
+  for (int L = threadIdx.x; L < n * (kDRow * 2 / 128); L += 32 * kTcSoftmaxWarps)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(base + 128 * L));
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -533,6 +554,8 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
   const int t_begin = sg.tok_begin, t_end = sg.tok_end, n_tiles = sg.n_tiles;
   float m_used = -INFINITY;
   float l_run = 0.f;
+  for (int d = 1; d < kTcPfDist && d < n_tiles; ++d)
+    tc_prefetch_tile(a, sg.b, t_begin + d * kTcTile + 64 * static_cast<int>(rank), t_end);
   for (int i = 0; i < n_tiles && ok; ++i, ++g) {
     const int j = g & 1;
     if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[j], static_cast<uint32_t>(g >> 1) & 1u, 0x30))) {
@@ -631,6 +654,8 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
       fence_release_smem_to_cluster();
       mbar_arrive_relaxed(lbar(&bars->p_full));
     }
+    if (i + kTcPfDist < n_tiles)
+      tc_prefetch_tile(a, sg.b, t_begin + (i + kTcPfDist) * kTcTile + 64 * static_cast<int>(rank), t_end);
   }
   // ---- epilogue of the segment (every warp passes the same barriers, also after a failure)
   if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_final, static_cast<uint32_t>(k) & 1u, 0x33))) ok = false;

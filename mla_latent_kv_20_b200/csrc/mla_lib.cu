@@ -541,6 +541,7 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
   a.ws = mla::ws_carve(workspace, P);
   a.out_lat = reinterpret_cast<__nv_bfloat16*>(out_lat);
   a.lse = lse;
+  a.cache = reinterpret_cast<const uint8_t*>(cache);
   CUtensorMap tka, tkb, tv, tq;
   if (!make_map_slabs(&tka, cache, desc.num_rows, mla::kTcKSlabsA) ||
       !make_map_slabs(&tkb, cache, desc.num_rows, mla::kTcKSlabsB) || !make_map_vbox(&tv, cache, desc.num_rows) ||
