@@ -432,17 +432,17 @@ __device__ __forceinline__ void store_rows_128b(uint8_t* stage, const uint32_t (
 // once QK^T has released the slot it refills (a single K slot per part), so its HBM latency sits
 // on the critical loop; with the rows already in L2 it shrinks to the L2 latency.  The softmax
 // warps issue the prefetches (plain prefetch.global.L2, not the TMA unit, which serialises its
-// copies): this CTA's 64 rows of the tile are one contiguous 72 KB run (a 64-token page, or 64
-// consecutive rows of a contiguous cache), 576 lines over 256 threads, once per tile.
+// copies): this CTA's 64 rows of the tile are one contiguous 72 KB run, 576 lines over 256
+// threads, once per tile.  Contiguous caches only: with pages at permuted addresses the
+// prefetches measured slower (b32 x 4096 paged 65.6 -> 66.6 us, 128 mixed lengths paged 219 ->
+// 223 us), against 61.8 -> 58.6 and 200 -> 195 us for the same batches contiguous.
 constexpr int kTcPfDist = 2;
 __device__ __forceinline__ void tc_prefetch_tile(const DecodeTcArgs& a, int b, int tok0, int t_end) {
-  if (tok0 >= t_end) return;
+  if (tok0 >= t_end || a.v.page_size != 0) return;
   const int64_t r = cache_row(a.v, b, tok0);
   if (r < 0) return;
-  // rows of one page (paged) and of the buffer only
   int n = min(64, t_end - tok0);
-  if (a.v.page_size != 0) n = min(n, kPage - tok0 % kPage);
-  if (a.v.num_rows - r < n) n = static_cast<int>(a.v.num_rows - r);
+  if (a.v.num_rows - r < n) n = static_cast<int>(a.v.num_rows - r);   // rows of the buffer only
   const uint8_t* base = a.cache + r * (kDRow * 2);
   for (int L = threadIdx.x; L < n * (kDRow * 2 / 128); L += 32 * kTcSoftmaxWarps)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(base + 128 * L));
