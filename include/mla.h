@@ -190,6 +190,29 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
                            size_t workspace_bytes, mla_bf16* out_lat, float* lse, void* stream);
 
 /*
+ * (7) Chunked prefill attention, absorbed form — [DR] §4.2 (prompt throughput is measured beside
+ *     generation) with the attention of (3): a chunk of new tokens of a sequence, appended to the
+ *     cache first (mla_cache_append with their positions), each attends causally to the cached
+ *     tokens up to and including itself.
+ * Query row i (one new token) reads sequence q_seq[i] of the cache and attends to its first
+ * q_len[i] tokens (q_len[i] = the token's position + 1 gives the causal mask; rows of later
+ * tokens of the same chunk are not read).  Otherwise identical to mla_decode_attn with the query
+ * rows in place of the batch: the same work ranges (planned from q_len), the same partials and
+ * combine, the same outputs per row:
+ *     out_lat[i, h, :] = sum_{t < q_len[i]} softmax_t(scale * q_full[i, h] . row(q_seq[i], t)) c_t
+ *   q_full [n_queries, 128, 576] bf16   q_seq, q_len [n_queries] int32 (device)
+ *   workspace >= mla_decode_workspace_size(n_queries, capacity, num_splits) bytes
+ *   out_lat [n_queries, 128, 512] bf16 (written)   lse [n_queries, 128] fp32 (written) or NULL
+ * Any number of rows may read the same sequence, and rows of several sequences may be mixed.
+ * q_seq[i] outside [0, desc.num_seqs) sets MLA_DEVERR_BLOCK_RANGE and the row reads zeros;
+ * q_len[i] > capacity sets MLA_DEVERR_SEQLEN_RANGE and is clamped.  n_queries <= 16384.
+ */
+mla_status mla_prefill_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
+                            const int32_t* q_seq, const int32_t* q_len, mla_cache_desc desc, int32_t n_queries,
+                            float softmax_scale, int32_t num_splits, void* workspace, size_t workspace_bytes,
+                            mla_bf16* out_lat, float* lse, void* stream);
+
+/*
  * Decode attention that allocates nothing and takes no workspace (the pages have no counterpart:
  * this is a deployment convenience of this library).
  * For callers that cannot obtain device memory at decode time, for example a plugin inside a

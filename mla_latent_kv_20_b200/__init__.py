@@ -59,6 +59,7 @@ def _load():
         "mla_decode_num_splits": (I32, [I32, I32, I32]),
         "mla_decode_workspace_size": (SZ, [I32, I32, I32]),
         "mla_decode_attn": (ctypes.c_int, [P, P, P, P, CacheDesc, I32, F32, I32, P, SZ, P, P, P]),
+        "mla_prefill_attn": (ctypes.c_int, [P, P, P, P, P, CacheDesc, I32, F32, I32, P, SZ, P, P, P]),
         "mla_unabsorb_v": (ctypes.c_int, [P, P, P, I32, P]),
         "mla_decode_attn_noalloc": (ctypes.c_int, [P, P, P, P, CacheDesc, I32, F32, I32, P, P, P]),
         "mla_get_device_error": (ctypes.c_int, [ctypes.POINTER(I32)]),
@@ -154,6 +155,18 @@ def decode_attn(q_full, cache, seq_lens, desc: CacheDesc, workspace, out_lat, *,
     _check(lib.mla_decode_attn(_ptr(q_full), _ptr(cache), _ptr(block_table), _ptr(seq_lens), desc, b,
                                softmax_scale, num_splits, _ptr(workspace), wb, _ptr(out_lat), _ptr(lse),
                                _stream(stream)), "mla_decode_attn")
+
+
+def prefill_attn(q_full, cache, q_seq, q_len, desc: CacheDesc, workspace, out_lat, *, lse=None,
+                 block_table=None, softmax_scale: float = 1.0 / 192 ** 0.5, num_splits: int = 0, stream=None,
+                 n_queries: int | None = None, workspace_bytes: int | None = None):
+    """mla_prefill_attn: query row i (a new token of sequence q_seq[i]) attends to the first
+    q_len[i] cached tokens of that sequence."""
+    n = q_full.shape[0] if n_queries is None else n_queries
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(lib.mla_prefill_attn(_ptr(q_full), _ptr(cache), _ptr(block_table), _ptr(q_seq), _ptr(q_len), desc, n,
+                                softmax_scale, num_splits, _ptr(workspace), wb, _ptr(out_lat), _ptr(lse),
+                                _stream(stream)), "mla_prefill_attn")
 
 
 NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024

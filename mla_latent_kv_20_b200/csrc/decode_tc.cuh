@@ -95,6 +95,7 @@ struct DecodeTcArgs {
   __nv_bfloat16* out_lat;
   float* lse;
   const uint8_t* cache;   // the cache buffer (L2 prefetch addresses)
+  const int32_t* seq_map; // query row -> cache sequence (chunked prefill), or null: row b reads sequence b
 };
 
 // This CTA pair's work range, computed once per CTA at entry (the cursor's starting state).
@@ -132,6 +133,18 @@ __device__ __forceinline__ int tma_row(const CacheView& v, int b, int t) {
 }
 
 __device__ __forceinline__ uint32_t lbar(const void* p) { return mapa_shared(smem_u32(p), 0); }
+
+// The cache sequence that query row b reads: b itself, or seq_map[b] in a chunked prefill (where
+// several query rows, one per new token, read one sequence).  A map entry outside the cache gives
+// -1 (rows read as zeros); the producer also reports it through the device error word.
+template <bool kMapped>
+__device__ __forceinline__ int tc_cache_seq(const DecodeTcArgs& a, int b, bool report) {
+  if (!kMapped) return b;
+  const int s = a.seq_map[b];
+  if (s >= 0 && s < a.v.num_seqs) return s;
+  if (report) set_dev_error(0x2);
+  return -1;
+}
 
 // 3-D TMA load (x: element in a 64-wide dim-slab, y: cache row, z: dim-slab) into this CTA's
 // shared memory; completion counted on a barrier that may live in the peer CTA.
@@ -207,6 +220,7 @@ __device__ __noinline__ bool tc_load_ragged_v(uint8_t* box, const CUtensorMap* t
   return true;
 }
 
+template <bool kMapped>
 __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, const CUtensorMap* tm_v,
                             const CUtensorMap* tm_q, const DecodeTcArgs& a, const TcPlan& plan, uint8_t* smem,
                             TcBars* bars, uint32_t rank, int pair, volatile int* abort_flag) {
@@ -242,10 +256,15 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
       else
         mbar_arrive_relaxed(lbar(&bars->q_full));
     }
+    // TMA row of token t of query row b's sequence (a fully out-of-bounds box for a bad map entry)
+    auto row_of = [&](int t) -> int {
+      const int cb = tc_cache_seq<kMapped>(a, b, true);
+      return (kMapped && cb < 0) ? -kTcTile : tma_row(a.v, cb, t);
+    };
     auto issue_k = [&](int i) -> bool {
       const int gi = g + i;
       const int my0 = t_begin + i * kTcTile + 64 * static_cast<int>(rank);
-      const int y = my0 < t_end ? tma_row(a.v, b, my0) : -kTcTile;
+      const int y = my0 < t_end ? row_of(my0) : -kTcTile;
 #pragma unroll 1
       for (int part = 0; part < 2; ++part) {
         if (gi >= 1 && !wait0(&bars->k_empty[part], static_cast<uint32_t>(gi - 1) & 1u, 0x10 + part)) return false;
@@ -274,14 +293,14 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
         const int vcount = min(max(t_end - tok0, 0), 64);
         if (vcount == 64) {
           if (l0) {
-            tma_load_4d_pair(box, tm_v, lbar(&bars->v_full[s]), 0, tma_row(a.v, b, tok0), 2 * static_cast<int>(rank), 0);
+            tma_load_4d_pair(box, tm_v, lbar(&bars->v_full[s]), 0, row_of(tok0), 2 * static_cast<int>(rank), 0);
             if (leader)
               mbar_arrive_expect_tx_relaxed(lbar(&bars->v_full[s]), 2u * kTcVBox);
             else
               mbar_arrive_relaxed(lbar(&bars->v_full[s]));
           }
         } else {
-          if (!tc_load_ragged_v(box, tm_v, &bars->fix, fix_phase, vcount > 0 ? tma_row(a.v, b, tok0) : 0,
+          if (!tc_load_ragged_v(box, tm_v, &bars->fix, fix_phase, vcount > 0 ? row_of(tok0) : 0,
                                 static_cast<int>(rank), vcount, lbar(&bars->v_full[s]), abort_flag))
             return false;
           if (vcount > 0) fix_phase ^= 1u;
@@ -437,9 +456,12 @@ __device__ __forceinline__ void store_rows_128b(uint8_t* stage, const uint32_t (
 // prefetches measured slower (b32 x 4096 paged 65.6 -> 66.6 us, 128 mixed lengths paged 219 ->
 // 223 us), against 61.8 -> 58.6 and 200 -> 195 us for the same batches contiguous.
 constexpr int kTcPfDist = 2;
+template <bool kMapped>
 __device__ __forceinline__ void tc_prefetch_tile(const DecodeTcArgs& a, int b, int tok0, int t_end) {
   if (tok0 >= t_end || a.v.page_size != 0) return;
-  const int64_t r = cache_row(a.v, b, tok0);
+  const int cb = tc_cache_seq<kMapped>(a, b, false);   // b is the query row
+  if (kMapped && cb < 0) return;
+  const int64_t r = cache_row(a.v, cb, tok0);
   if (r < 0) return;
   int n = min(64, t_end - tok0);
   if (a.v.num_rows - r < n) n = static_cast<int>(a.v.num_rows - r);   // rows of the buffer only
@@ -535,6 +557,7 @@ __device__ __noinline__ void tc_rescale_o(uint32_t addr, float alpha) {
   tmem_st_wait();
 }
 
+template <bool kMapped>
 __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, uint8_t* smem, TcBars* bars,
                            float* red, uint32_t tmem, uint32_t rank, volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5;
@@ -555,7 +578,7 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
   float m_used = -INFINITY;
   float l_run = 0.f;
   for (int d = 1; d < kTcPfDist && d < n_tiles; ++d)
-    tc_prefetch_tile(a, sg.b, t_begin + d * kTcTile + 64 * static_cast<int>(rank), t_end);
+    tc_prefetch_tile<kMapped>(a, sg.b, t_begin + d * kTcTile + 64 * static_cast<int>(rank), t_end);
   for (int i = 0; i < n_tiles && ok; ++i, ++g) {
     const int j = g & 1;
     if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[j], static_cast<uint32_t>(g >> 1) & 1u, 0x30))) {
@@ -655,7 +678,7 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
       mbar_arrive_relaxed(lbar(&bars->p_full));
     }
     if (i + kTcPfDist < n_tiles)
-      tc_prefetch_tile(a, sg.b, t_begin + (i + kTcPfDist) * kTcTile + 64 * static_cast<int>(rank), t_end);
+      tc_prefetch_tile<kMapped>(a, sg.b, t_begin + (i + kTcPfDist) * kTcTile + 64 * static_cast<int>(rank), t_end);
   }
   // ---- epilogue of the segment (every warp passes the same barriers, also after a failure)
   if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_final, static_cast<uint32_t>(k) & 1u, 0x33))) ok = false;
@@ -818,7 +841,9 @@ __device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacit
 }
 
 // ------------------------------------------------------------------------------ kernel
-// grid = 2 * P CTAs, clusters of 2 along x: blockIdx.x = 2 * pair + rank.
+// grid = 2 * P CTAs, clusters of 2 along x: blockIdx.x = 2 * pair + rank.  kMapped: query rows
+// read the cache sequences of a.seq_map (chunked prefill); the decode instance carries none of it.
+template <bool kMapped>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_ka, const __grid_constant__ CUtensorMap tm_kb,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
@@ -900,9 +925,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   if (!busy) {
     // an idle range: only the teardown below
   } else if (warp < kTcSoftmaxWarps) {
-    tc_softmax(a, pl, pair, smem, bars, red, tmem, rank, abort_flag);
+    tc_softmax<kMapped>(a, pl, pair, smem, bars, red, tmem, rank, abort_flag);
   } else if (warp == kTcProducerWarp) {
-    if (!tc_producer(&tm_ka, &tm_kb, &tm_v, &tm_q, a, pl, smem, bars, rank, pair, abort_flag) &&
+    if (!tc_producer<kMapped>(&tm_ka, &tm_kb, &tm_v, &tm_q, a, pl, smem, bars, rank, pair, abort_flag) &&
         (threadIdx.x & 31) == 0)
       *abort_flag = 1;
   } else if (rank == 0 && (threadIdx.x & 31) == 0) {

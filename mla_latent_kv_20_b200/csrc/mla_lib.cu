@@ -180,13 +180,13 @@ int decode_cluster_slots() {
   static int cached[64] = {0};
   if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
   int n = 0;
-  if (cudaFuncSetAttribute(mla::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(mla::decode_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            mla::kTcSmemBytes) == cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(mla::kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = mla::kTcSmemBytes;
-    if (cudaOccupancyMaxActiveClusters(&n, mla::decode_tc_kernel, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, mla::decode_tc_kernel<false>, &cfg) != cudaSuccess) n = 0;
   }
   cudaGetLastError();
   if (n <= 0) n = device_sm_count() / 2;
@@ -510,31 +510,38 @@ size_t mla_decode_workspace_size(int32_t batch, int32_t max_seq_len, int32_t num
   return mla::ws_bytes(batch, mla_decode_num_splits(batch, max_seq_len, num_splits));
 }
 
-mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
-                           const int32_t* seq_lens, mla_cache_desc desc, int32_t batch, float softmax_scale,
-                           int32_t num_splits, void* workspace, size_t workspace_bytes, mla_bf16* out_lat,
-                           float* lse, void* stream) {
-  if (batch < 0 || num_splits < 0) return MLA_ERR_INVALID_ARG;
-  if (batch > mla::kMaxDecodeBatch) return MLA_ERR_UNSUPPORTED;
+}  // extern "C"
+
+namespace {
+
+// The decode kernel and its combine over `rows` query rows: row b attends to the first
+// lens[b] cached tokens of sequence b, or of sequence seq_map[b] when a map is given (chunked
+// prefill).  Host checks shared by both entry points.
+mla_status launch_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
+                       const int32_t* lens, const int32_t* seq_map, mla_cache_desc desc, int32_t rows,
+                       float softmax_scale, int32_t num_splits, void* workspace, size_t workspace_bytes,
+                       mla_bf16* out_lat, float* lse, void* stream) {
+  if (rows < 0 || num_splits < 0) return MLA_ERR_INVALID_ARG;
+  if (rows > mla::kMaxDecodeBatch) return MLA_ERR_UNSUPPORTED;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
   CacheView v;
   const mla_status st = check_cache(desc, cache, block_table, &v);
   if (st != MLA_OK) return st;
-  if (batch == 0) return MLA_OK;
-  if (batch > desc.num_seqs) return MLA_ERR_INVALID_ARG;
-  if (q_full == nullptr || seq_lens == nullptr || out_lat == nullptr) return MLA_ERR_INVALID_ARG;
+  if (rows == 0) return MLA_OK;
+  if (seq_map == nullptr && rows > desc.num_seqs) return MLA_ERR_INVALID_ARG;
+  if (q_full == nullptr || lens == nullptr || out_lat == nullptr) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_full) || !aligned16(out_lat) || (lse != nullptr && !aligned16(lse))) return MLA_ERR_INVALID_ARG;
   const int capacity = cache_capacity(desc);
-  const int P = mla_decode_num_splits(batch, capacity, num_splits);
-  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < mla::ws_bytes(batch, P))
+  const int P = mla_decode_num_splits(rows, capacity, num_splits);
+  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < mla::ws_bytes(rows, P))
     return MLA_ERR_WORKSPACE;
-  if (desc.num_rows >= (int64_t(1) << 31) || static_cast<int64_t>(batch) * mla::kHeads >= (int64_t(1) << 31))
+  if (desc.num_rows >= (int64_t(1) << 31) || static_cast<int64_t>(rows) * mla::kHeads >= (int64_t(1) << 31))
     return MLA_ERR_UNSUPPORTED;
   cudaStream_t s = as_stream(stream);
   mla::DecodeTcArgs a;
   a.v = v;
-  a.seq_lens = seq_lens;
-  a.batch = batch;
+  a.seq_lens = lens;
+  a.batch = rows;
   a.capacity = capacity;
   a.P = P;
   a.scale_log2 = softmax_scale * mla::kLog2e;
@@ -542,19 +549,41 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
   a.out_lat = reinterpret_cast<__nv_bfloat16*>(out_lat);
   a.lse = lse;
   a.cache = reinterpret_cast<const uint8_t*>(cache);
+  a.seq_map = seq_map;
   CUtensorMap tka, tkb, tv, tq;
   if (!make_map_slabs(&tka, cache, desc.num_rows, mla::kTcKSlabsA) ||
       !make_map_slabs(&tkb, cache, desc.num_rows, mla::kTcKSlabsB) || !make_map_vbox(&tv, cache, desc.num_rows) ||
-      !make_map_slabs(&tq, q_full, static_cast<uint64_t>(batch) * mla::kHeads, 9))
+      !make_map_slabs(&tq, q_full, static_cast<uint64_t>(rows) * mla::kHeads, 9))
     return MLA_ERR_CUDA;
-  if (cudaFuncSetAttribute(mla::decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kTcSmemBytes) !=
-      cudaSuccess)
+  auto kernel = seq_map != nullptr ? mla::decode_tc_kernel<true> : mla::decode_tc_kernel<false>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kTcSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
-  mla_status ls = launch_chained(mla::decode_tc_kernel, dim3(2 * P), dim3(mla::kTcThreads),
-                                 static_cast<size_t>(mla::kTcSmemBytes), s, tka, tkb, tv, tq, a);
+  mla_status ls = launch_chained(kernel, dim3(2 * P), dim3(mla::kTcThreads), static_cast<size_t>(mla::kTcSmemBytes), s,
+                                 tka, tkb, tv, tq, a);
   if (ls != MLA_OK) return ls;
-  return launch_chained(mla::combine_kernel, dim3(batch, mla::kHeads / 4), dim3(128), 0, s, a.ws, P,
+  return launch_chained(mla::combine_kernel, dim3(rows, mla::kHeads / 4), dim3(128), 0, s, a.ws, P,
                         reinterpret_cast<__nv_bfloat16*>(out_lat), lse);
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
+                           const int32_t* seq_lens, mla_cache_desc desc, int32_t batch, float softmax_scale,
+                           int32_t num_splits, void* workspace, size_t workspace_bytes, mla_bf16* out_lat,
+                           float* lse, void* stream) {
+  return launch_attn(q_full, cache, block_table, seq_lens, nullptr, desc, batch, softmax_scale, num_splits, workspace,
+                     workspace_bytes, out_lat, lse, stream);
+}
+
+mla_status mla_prefill_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
+                            const int32_t* q_seq, const int32_t* q_len, mla_cache_desc desc, int32_t n_queries,
+                            float softmax_scale, int32_t num_splits, void* workspace, size_t workspace_bytes,
+                            mla_bf16* out_lat, float* lse, void* stream) {
+  if (n_queries > 0 && q_seq == nullptr) return MLA_ERR_INVALID_ARG;
+  return launch_attn(q_full, cache, block_table, q_len, q_seq, desc, n_queries, softmax_scale, num_splits, workspace,
+                     workspace_bytes, out_lat, lse, stream);
 }
 
 }  // extern "C"

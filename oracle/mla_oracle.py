@@ -221,6 +221,56 @@ def merge_partials(parts):
 
 
 # ----------------------------------------------------------------------------------------
+# Chunked prefill ([DR] §4.2 measures prompt throughput beside generation; the attention is
+# that of §2.3/§2.4).  A chunk of new tokens is appended first; each new token then attends
+# causally: to the tokens before it and to itself.
+# ----------------------------------------------------------------------------------------
+def prefill_rows(qf, seq_rows, q_seq, q_len, scale, d_latent):
+    """Absorbed form, one query row at a time: row i attends to the first q_len[i] cached rows of
+    sequence q_seq[i] (q_len = position + 1 is the causal mask).
+
+    qf: [n, H, d_c + d_R]; seq_rows: list of [L_s, d_c + d_R], one per cache sequence.
+    Returns out_lat [n, H, d_c] and lse [n, H]; a row with q_len 0 gives zeros and -inf.
+    """
+    qf = np.asarray(qf, np.float64)
+    n, H = qf.shape[0], qf.shape[1]
+    out_lat = np.zeros((n, H, d_latent))
+    lse = np.full((n, H), -np.inf)
+    for i in range(n):
+        L = int(q_len[i])
+        if L == 0:
+            continue
+        r = attend_rows(qf[i], np.asarray(seq_rows[int(q_seq[i])], np.float64)[:L], scale, d_latent)
+        out_lat[i], lse[i] = r["out_lat"], r["lse"]
+    return dict(out_lat=out_lat, lse=lse)
+
+
+def prefill_explicit_masked(q_nope, q_pe, c, kr_rot, w_uk, w_uv, scale, q_pos):
+    """Textbook causal attention of a chunk of queries of one sequence in the explicit form:
+    per-head keys and values decompressed from the latents ([DR] §2.2), one score tensor
+    s[h, i, t] = scale * [q_nope_ih ; q_pe_ih] . [k^C_th ; k^R_t] over all L cached tokens, the
+    entries of tokens after the query's position (t > q_pos[i]) set to -inf, a softmax along t,
+    then out = P v^C and out_lat = P c.
+
+    q_nope: [n, H, d_h]; q_pe: [n, H, d_R] (rotated); c: [L, d_c]; kr_rot: [L, d_R]; q_pos: [n].
+    """
+    q_nope = np.asarray(q_nope, np.float64)
+    q_pe = np.asarray(q_pe, np.float64)
+    c = np.asarray(c, np.float64)
+    kC, vC = decompress(c, w_uk, w_uv)                                   # [L, H, d_h]
+    s = np.einsum("ihj,thj->hit", q_nope, kC, optimize=True)            # content channel
+    s = s + np.einsum("ihr,tr->hit", q_pe, np.asarray(kr_rot, np.float64), optimize=True)
+    s = scale * s
+    L = c.shape[0]
+    future = np.arange(L)[None, :] > np.asarray(q_pos)[:, None]          # [n, L]
+    s = np.where(future[None, :, :], -np.inf, s)
+    p, lse = softmax_stats(s)                                            # along t
+    out = np.einsum("hit,thj->ihj", p, vC, optimize=True)
+    out_lat = np.einsum("hit,tk->ihk", p, c, optimize=True)
+    return dict(out=out, out_lat=out_lat, lse=lse.T)
+
+
+# ----------------------------------------------------------------------------------------
 # One whole decode step for a batch ([DR] §3.1 flow: append, absorb, attend, un-absorb)
 # ----------------------------------------------------------------------------------------
 def decode_step(q_nope, q_pe, cs, krs_raw, w_uk, w_uv, scale, base=ROPE_BASE,

@@ -26,7 +26,7 @@ def declared_functions():
 
 def test_header_declares_the_path():
     names = declared_functions()
-    for n in ("mla_cache_append", "mla_absorb_q", "mla_decode_attn", "mla_unabsorb_v",
+    for n in ("mla_cache_append", "mla_absorb_q", "mla_decode_attn", "mla_prefill_attn", "mla_unabsorb_v",
               "mla_decode_workspace_size", "mla_get_device_error", "mla_status_string"):
         assert n in names
 
@@ -102,6 +102,21 @@ def test_decode_validation_and_workspace(mla):
     big = mla.contiguous_desc(16385, 64)
     assert lib.mla_decode_attn(*args(FAKE, 1 << 40, batch=16385, desc=big)) == 2   # batch beyond the plan's limit
     assert lib.mla_get_device_error(None) == 1
+
+
+def test_prefill_validation(mla):
+    """Host checks of mla_prefill_attn (no kernel is launched on any of these paths): the query
+    rows may outnumber the cache's sequences (several rows read one sequence), the map is required."""
+    lib = mla.lib
+    d = mla.contiguous_desc(2, 4096)
+    need = lib.mla_decode_workspace_size(40, 4096, 16)
+    args = lambda ws, nbytes, q_seq=FAKE, n=40, scale=0.072: (  # noqa: E731
+        FAKE, FAKE, None, q_seq, FAKE, d, n, scale, 16, ws, nbytes, FAKE, None, None)
+    assert lib.mla_prefill_attn(*args(FAKE, need - 16)) == 3          # workspace too small
+    assert lib.mla_prefill_attn(*args(FAKE, need, q_seq=None)) == 1  # the row -> sequence map is required
+    assert lib.mla_prefill_attn(*args(FAKE, need, scale=-1.0)) == 1
+    assert lib.mla_prefill_attn(*args(FAKE, need, n=0)) == 0         # no rows: a no-op
+    assert lib.mla_prefill_attn(*args(FAKE, need, n=16385)) == 2     # beyond the plan's limit
 
 
 def test_wait_selftest_validates_arguments(mla):

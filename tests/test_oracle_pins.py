@@ -422,3 +422,108 @@ def test_pins_catch_planted_output_proj_mistakes():
 
     for bad in (dim_major_concat, heads_reversed):
         assert _fails(check_output_proj, bad), bad.__name__
+
+
+# ------------------------------------------------------------------ chunked prefill
+def bf_prefill_row(qf, rows, L, scale, d_latent):
+    """Scalar loops: one absorbed query row [H][d_c + d_R] over the first L rows."""
+    H = len(qf)
+    lat, lse = [], []
+    for h in range(H):
+        s = [scale * sum(float(qf[h][k]) * float(rows[t][k]) for k in range(len(qf[h]))) for t in range(L)]
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        z = sum(e)
+        lat.append([sum(e[t] / z * float(rows[t][k]) for t in range(L)) for k in range(d_latent)])
+        lse.append(m + math.log(z))
+    return lat, lse
+
+
+def prefill_case(seed, L=9, n=4, H=2, dh=3, dc=4, dr=2):
+    """One sequence of L cached tokens whose last n are a new chunk (positions L-n .. L-1)."""
+    t = tiny_case(seed, L, H, dh, dc, dr)
+    rng = np.random.default_rng(seed + 100)
+    t["q_nope"] = rng.standard_normal((n, H, dh))
+    t["q_pe"] = rng.standard_normal((n, H, dr))
+    t["q_pos"] = np.arange(L - n, L)
+    return t
+
+
+def check_prefill_bruteforce(prefill_rows):
+    """Scalar-loop pin: every row attends to exactly the tokens at or before its position, in
+    several sequences at once, and an empty row gives zeros and -inf."""
+    t = prefill_case(31)
+    rows = np.concatenate([t["c"], t["kr_rot"]], axis=1)
+    other = np.random.default_rng(32).standard_normal((5, rows.shape[1]))
+    qf = np.concatenate([oracle.absorb_q(t["q_nope"], t["w_uk"]), t["q_pe"]], axis=-1)
+    qf = np.concatenate([qf, qf[:2]], axis=0)                       # two more rows, on sequence 1
+    q_seq = np.array([0, 0, 0, 0, 1, 1])
+    q_len = np.concatenate([t["q_pos"] + 1, [3, 0]])
+    r = prefill_rows(qf, [rows, other], q_seq, q_len, 0.41, 4)
+    for i in range(5):
+        lat, lse = bf_prefill_row(qf[i], [rows, other][q_seq[i]], int(q_len[i]), 0.41, 4)
+        assert np.allclose(r["out_lat"][i], lat, rtol=1e-12, atol=1e-12), i
+        assert np.allclose(r["lse"][i], lse, rtol=1e-12, atol=1e-12), i
+    assert np.array_equal(r["out_lat"][5], np.zeros_like(r["out_lat"][5])) and np.all(r["lse"][5] == -np.inf)
+
+
+def check_prefill_causal(prefill_rows):
+    """Rows of tokens after a query's position never reach it; its own row does."""
+    t = prefill_case(33)
+    rows = np.concatenate([t["c"], t["kr_rot"]], axis=1)
+    qf = np.concatenate([oracle.absorb_q(t["q_nope"], t["w_uk"]), t["q_pe"]], axis=-1)
+    q_seq, q_len = np.zeros(4, int), t["q_pos"] + 1
+    base = prefill_rows(qf, [rows], q_seq, q_len, 0.41, 4)
+    for i, p in enumerate(t["q_pos"]):
+        later = rows.copy()
+        later[p + 1:] = 1e3                                          # every token after position p
+        r = prefill_rows(qf, [later], q_seq, q_len, 0.41, 4)
+        assert np.array_equal(r["out_lat"][i], base["out_lat"][i]), i
+        own = rows.copy()
+        own[p] += 1.0                                                # the query's own token
+        r = prefill_rows(qf, [own], q_seq, q_len, 0.41, 4)
+        assert not np.allclose(r["out_lat"][i], base["out_lat"][i]), i
+
+
+def check_prefill_against_masked_explicit(prefill_rows, prefill_explicit_masked):
+    """The absorbed row-at-a-time form against the textbook masked-matrix form in the explicit
+    (decompressed) basis, at the real head and latent widths."""
+    rng = np.random.default_rng(35)
+    H, dh, dc, dr, L, n = 4, mi.D_HEAD, mi.D_LATENT, mi.D_ROPE, 40, 7
+    c = rng.standard_normal((L, dc))
+    kr = rng.standard_normal((L, dr))
+    w_uk = rng.standard_normal((H, dh, dc)) / math.sqrt(dc)
+    w_uv = rng.standard_normal((H, dc, dh)) / math.sqrt(dc)
+    qn, qp = rng.standard_normal((n, H, dh)), rng.standard_normal((n, H, dr))
+    q_pos = np.array([33, 34, 35, 36, 37, 38, 39])
+    ex = prefill_explicit_masked(qn, qp, c, kr, w_uk, w_uv, SCALE, q_pos)
+    qf = np.concatenate([oracle.absorb_q(qn, w_uk), qp], axis=-1)
+    r = prefill_rows(qf, [np.concatenate([c, kr], axis=1)], np.zeros(n, int), q_pos + 1, SCALE, dc)
+    assert np.allclose(r["out_lat"], ex["out_lat"], rtol=1e-10, atol=1e-12)
+    assert np.allclose(r["lse"], ex["lse"], rtol=1e-10, atol=1e-12)
+    assert np.allclose(oracle.unabsorb_v(r["out_lat"], w_uv), ex["out"], rtol=1e-10, atol=1e-12)
+
+
+def test_prefill_pins():
+    check_prefill_bruteforce(oracle.prefill_rows)
+    check_prefill_causal(oracle.prefill_rows)
+    check_prefill_against_masked_explicit(oracle.prefill_rows, oracle.prefill_explicit_masked)
+
+
+def test_pins_catch_planted_prefill_mistakes():
+    def mask_off_by_one(qf, seq_rows, q_seq, q_len, scale, d_latent):          # the query misses itself
+        return oracle.prefill_rows(qf, seq_rows, q_seq, np.maximum(np.asarray(q_len) - 1, 0), scale, d_latent)
+
+    def sees_whole_sequence(qf, seq_rows, q_seq, q_len, scale, d_latent):      # no causal mask
+        return oracle.prefill_rows(qf, seq_rows, q_seq, [len(seq_rows[s]) for s in q_seq], scale, d_latent)
+
+    def first_sequence_only(qf, seq_rows, q_seq, q_len, scale, d_latent):      # map ignored
+        return oracle.prefill_rows(qf, seq_rows, np.zeros_like(np.asarray(q_seq)), q_len, scale, d_latent)
+
+    for bad in (mask_off_by_one, sees_whole_sequence, first_sequence_only):
+        assert _fails(check_prefill_bruteforce, bad), bad.__name__
+
+    def masked_inclusive(qn, qp, c, kr, w_uk, w_uv, scale, q_pos):             # masks the query's own token
+        return oracle.prefill_explicit_masked(qn, qp, c, kr, w_uk, w_uv, scale, np.asarray(q_pos) - 1)
+
+    assert _fails(check_prefill_against_masked_explicit, oracle.prefill_rows, masked_inclusive)
