@@ -434,6 +434,60 @@ def measure_output_proj(st, steps, warmup):
             "frac": gbs / hbm, "l2": "weight (168 MB) larger than L2 (median of %d back-to-back calls)" % n}
 
 
+PREFILL_SEQS, PREFILL_PREFIX, PREFILL_CHUNK = 4, 3072, 1024
+
+
+def measure_prefill(steps, warmup):
+    """The chunked-prefill row (mla_prefill_attn, absorbed form): 4 sequences each append a chunk of
+    1024 new tokens to a 3072-token prefix, and every new token attends causally to the 3073 ..
+    4096 cached tokens up to itself (4096 query rows).  Synthetic N(0,1) cache rows and queries
+    on the device; the 18.9 MB cache stays in L2 across the rows that share it, so the call is
+    bound by the tensor cores: 278,528 flop per (query, cached token) pair.  Timed per call with
+    CUDA events (median)."""
+    import torch
+    import mla_latent_kv_20_b200 as m
+    from mla_latent_kv_20_b200 import harness as hz
+    L = PREFILL_PREFIX + PREFILL_CHUNK
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(9003)
+    cache = hz.Cache([L] * PREFILL_SEQS, False, fill_value=None)
+    cache.data.copy_(torch.randn(cache.data.shape, device="cuda", generator=gen).to(torch.bfloat16))
+    n = PREFILL_SEQS * PREFILL_CHUNK
+    q_seq = torch.arange(PREFILL_SEQS, dtype=torch.int32, device="cuda").repeat_interleave(PREFILL_CHUNK)
+    q_len = (torch.arange(PREFILL_CHUNK, dtype=torch.int32, device="cuda") + PREFILL_PREFIX + 1).repeat(PREFILL_SEQS)
+    qf = torch.randn((n, mi.N_HEADS, mi.D_ROW), device="cuda", generator=gen).to(torch.bfloat16)
+    out_lat = torch.empty((n, mi.N_HEADS, mi.D_LATENT), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((n, mi.N_HEADS), dtype=torch.float32, device="cuda")
+    ws = torch.empty((m.decode_workspace_size(n, L, 0),), dtype=torch.uint8, device="cuda")
+
+    def call():
+        m.prefill_attn(qf, cache.data, q_seq, q_len, cache.desc, ws, out_lat, lse=lse)
+
+    for _ in range(max(warmup, 1)):
+        call()
+    torch.cuda.synchronize()
+    k = min(max(steps, 1), 10)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+    for e0, e1 in ev:
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+    ms = sorted(e0.elapsed_time(e1) for e0, e1 in ev)[k // 2]
+    pairs = int(q_len.sum().item())
+    flops = pairs * 2 * mi.N_HEADS * (mi.D_ROW + mi.D_LATENT)
+    _, tc_burst, tc_sustained, _ = load_peaks()
+    peak = tc_sustained or tc_burst
+    tf = flops / (ms * 1e-3) / 1e12
+    del cache, qf, out_lat, lse, ws
+    return {"kernel": "decode_tc_kernel<true> + combine_kernel", "sequences": PREFILL_SEQS,
+            "new_tokens": n, "prefix": PREFILL_PREFIX, "ms_per_call": ms, "tokens_per_s": n / (ms * 1e-3),
+            "bound": "tensor", "algorithmic_flops_per_launch": flops, "achieved": tf, "peak": peak,
+            "peak_kind": "sustained bf16 (a call of several ms)", "unit": "TFLOP/s", "frac": tf / peak,
+            "l2": "cache (18.9 MB) L2-resident, shared by the rows of a chunk (median of %d calls)" % k}
+
+
 def run_step(st, i):
     """One decode step over every layer of the workload, through plain API calls."""
     for li in range(len(st["layers"])):
@@ -581,7 +635,8 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
     next_rows = {"project_append": measure_project_append(st, args.steps, args.warmup),
-                 "output_proj": measure_output_proj(st, args.steps, args.warmup)}
+                 "output_proj": measure_output_proj(st, args.steps, args.warmup),
+                 "prefill": measure_prefill(args.steps, args.warmup)}
     ms, e2e_ms, dec_ms = reduce_max_over_ranks([ms, e2e_ms, dec_ms], world, device=dev)
     if rank != 0:
         return
