@@ -696,7 +696,7 @@ def run_ours(args, rank, world, local_rank):
         pos = flat[offs[j]:offs[j] + st["pos"].numel() * 4].view(torch.int32).view(st["pos"].shape)
         bufs.append((flat, views, pos, torch.empty_like(st["out"])))
     out_host = [torch.empty(st["out"].shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    h2d = sum(a.size for a in srcs)
+    h2d = total   # the packed buffer, padding included: what each step copies
     d2h = out_host[0].numel() * out_host[0].element_size()
     cs, ks_ = copy_stream.cuda_stream, compute_stream.cuda_stream
     in_ready, step_done, out_read = rt.events(2), rt.events(2), rt.events(2)
