@@ -282,7 +282,7 @@ def setup_replica(name, device):
 # counters were taken, and the traffic is reported as null.
 TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh", "csrc/mla_lib.cu")
 MEASURED_TRAFFIC = {   # workload -> {"bytes": int, "sha256": str, "profile": str}
-    "b32_l4096": {"bytes": 155796480 + 3692032 + 16858368, "sha256": "c207dcc53529bbe15f8b1ae24d8d9d575d0a93708359ee0a790fee19e32dac5c",
+    "b32_l4096": {"bytes": 155799552 + 3387904 + 16860928, "sha256": "9fa4020d9de8ec2be4d31ff6e53526e7fd0c95e9678f26aadeaecb6df04e7896",
                   "profile": "profiles/decode_tc_b32_l4096.md (decode + combine, ncu cache flush per kernel)"},
 }
 
