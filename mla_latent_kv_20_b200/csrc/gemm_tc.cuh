@@ -52,10 +52,11 @@ struct AppendJob {
 // Query side only (qpe != nullptr, KTOT = d_h): the epilogue warps also fill the RoPE part of the
 // query rows, out[n, h, 512:576] = q_pe[n, h, :] rotated at q_pos[n] (or copied when q_pos is
 // null), and write the new tokens' cache rows of `app` (if any), while the MMAs run: CTA c (linear
-// index) takes rows n = c, c + #CTAs, ... (for all 128 heads, so each row's 32 angles are formed
-// once).
+// index) takes work units c, c + #CTAs, ... (a unit is one new token's cache row and one group of
+// heads of one query row).
+// At most 72 registers a thread, so that four CTAs fit an SM (the absorption's 512 CTAs are one wave).
 template <int KTOT, int NSTAGE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 4)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      __nv_bfloat16* __restrict__ out, int batch, int nt, int64_t out_bstride,
                      int out_hstride, const uint4* __restrict__ qpe, const int32_t* __restrict__ q_pos,
@@ -164,16 +165,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // Warp w owns outputs m0 + 32w + [0, 32) for every n of the tile.  Lane = m in TMEM, so the
     // warp's [n][32 m] block goes through a stage in the (now idle) operand ring: each lane writes
     // its column, then every global store instruction covers eight whole 64-byte rows.
-    const int nrows = max(qpe != nullptr ? batch : 0, app.cache != nullptr ? app.n_tokens : 0);
+    // Work units of the side jobs: unit u is new token u of the append job (u < app.n_tokens) and,
+    // for the query rows, head group u % G of row u / G (G groups of 128 / G heads per row, G the
+    // largest power of two <= min(16, #CTAs / batch), so a small batch still spreads its rows'
+    // rotations over many CTAs).
+    const int ncta = gridDim.x * gridDim.y * gridDim.z;
+    int G = 1;
+    if (qpe != nullptr && batch > 0)
+      while (G < 16 && 2 * G * batch <= ncta) G *= 2;
+    const int nunits = max(qpe != nullptr ? batch * G : 0, app.cache != nullptr ? app.n_tokens : 0);
     {
       // Angle and rotation in fp64, one rounding per output (the same arithmetic as the cache
       // append's RoPE).  cs_sn: a query row's 32 (cos, sin) pairs, formed by threads 0..31.
       double* cs_sn = reinterpret_cast<double*>(tmem_slot + 4);
-      const int ncta = gridDim.x * gridDim.y * gridDim.z;
       const int c = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-      for (int n = c; n < nrows; n += ncta) {
-        if (app.cache != nullptr && n < app.n_tokens) {
-          // new token n: threads 0..63 copy the latent (16 B each), 64..95 rotate one key pair each
+      for (int u = c; u < nunits; u += ncta) {
+        if (app.cache != nullptr && u < app.n_tokens) {
+          // new token u: threads 0..63 copy the latent (16 B each), 64..95 rotate one key pair each
+          const int n = u;
           const int seq = app.seq_ids ? app.seq_ids[n] : n;
           const int p = app.pos[n];
           const int capacity = app.v.page_size == 0 ? app.v.max_seq_len : app.v.max_blocks * kPage;
@@ -195,28 +204,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
-        if (qpe == nullptr || n >= batch) continue;   // uniform across the 128 threads
-        if (q_pos != nullptr && threadIdx.x < kDRope / 2) {
-          double sn, cs;
-          sincos(static_cast<double>(q_pos[n]) * rope.inv_freq[threadIdx.x], &sn, &cs);
-          cs_sn[2 * threadIdx.x] = cs;
-          cs_sn[2 * threadIdx.x + 1] = sn;
-        }
-        named_bar_sync(1, 128);
-        for (int idx = threadIdx.x; idx < kHeads * (kDRope / 8); idx += 128) {   // (head, 16-byte chunk)
-          const int hh = idx >> 3;
-          const int ch = idx & 7;
-          const int64_t row = static_cast<int64_t>(n) * kHeads + hh;
-          uint4 r = qpe[row * (kDRope / 8) + ch];
-          if (q_pos != nullptr) {
-            __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(&r);
+        if (qpe == nullptr || u >= batch * G) continue;   // uniform across the 128 threads
+        const int n = u / G;
+        const int items = (kHeads / G) * (kDRope / 8);      // (head, 16-byte chunk) pairs of the group
+        const int item0 = (u % G) * items;
+        // The group's q_pe chunks are loaded (kChunk per thread at a time) before the angles are
+        // formed, so the two latencies overlap.
+        constexpr int kChunk = 4;
+        for (int k0 = 0; k0 < items; k0 += 128 * kChunk) {
+          uint4 r[kChunk];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) x[k] = rope_pair(x[k], cs_sn[2 * (4 * ch + k)], cs_sn[2 * (4 * ch + k) + 1]);
+          for (int k = 0; k < kChunk; ++k) {
+            const int idx = k0 + threadIdx.x + 128 * k;
+            if (idx < items) r[k] = qpe[static_cast<int64_t>(n) * kHeads * (kDRope / 8) + item0 + idx];
           }
-          reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * out_bstride +
-                                   static_cast<int64_t>(hh) * out_hstride)[kDLat / 8 + ch] = r;
+          if (k0 == 0) {
+            if (q_pos != nullptr && threadIdx.x < kDRope / 2) {
+              double sn, cs;
+              sincos(static_cast<double>(q_pos[n]) * rope.inv_freq[threadIdx.x], &sn, &cs);
+              cs_sn[2 * threadIdx.x] = cs;
+              cs_sn[2 * threadIdx.x + 1] = sn;
+            }
+            named_bar_sync(1, 128);
+          }
+#pragma unroll
+          for (int k = 0; k < kChunk; ++k) {
+            const int idx = k0 + threadIdx.x + 128 * k;
+            if (idx >= items) continue;
+            const int hh = (item0 + idx) >> 3;
+            const int ch = (item0 + idx) & 7;
+            if (q_pos != nullptr) {
+              __nv_bfloat162* x = reinterpret_cast<__nv_bfloat162*>(&r[k]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) x[e] = rope_pair(x[e], cs_sn[2 * (4 * ch + e)], cs_sn[2 * (4 * ch + e) + 1]);
+            }
+            reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * out_bstride +
+                                     static_cast<int64_t>(hh) * out_hstride)[kDLat / 8 + ch] = r[k];
+          }
         }
-        named_bar_sync(1, 128);   // the table is read before the next row overwrites it
+        named_bar_sync(1, 128);   // the table is read before the next unit overwrites it
       }
     }
     const bool ok = mbar_wait(done, 0);
