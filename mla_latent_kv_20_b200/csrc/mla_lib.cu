@@ -485,6 +485,13 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
   if (batch == 0) return MLA_OK;
   if (out_lat == nullptr || w_uv == nullptr || out == nullptr) return MLA_ERR_INVALID_ARG;
   if (!aligned16(out_lat) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
+  // One CTA per head streams that head's 128 KB of W_UV in four 128-row stages: with a batch of up
+  // to 64 rows all four stages fit in shared memory and are requested at once (one HBM round trip);
+  // larger batches (larger stages) go through a two-stage ring.
+  if (batch <= 64)
+    return launch_proj_gemm<mla::kDLat, 4>(w_uv, mla::kDHead, out_lat, batch, reinterpret_cast<__nv_bfloat16*>(out),
+                                           static_cast<int64_t>(mla::kHeads) * mla::kDHead, mla::kDHead,
+                                           as_stream(stream));
   return launch_proj_gemm<mla::kDLat, 2>(w_uv, mla::kDHead, out_lat, batch, reinterpret_cast<__nv_bfloat16*>(out),
                                          static_cast<int64_t>(mla::kHeads) * mla::kDHead, mla::kDHead,
                                          as_stream(stream));
