@@ -141,26 +141,32 @@ struct SegmentCursor {
   }
 };
 
-// Combine: one warp per (b, h); lanes own 16 of the 512 latent columns.  grid = (batch, 128 / 4),
-// block = 128, at most 64 registers a thread (8 blocks per SM: a 32-sequence batch is one wave).
-// Empty sequences get out_lat = 0 and lse = -inf; sequences finished by the decode kernel (one
-// segment) are skipped; the others merge their partials in ascending range order.
-__global__ void __launch_bounds__(128, 8) combine_kernel(Workspace ws, int P, __nv_bfloat16* __restrict__ out_lat,
+// Combine: one warp per (b, h) at a time; lanes own 16 of the 512 latent columns.  grid = (batch,
+// 128 / (4 hpw)), block = 128: warp w of block (b, y) takes heads 4 hpw y + w hpw + [0, hpw), so the
+// row's plan entries are read once for hpw heads (hpw = 1 for decode batches; 8 for many rows, as in
+// a prefill, where most rows are finished by the decode kernel and the blocks only read the plan).
+// At most 64 registers a thread for hpw = 1 (8 blocks per SM: a 32-sequence batch is one wave),
+// 128 otherwise.  Empty rows get out_lat = 0 and lse = -inf; rows finished by the decode kernel
+// (one segment) are skipped; the others merge their partials in ascending range order.
+template <int hpw>
+__global__ void __launch_bounds__(128, hpw == 1 ? 8 : 4) combine_kernel(Workspace ws, int P, __nv_bfloat16* __restrict__ out_lat,
                                                       float* __restrict__ lse) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x;
-  const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
+  const int h0 = (blockIdx.y * 4 + (threadIdx.x >> 5)) * hpw;
   const int lane = threadIdx.x & 31;
   const int B = gridDim.x;
   const bool per_seq = ws.off[B + 1] == kPlanPerSequence;
   const int T = ws.off[B];
   const int off = ws.off[b];
   const int span = ws.off[b + 1] - off;   // tiles (balanced) or ranges (per sequence) of b
-  __nv_bfloat16* dst = out_lat + (static_cast<int64_t>(b) * kHeads + h) * kDLat;
   if (span == 0) {
-    for (int i = lane; i < kDLat / 8; i += 32) reinterpret_cast<uint4*>(dst)[i] = make_uint4(0, 0, 0, 0);
-    if (lse != nullptr && lane == 0) lse[static_cast<int64_t>(b) * kHeads + h] = -INFINITY;
+    for (int h = h0; h < h0 + hpw; ++h) {
+      __nv_bfloat16* dst = out_lat + (static_cast<int64_t>(b) * kHeads + h) * kDLat;
+      for (int i = lane; i < kDLat / 8; i += 32) reinterpret_cast<uint4*>(dst)[i] = make_uint4(0, 0, 0, 0);
+      if (lse != nullptr && lane == 0) lse[static_cast<int64_t>(b) * kHeads + h] = -INFINITY;
+    }
     return;
   }
   // Ranges [p0, p1] that hold pieces of b; in the per-sequence plan each holds one (slot 2p).
@@ -169,60 +175,64 @@ __global__ void __launch_bounds__(128, 8) combine_kernel(Workspace ws, int P, __
   if (p0 == p1) return;
   auto slot_of = [&](int p) { return (!per_seq && range_start(p, P, T) < off) ? 2 * p + 1 : 2 * p; };
   auto nonempty = [&](int p) { return per_seq || range_start(p, P, T) < range_start(p + 1, P, T); };
-  // Online merge in ascending range order: after each range, (M, den, acc) hold the merge of the
-  // ranges so far relative to M.  Two ranges are fetched per step so their loads overlap (every
-  // partial's m is finite: a non-empty range holds at least one valid token of b).
-  float M = -INFINITY, den = 0.f;
-  float acc[16];
+#pragma unroll 1
+  for (int h = h0; h < h0 + hpw; ++h) {
+    __nv_bfloat16* dst = out_lat + (static_cast<int64_t>(b) * kHeads + h) * kDLat;
+    // Online merge in ascending range order: after each range, (M, den, acc) hold the merge of the
+    // ranges so far relative to M.  Two ranges are fetched per step so their loads overlap (every
+    // partial's m is finite: a non-empty range holds at least one valid token of b).
+    float M = -INFINITY, den = 0.f;
+    float acc[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  auto fetch = [&](int p, float& m, float& l, float4 (&o)[4]) -> bool {
-    if (p > p1 || !nonempty(p)) return false;
-    const int64_t ml = static_cast<int64_t>(slot_of(p)) * kHeads + h;
-    m = ws.m[ml];
-    l = ws.l[ml];
-    const float4* src = reinterpret_cast<const float4*>(ws.o + ml * kDLat);
+    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    auto fetch = [&](int p, float& m, float& l, float4 (&o)[4]) -> bool {
+      if (p > p1 || !nonempty(p)) return false;
+      const int64_t ml = static_cast<int64_t>(slot_of(p)) * kHeads + h;
+      m = ws.m[ml];
+      l = ws.l[ml];
+      const float4* src = reinterpret_cast<const float4*>(ws.o + ml * kDLat);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = src[lane + 32 * i];
-    return true;
-  };
-  auto merge = [&](float m, float l, const float4 (&o)[4]) {
-    const float Mn = fmaxf(M, m);
-    const float sa = M == -INFINITY ? 0.f : exp2f(M - Mn);
-    const float w = exp2f(m - Mn);
-    den = den * sa + w * l;
+      for (int i = 0; i < 4; ++i) o[i] = src[lane + 32 * i];
+      return true;
+    };
+    auto merge = [&](float m, float l, const float4 (&o)[4]) {
+      const float Mn = fmaxf(M, m);
+      const float sa = M == -INFINITY ? 0.f : exp2f(M - Mn);
+      const float w = exp2f(m - Mn);
+      den = den * sa + w * l;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[4 * i + 0] = acc[4 * i + 0] * sa + w * o[i].x;
+        acc[4 * i + 1] = acc[4 * i + 1] * sa + w * o[i].y;
+        acc[4 * i + 2] = acc[4 * i + 2] * sa + w * o[i].z;
+        acc[4 * i + 3] = acc[4 * i + 3] * sa + w * o[i].w;
+      }
+      M = Mn;
+    };
+    constexpr int kStep = 2;
+    for (int p = p0; p <= p1; p += kStep) {
+      float m[kStep], l[kStep];
+      float4 o[kStep][4];
+      bool has[kStep];
+#pragma unroll
+      for (int u = 0; u < kStep; ++u) has[u] = fetch(p + u, m[u], l[u], o[u]);
+#pragma unroll
+      for (int u = 0; u < kStep; ++u)
+        if (has[u]) merge(m[u], l[u], o[u]);
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      acc[4 * i + 0] = acc[4 * i + 0] * sa + w * o[i].x;
-      acc[4 * i + 1] = acc[4 * i + 1] * sa + w * o[i].y;
-      acc[4 * i + 2] = acc[4 * i + 2] * sa + w * o[i].z;
-      acc[4 * i + 3] = acc[4 * i + 3] * sa + w * o[i].w;
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc[4 * i + 0] * inv, acc[4 * i + 1] * inv);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc[4 * i + 2] * inv, acc[4 * i + 3] * inv);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(dst)[lane + 32 * i] = pk;
     }
-    M = Mn;
-  };
-  constexpr int kStep = 2;
-  for (int p = p0; p <= p1; p += kStep) {
-    float m[kStep], l[kStep];
-    float4 o[kStep][4];
-    bool has[kStep];
-#pragma unroll
-    for (int u = 0; u < kStep; ++u) has[u] = fetch(p + u, m[u], l[u], o[u]);
-#pragma unroll
-    for (int u = 0; u < kStep; ++u)
-      if (has[u]) merge(m[u], l[u], o[u]);
+    if (lse != nullptr && lane == 0)
+      lse[static_cast<int64_t>(b) * kHeads + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
   }
-  const float inv = den > 0.f ? 1.f / den : 0.f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc[4 * i + 0] * inv, acc[4 * i + 1] * inv);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc[4 * i + 2] * inv, acc[4 * i + 3] * inv);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&lo);
-    pk.y = *reinterpret_cast<uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(dst)[lane + 32 * i] = pk;
-  }
-  if (lse != nullptr && lane == 0)
-    lse[static_cast<int64_t>(b) * kHeads + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
 }
 
 }  // namespace mla

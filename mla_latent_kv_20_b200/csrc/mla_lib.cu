@@ -568,7 +568,11 @@ mla_status launch_attn(const mla_bf16* q_full, const mla_bf16* cache, const int3
   mla_status ls = launch_chained(kernel, dim3(2 * P), dim3(mla::kTcThreads), static_cast<size_t>(mla::kTcSmemBytes), s,
                                  tka, tkb, tv, tq, a);
   if (ls != MLA_OK) return ls;
-  return launch_chained(mla::combine_kernel, dim3(rows, mla::kHeads / 4), dim3(128), 0, s, a.ws, P,
+  // Many rows (a prefill): each warp takes 8 heads of its row, so the plan is read by 8x fewer blocks.
+  if (rows > 512)
+    return launch_chained(mla::combine_kernel<8>, dim3(rows, mla::kHeads / 32), dim3(128), 0, s, a.ws, P,
+                          reinterpret_cast<__nv_bfloat16*>(out_lat), lse);
+  return launch_chained(mla::combine_kernel<1>, dim3(rows, mla::kHeads / 4), dim3(128), 0, s, a.ws, P,
                         reinterpret_cast<__nv_bfloat16*>(out_lat), lse);
 }
 

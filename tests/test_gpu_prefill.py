@@ -73,6 +73,22 @@ def test_prefill_vs_oracle(env, paged, splits):
         assert_lse(g_lse[i], ref["lse"][i])
 
 
+def test_prefill_many_rows_vs_oracle(env):
+    """More than 512 query rows (the combine then gives each warp 8 heads of a row): 600 new tokens of
+    two sequences, many rows split between work ranges."""
+    m = env[0]
+    lens, news = [640, 400], [360, 240]
+    cache, qf_bits, q_seq, q_len, rows = _case(env, lens, news, 950, False)
+    g_lat, g_lse = _prefill(env, cache, qf_bits, q_seq, q_len)
+    assert m.get_device_error() == 0
+    ref = oracle.prefill_rows(f64(qf_bits), rows, q_seq, q_len, SCALE, 512)
+    for i in range(len(q_seq)):
+        kv = rows[q_seq[i]][:q_len[i]]
+        p = oracle.attend_rows(f64(qf_bits[i]), kv, SCALE, 512)["p"]
+        assert_out_lat_rows(g_lat[i], ref["out_lat"][i], p @ np.abs(kv[:, :512]))
+        assert_lse(g_lse[i], ref["lse"][i])
+
+
 def test_prefill_paged_bit_identical_to_contiguous(env):
     lens, news = [200, 77], [64, 30]
     c1 = _case(env, lens, news, 910, False)
