@@ -290,20 +290,21 @@ bool cluster16_ok(K kernel, int threads, int smem) {
 }
 
 // One output-projection launch with K split over SPLIT-CTA clusters.
-template <int SPLIT>
+template <int SPLIT, int NT>
 mla_status launch_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y, int32_t batch, void* stream) {
+  using Sh = mla::OpShape<NT>;
   CUtensorMap tw, tx;
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kOpIn) * 2, 128};
   const cuuint64_t dw[3] = {64, static_cast<cuuint64_t>(mla::kOpOut), mla::kOpIn / 64};
   const cuuint64_t dx[3] = {64, static_cast<cuuint64_t>(batch), mla::kOpIn / 64};
   const cuuint32_t bw[3] = {64, 128, static_cast<cuuint32_t>(mla::kOpKS / 64)};
-  const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(mla::kOpNt), static_cast<cuuint32_t>(mla::kOpKS / 64)};
+  const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(NT), static_cast<cuuint32_t>(mla::kOpKS / 64)};
   if (!make_map_3d(&tw, w_o, dw, strides, bw) || !make_map_3d(&tx, out, dx, strides, bx)) return MLA_ERR_CUDA;
-  auto kern = mla::out_proj_kernel<SPLIT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kOpSmemBytes) != cudaSuccess)
+  auto kern = mla::out_proj_kernel<SPLIT, NT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
-  const dim3 grid(SPLIT, mla::kOpMTiles, (batch + mla::kOpNt - 1) / mla::kOpNt);
-  return launch_chained_cluster(kern, grid, dim3(mla::kOpThreads), static_cast<size_t>(mla::kOpSmemBytes),
+  const dim3 grid(SPLIT, mla::kOpMTiles, (batch + NT - 1) / NT);
+  return launch_chained_cluster(kern, grid, dim3(mla::kOpThreads), static_cast<size_t>(Sh::kSmemBytes),
                                 as_stream(stream), SPLIT, tw, tx, reinterpret_cast<__nv_bfloat16*>(y), batch);
 }
 
@@ -389,7 +390,9 @@ mla_status mla_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y
   if (!aligned16(out) || !aligned16(w_o) || !aligned16(y)) return MLA_ERR_INVALID_ARG;
   // 8-CTA clusters: twice as many clusters are resident at once as with 16 (measured 57 vs 72 us
   // per call on 32 sequences with the weight coming from HBM).
-  return launch_output_proj<8>(out, w_o, y, batch, stream);
+  // Tiles of 32 sequences up to 32, else of 128 (W_O then streams once per 128 sequences).
+  if (batch <= 32) return launch_output_proj<8, 32>(out, w_o, y, batch, stream);
+  return launch_output_proj<8, 128>(out, w_o, y, batch, stream);
 }
 
 }  // extern "C"

@@ -6,13 +6,15 @@
 // on the un-absorbed heads' outputs.  Products exact in fp32, sums over the 16384 inputs in fp32,
 // one rounding of y to bf16.
 //
-// B200 mapping.  The weight (5120 x 16384 bf16, 168 MB) streams from HBM once per call and is the
-// M operand ("swap-AB": M = output dims in 40 tiles of 128, N = sequences in tiles of 32, K =
-// 16384); K is split over the SPLIT CTAs of a cluster (8: twice as many such clusters are
-// resident at once as 16-CTA ones), each streaming its share through a 4-stage ring of 40 KB stages while two
-// threads issue the MMAs into two TMEM accumulators; the SPLIT partial tiles are reduced through
-// distributed shared memory (CTA r sums rows [R r, R r + R), R = 128 / SPLIT) and written as bf16.
-// grid = (SPLIT, 40, ceil(B / 32)), clusters of SPLIT along x (set at launch); 224 threads: warps
+// B200 mapping.  The weight (5120 x 16384 bf16, 168 MB) streams from HBM once per N tile and is the
+// M operand ("swap-AB": M = output dims in 40 tiles of 128, N = sequences in tiles of NT = 32, or
+// of 128 for batches above 32 so that the weight streams once per 128 sequences, K = 16384); K is
+// split over the SPLIT CTAs of a cluster (8: twice as many such clusters are resident at once as
+// 16-CTA ones), each streaming its share through a ring of 40 KB (NT = 32, 4 stages) or 64 KB
+// (NT = 128, 3 stages) stages while two threads issue the MMAs into two TMEM accumulators; the
+// SPLIT partial tiles are reduced through distributed shared memory (CTA r sums rows [R r, R r + R),
+// R = 128 / SPLIT) and written as bf16.
+// grid = (SPLIT, 40, ceil(B / NT)), clusters of SPLIT along x (set at launch); 224 threads: warps
 // 0-3 epilogue and reduction, warp 4 TMA producer, warps 5-6 MMA issuers.
 #pragma once
 
@@ -26,21 +28,25 @@ namespace mla {
 constexpr int kOpIn = kHeads * kDHead;   // 16384 inputs
 constexpr int kOpOut = kDHidden;         // 5120 outputs
 constexpr int kOpMTiles = kOpOut / 128;
-constexpr int kOpNt = 32;                // sequences per N tile
 constexpr int kOpKS = 128;               // contraction columns per stage
-constexpr int kOpRing = 4;               // stages in flight
 constexpr int kOpThreads = 224;
 constexpr int kOpWBytes = kOpKS * 128 * 2;
-constexpr int kOpXBytes = kOpKS * kOpNt * 2;
-constexpr int kOpStageBytes = kOpWBytes + kOpXBytes;
-constexpr int kOpSmemBytes = 1024 + kOpRing * kOpStageBytes + 256;
 static_assert(kOpOut % 128 == 0, "M tiles");
-static_assert(128 * (kOpNt + 1) * 4 <= kOpRing * kOpStageBytes, "reduction tile fits in the operand ring");
-static_assert(kOpSmemBytes <= 232448, "shared memory budget");
+// Per N tile of NT sequences (32, or 128 for larger batches, so that W_O streams once per 128
+// sequences): stages in flight, stage and shared-memory bytes.
+template <int NT>
+struct OpShape {
+  static constexpr int kRing = NT <= 32 ? 4 : 3;
+  static constexpr int kXBytes = kOpKS * NT * 2;
+  static constexpr int kStageBytes = kOpWBytes + kXBytes;
+  static constexpr int kSmemBytes = 1024 + kRing * kStageBytes + 256;
+  static_assert(128 * (NT + 1) * 4 <= kRing * kStageBytes, "reduction tile fits in the operand ring");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
 
 // tmW: 3-D view of W_O [5120][16384] (64-column chunk, row, chunk index), box {64, 128, 2}.
-// tmX: the same view of out [B][16384], box {64, 32, 2} (rows past B arrive as zeros).
-template <int SPLIT>
+// tmX: the same view of out [B][16384], box {64, NT, 2} (rows past B arrive as zeros).
+template <int SPLIT, int NT>
 __global__ void __launch_bounds__(kOpThreads, 1)
     out_proj_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                     __nv_bfloat16* __restrict__ y, int batch) {
@@ -48,7 +54,10 @@ __global__ void __launch_bounds__(kOpThreads, 1)
   constexpr int KPER = kOpIn / SPLIT;       // contraction columns of one CTA
   constexpr int NST = KPER / kOpKS;         // its stages
   constexpr int R = 128 / SPLIT;            // tile rows each CTA reduces
-  constexpr int JN = kOpNt * R / 128;       // outputs per thread in the reduction
+  constexpr int JN = NT * R / 128;          // outputs per thread in the reduction
+  using Sh = OpShape<NT>;
+  constexpr int kOpRing = Sh::kRing;
+  constexpr int kOpStageBytes = Sh::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOpRing * kOpStageBytes);
@@ -62,10 +71,10 @@ __global__ void __launch_bounds__(kOpThreads, 1)
   const int lane = threadIdx.x & 31;
   const int rank = static_cast<int>(cluster_ctarank());
   const int mt = blockIdx.y;
-  const int n0 = blockIdx.z * kOpNt;
+  const int n0 = blockIdx.z * NT;
   const int kc0 = rank * KPER / 64;   // first 64-column chunk of this CTA
-  constexpr uint32_t kAccCols = kOpNt;
-  constexpr uint32_t kTmemCols = 64;
+  constexpr uint32_t kAccCols = NT;
+  constexpr uint32_t kTmemCols = 2 * NT;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kOpRing; ++s) {
@@ -114,7 +123,7 @@ __global__ void __launch_bounds__(kOpThreads, 1)
     // ---------------- MMA issuers: warp 5 + j takes the 16-deep K steps with index % 2 == j
     const int j = warp - 5;
     const uint32_t acc = tmem_d + j * kAccCols;
-    const uint32_t idesc = idesc_bf16_f32(128, kOpNt, /*a_mn_major=*/false, /*b_mn_major=*/false);
+    const uint32_t idesc = idesc_bf16_f32(128, NT, /*a_mn_major=*/false, /*b_mn_major=*/false);
     bool first = true;
     for (int q = 0; q < NST; ++q) {
       const int s = q % kOpRing;
@@ -129,7 +138,7 @@ __global__ void __launch_bounds__(kOpThreads, 1)
       for (int kk = j; kk < kOpKS / 16; kk += 2) {
         // A (K-major): chunk kk / 4 of 128 rows x 128 B; B (K-major): chunk kk / 4 of 32 rows x 128 B.
         const uint64_t adesc = sdesc_sw128(sa + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-        const uint64_t bdesc = sdesc_sw128(sb + (kk >> 2) * (kOpNt * 128) + (kk & 3) * 32, 16, 1024);
+        const uint64_t bdesc = sdesc_sw128(sb + (kk >> 2) * (NT * 128) + (kk & 3) * 32, 16, 1024);
         umma_bf16_ss(acc, adesc, bdesc, idesc, first ? 0u : 1u);
         first = false;
       }
@@ -144,13 +153,13 @@ __global__ void __launch_bounds__(kOpThreads, 1)
     const uint32_t trow = tmem_d + (static_cast<uint32_t>(warp * 32) << 16);
     uint32_t r0[16], r1[16];
 #pragma unroll
-    for (int c = 0; c < kOpNt; c += 16) {
+    for (int c = 0; c < NT; c += 16) {
       tmem_ld16(trow + c, r0);
       tmem_ld16(trow + kAccCols + c, r1);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        red[m * (kOpNt + 1) + c + i] = ok ? __uint_as_float(r0[i]) + __uint_as_float(r1[i]) : 0.f;
+        red[m * (NT + 1) + c + i] = ok ? __uint_as_float(r0[i]) + __uint_as_float(r1[i]) : 0.f;
     }
     if (!ok) *abort_flag = 1;
     // Cluster barrier 1 (each thread arrives once; warps 4-6 arrive below, after their roles).
@@ -171,22 +180,26 @@ __global__ void __launch_bounds__(kOpThreads, 1)
 #pragma unroll
       for (int q = 0; q < SPLIT; ++q) flags |= __float_as_int(f[q]);
     }
-    float part[JN][SPLIT];   // all loads in flight at once, then the sums in rank order
+    constexpr int kJC = JN < 4 ? JN : 4;   // outputs per batch of loads
+#pragma unroll 1
+    for (int j0 = 0; j0 < JN; j0 += kJC) {
+      float part[kJC][SPLIT];   // a batch's loads all in flight at once, then the sums in rank order
 #pragma unroll
-    for (int jn = 0; jn < JN; ++jn) {
-      const int nl = t / R + (128 / R) * jn;
-      const uint32_t off = red_addr + 4u * static_cast<uint32_t>(mr * (kOpNt + 1) + nl);
+      for (int jj = 0; jj < kJC; ++jj) {
+        const int nl = t / R + (128 / R) * (j0 + jj);
+        const uint32_t off = red_addr + 4u * static_cast<uint32_t>(mr * (NT + 1) + nl);
 #pragma unroll
-      for (int q = 0; q < SPLIT; ++q) part[jn][q] = ld_shared_cluster_f32(mapa_shared(off, q));
-    }
+        for (int q = 0; q < SPLIT; ++q) part[jj][q] = ld_shared_cluster_f32(mapa_shared(off, q));
+      }
 #pragma unroll
-    for (int jn = 0; jn < JN; ++jn) {
-      float sum = 0.f;
+      for (int jj = 0; jj < kJC; ++jj) {
+        float sum = 0.f;
 #pragma unroll
-      for (int q = 0; q < SPLIT; ++q) sum += part[jn][q];
-      const int n = n0 + t / R + (128 / R) * jn;
-      if (n < batch && flags == 0)
-        y[static_cast<int64_t>(n) * kOpOut + 128 * mt + mr] = __float2bfloat16_rn(sum);
+        for (int q = 0; q < SPLIT; ++q) sum += part[jj][q];
+        const int n = n0 + t / R + (128 / R) * (j0 + jj);
+        if (n < batch && flags == 0)
+          y[static_cast<int64_t>(n) * kOpOut + 128 * mt + mr] = __float2bfloat16_rn(sum);
+      }
     }
   }
   if (warp >= 4) {

@@ -27,7 +27,7 @@ def _heads_out(seed, batch):
     return mi.f64_to_bf16(rng.standard_normal((batch, mi.N_HEADS, mi.D_HEAD)))
 
 
-@pytest.mark.parametrize("batch", [1, 17, 32, 33, 100])
+@pytest.mark.parametrize("batch", [1, 17, 32, 33, 100, 300])
 def test_output_proj_vs_oracle(env, batch):
     m, hz, torch, w_o, w_o_dev = env
     out = _heads_out(700 + batch, batch)
