@@ -282,7 +282,7 @@ def setup_replica(name, device):
 # counters were taken, and the traffic is reported as null.
 TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh", "csrc/mla_lib.cu")
 MEASURED_TRAFFIC = {   # workload -> {"bytes": int, "sha256": str, "profile": str}
-    "b32_l4096": {"bytes": 155799552 + 3456512 + 16860928, "sha256": "bfca7041f9b220c431aa9e2f337e6d795c279e2bacf3a22fe757ff616d27bf43",
+    "b32_l4096": {"bytes": 155800320 + 3449344 + 16858880, "sha256": "d2d222cae8eb16d5ba01634a13f5b483c3a047b20bbfdaf4e77e73e9e52a37bb",
                   "profile": "profiles/decode_tc_b32_l4096.md (decode + combine, ncu cache flush per kernel)"},
 }
 
