@@ -151,7 +151,7 @@ def block_permutation(seed: int, seq_lens, page: int = PAGE, max_blocks: int | N
     return table, total
 
 
-# Workload presets (sizes of the five decode workloads; see the design doc for the recipe).
+# Workload presets: the five decode workloads (batch, length distribution, cache layout, seed).
 WORKLOADS = {
     "b1_l256": dict(batch=1, lens="fixed", L=256, paged=False, seed=1001),
     "b32_l4096": dict(batch=32, lens="fixed", L=4096, paged=False, seed=1002),

@@ -14,7 +14,7 @@ Sources (page title, section):
        §2.1 MLA把KV缓存从瓶颈变成可压缩项.
   [DP] DeepSeek V2技术解析：MLA架构如何重塑大模型推理效率 (devpress.csdn.net), §1.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
   * softmax scale 1/sqrt(d_h + d_R) = 1/sqrt(192) (the pages never state it);
   * RoPE on the decoupled branch uses the interleaved pairing (x[2i], x[2i+1]) rotated by
     pos * theta_i, theta_i = base^(-2i/d_R), base 10000 (the pages name RoPE but print no
