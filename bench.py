@@ -495,7 +495,7 @@ def run_step(st, i):
             layer_phase(st, i, li, k)
 
 
-class cuda_runtime:
+class CudaRuntime:
     """The few CUDA runtime calls the end-to-end loop issues directly (async copies from and to
     pinned host memory, events without timing): the process's libcudart, loaded by torch."""
     H2D, D2H = 1, 2
@@ -664,7 +664,7 @@ def run_ours(args, rank, world, local_rank):
     # inputs, and its read-back waits for its own kernels.  Copies and the events that order them are
     # issued straight through the CUDA runtime (what a native serving loop calls).  The timed region
     # spans all K steps, from before the first input copy to the end of the last read-back.
-    rt = cuda_runtime()
+    rt = CudaRuntime()
     copy_stream = torch.cuda.Stream()
     compute_stream = torch.cuda.current_stream()
     keys = [list(layer["dev"].keys()) for layer in st["layers"]]
