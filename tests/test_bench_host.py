@@ -28,3 +28,37 @@ def test_clock_summary_without_nvidia_smi():
     cs = bench.ClockSampler(0)
     got = cs.summary(0.0, 1.0)
     assert got["reasons"] == ["nvidia-smi unavailable"] and got["samples"] == 0
+
+
+def test_recorded_traffic_follows_the_sources():
+    """The decode call's DRAM bytes are reported only while the kernel sources hash to the digest
+    recorded with them (a changed kernel reports null, not a stale number)."""
+    import bench
+    rec = bench.MEASURED_TRAFFIC["b32_l4096"]
+    assert bench.recorded_traffic("b32_l4096") in (None, rec["bytes"])
+    assert bench.recorded_traffic("no_such_workload") is None
+    saved = rec["sha256"]
+    try:
+        rec["sha256"] = "0" * 64
+        assert bench.recorded_traffic("b32_l4096") is None
+    finally:
+        rec["sha256"] = saved
+
+
+def test_job_throughput_is_whole_job():
+    """value = the bytes every rank processed over the max-over-ranks time."""
+    import bench
+    assert abs(bench.job_throughput(1e9, 1, 1.0) - 1000.0) < 1e-9
+    assert abs(bench.job_throughput(1e9, 4, 2.0) - 2000.0) < 1e-9
+
+
+def test_step_work_counts_bytes_and_flops():
+    """Per cached token per layer: 1152 bytes and 2*128*(576 + 512) flops; per sequence the absorb
+    and un-absorb GEMMs (2 x 2*128*128*512 flops); the decode call's bytes add q_full in and out_lat
+    out per sequence."""
+    import bench
+    lens = [3, 5]
+    tokens, cache_bytes, flops, dec_bytes = bench.step_work(lens)
+    assert tokens == 8 and cache_bytes == 8 * 1152
+    assert flops == 8 * 2 * 128 * (576 + 512) + 2 * 2 * (2 * 128 * 128 * 512)
+    assert dec_bytes == cache_bytes + 2 * 128 * (576 + 512) * 2
