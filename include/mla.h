@@ -1,10 +1,14 @@
 /*
  * mla.h — C ABI of the B200 (sm_100a) library for DeepSeek-V2 Multi-head Latent Attention (MLA)
- * decode over the compressed latent KV cache, in its weight-absorbed form.
+ * decode over the compressed latent KV cache, in its weight-absorbed form: (1) cache append,
+ * (2) query absorption, (3) decode attention (split over work ranges, merged by a combine),
+ * (4) value un-absorption, and beside them (1') the down-projection + append of new tokens,
+ * (6) the output projection and (7) chunked-prefill attention.
  *
  * Sources (page title, section):
  *   [DR] 《DeepSeek-V2》深度解读报告 — §2.2 Low-Rank Key-Value Joint Compression,
- *        §2.3 Absorption, §2.4 Decoupled Rotary Position Embedding, §3.1 MLA 完整计算链路与参数核算.
+ *        §2.3 Absorption, §2.4 Decoupled Rotary Position Embedding, §3.1 MLA 完整计算链路与参数核算,
+ *        §3.3 (model width), §4.2 效率证据 (prompt throughput).
  *   [XD] DeepSeek-V2论文解读：MoE架构如何实现训练成本降42.5%与KV缓存压93.3% — §2.1.
  *
  * Fixed model dimensions ([DR] §3.1): n_h = 128 heads, d_h = 128, d_c = 512, d_R = 64.
