@@ -527,3 +527,86 @@ def test_pins_catch_planted_prefill_mistakes():
         return oracle.prefill_explicit_masked(qn, qp, c, kr, w_uk, w_uv, scale, np.asarray(q_pos) - 1)
 
     assert _fails(check_prefill_against_masked_explicit, oracle.prefill_rows, masked_inclusive)
+
+
+# ------------------------------------------------------------------ whole decode step: positions
+# 《DeepSeek-V2》深度解读报告 §2.4 Decoupled RoPE: the shared key k^R of the token at position t is
+# cached rotated by RoPE at t, and the query's position part q^R is rotated at the query's own
+# position.  decode_step does that rotation itself (token t of sequence b sits at position t), so
+# its positional glue is pinned here by scalar loops that rotate every pair with math.cos/sin.
+def bf_rotate(x, pos, base=oracle.ROPE_BASE):
+    """One interleaved RoPE rotation by scalar loops: pair (x[2i], x[2i+1]) turned by
+    pos * base^(-2i/d)."""
+    d = len(x)
+    y = []
+    for i in range(d // 2):
+        a = float(pos) * float(base) ** (-2.0 * i / d)
+        u, v = float(x[2 * i]), float(x[2 * i + 1])
+        y += [u * math.cos(a) - v * math.sin(a), u * math.sin(a) + v * math.cos(a)]
+    return np.array(y)
+
+
+def bf_decode_step(q_nope, q_pe, cs, krs_raw, w_uk, w_uv, scale, q_pos=None):
+    """Scalar-loop decode step: keys rotated at their token index, q^R at q_pos[b] (as given when
+    q_pos is None), then the scalar-loop attention and the scalar-loop absorbed query."""
+    out, lat, lse, qa = [], [], [], []
+    for b in range(len(cs)):
+        L = cs[b].shape[0]
+        kr_rot = np.array([bf_rotate(krs_raw[b][t], t) for t in range(L)])
+        qpe = np.array(q_pe[b]) if q_pos is None else np.array([bf_rotate(q_pe[b][h], q_pos[b])
+                                                                 for h in range(q_pe.shape[1])])
+        o, l_, s = bf_attention(q_nope[b], qpe, cs[b], kr_rot, w_uk, w_uv, scale)
+        out.append(o); lat.append(l_); lse.append(s)
+        H, dh, dc = w_uk.shape
+        qa.append([[sum(float(q_nope[b, h, j]) * float(w_uk[h, j, k]) for j in range(dh)) for k in range(dc)]
+                   for h in range(H)])
+    return dict(out=np.array(out), out_lat=np.array(lat), lse=np.array(lse), q_abs=np.array(qa))
+
+
+def check_decode_step_positions(decode_step):
+    rng = np.random.default_rng(61)
+    H, dh, dc, dr = 2, 3, 4, 4           # two RoPE pairs: theta_0 = 1 and theta_1 = 10000^(-1/2)
+    lens = [3, 5]
+    q_nope = rng.standard_normal((2, H, dh))
+    q_pe = rng.standard_normal((2, H, dr))
+    cs = [rng.standard_normal((L, dc)) for L in lens]
+    krs = [rng.standard_normal((L, dr)) for L in lens]
+    w_uk = rng.standard_normal((H, dh, dc)) * 0.5
+    w_uv = rng.standard_normal((H, dc, dh)) * 0.5
+    # the new token's own position (L - 1), an arbitrary one, and q^R taken as already rotated
+    for q_pos in ([L - 1 for L in lens], [7, 1], None):
+        ref = bf_decode_step(q_nope, q_pe, cs, krs, w_uk, w_uv, 0.45, q_pos)
+        for form in ("explicit", "absorbed"):
+            got = decode_step(q_nope, q_pe, cs, krs, w_uk, w_uv, 0.45, q_pos=q_pos, form=form)
+            for k in ("out", "out_lat", "lse", "q_abs"):
+                assert np.allclose(got[k], ref[k], rtol=1e-12, atol=1e-12), (q_pos, form, k)
+
+
+def test_decode_step_positions_pin():
+    check_decode_step_positions(oracle.decode_step)
+
+
+def test_pins_catch_planted_decode_step_mistakes():
+    # R(t) R(1) = R(t + 1): rotating every raw key by one position first plants "keys at t + 1".
+    def keys_one_late(q_nope, q_pe, cs, krs, w_uk, w_uv, scale, base=oracle.ROPE_BASE, q_pos=None, form="explicit"):
+        krs1 = [oracle.apply_rope(k, 1, base) for k in krs]
+        return oracle.decode_step(q_nope, q_pe, cs, krs1, w_uk, w_uv, scale, base, q_pos, form)
+
+    def keys_unrotated(q_nope, q_pe, cs, krs, w_uk, w_uv, scale, base=oracle.ROPE_BASE, q_pos=None, form="explicit"):
+        # R(-t) R(t) = identity: undo the step's own rotation of token t
+        krs0 = [oracle.apply_rope(k, -np.arange(len(k)), base) for k in krs]
+        return oracle.decode_step(q_nope, q_pe, cs, krs0, w_uk, w_uv, scale, base, q_pos, form)
+
+    def query_unrotated(q_nope, q_pe, cs, krs, w_uk, w_uv, scale, base=oracle.ROPE_BASE, q_pos=None, form="explicit"):
+        return oracle.decode_step(q_nope, q_pe, cs, krs, w_uk, w_uv, scale, base, None, form)
+
+    def query_at_length(q_nope, q_pe, cs, krs, w_uk, w_uv, scale, base=oracle.ROPE_BASE, q_pos=None, form="explicit"):
+        qp = None if q_pos is None else [len(c) for c in cs]
+        return oracle.decode_step(q_nope, q_pe, cs, krs, w_uk, w_uv, scale, base, qp, form)
+
+    def query_negated_angle(q_nope, q_pe, cs, krs, w_uk, w_uv, scale, base=oracle.ROPE_BASE, q_pos=None, form="explicit"):
+        qp = None if q_pos is None else [-p for p in q_pos]
+        return oracle.decode_step(q_nope, q_pe, cs, krs, w_uk, w_uv, scale, base, qp, form)
+
+    for bad in (keys_one_late, keys_unrotated, query_unrotated, query_at_length, query_negated_angle):
+        assert _fails(check_decode_step_positions, bad), bad.__name__
