@@ -227,8 +227,11 @@ mla_status mla_prefill_attn(const mla_bf16* q_full, const mla_bf16* cache, const
  * loads the library holds until the process exits.
  *   - Returns MLA_ERR_WORKSPACE, launching nothing, when mla_decode_workspace_size(batch,
  *     capacity, num_splits) exceeds MLA_NOALLOC_SCRATCH_BYTES (use fewer ranges).
- *   - The first call on a device looks up the buffer's device address (once per device, with that
- *     device current); make that first call before any stream capture.
+ *   - Every call looks up the buffer's device address for the calling thread's current context
+ *     (cudaGetSymbolAddress: no allocation, about a microsecond of host time), so a host engine
+ *     that runs the library under a context of its own, or re-creates a context after a device
+ *     reset, gets that context's copy.  The first call in a context may load the library's device
+ *     code there; make that first call before any stream capture.
  *   - All calls share the one buffer: calls whose kernels overlap on the GPU (different streams,
  *     no ordering between them) race and give wrong results.  The buffer keeps the last call's
  *     contents; nothing in it needs to start at zero (the kernels overwrite what they read).
@@ -239,6 +242,9 @@ mla_status mla_decode_attn_noalloc(const mla_bf16* q_full, const mla_bf16* cache
                                    const int32_t* seq_lens, mla_cache_desc desc, int32_t batch,
                                    float softmax_scale, int32_t num_splits, mla_bf16* out_lat, float* lse,
                                    void* stream);
+/* The size of that static buffer in bytes (MLA_NOALLOC_SCRATCH_BYTES as this build was compiled),
+ * so that a binding need not restate the constant. */
+size_t mla_noalloc_scratch_bytes(void);
 
 /*
  * (4) Value un-absorption — [DR] §2.3 and [XD] §2.1 (W_UV applied after attention; folding

@@ -62,6 +62,7 @@ def _load():
         "mla_prefill_attn": (ctypes.c_int, [P, P, P, P, P, CacheDesc, I32, F32, I32, P, SZ, P, P, P]),
         "mla_unabsorb_v": (ctypes.c_int, [P, P, P, I32, P]),
         "mla_decode_attn_noalloc": (ctypes.c_int, [P, P, P, P, CacheDesc, I32, F32, I32, P, P, P]),
+        "mla_noalloc_scratch_bytes": (SZ, []),
         "mla_get_device_error": (ctypes.c_int, [ctypes.POINTER(I32)]),
     }
     for name, (res, args) in sigs.items():
@@ -169,7 +170,7 @@ def prefill_attn(q_full, cache, q_seq, q_len, desc: CacheDesc, workspace, out_la
                                 _stream(stream)), "mla_prefill_attn")
 
 
-NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
+NOALLOC_SCRATCH_BYTES = int(lib.mla_noalloc_scratch_bytes())   # the library's own constant
 
 
 def decode_attn_noalloc(q_full, cache, seq_lens, desc: CacheDesc, out_lat, *, lse=None, block_table=None,

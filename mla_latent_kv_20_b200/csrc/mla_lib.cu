@@ -607,26 +607,19 @@ mla_status mla_prefill_attn(const mla_bf16* q_full, const mla_bf16* cache, const
 // ------------------------------------------------------------------------------------------
 namespace {
 
-// One buffer per device (a __device__ array exists once in every context that loads the
-// library).  Host code must not pass its host-side symbol: the device address is looked up with
-// cudaGetSymbolAddress once per device, with that device current.
+// One buffer per context: a __device__ array exists once in every CUDA context that loads the
+// library (the primary context of each device, and any context a host engine creates and makes
+// current).  Host code must not pass the array's host-side symbol to a kernel: its device address
+// is looked up with cudaGetSymbolAddress, with the calling thread's context current, on every call.
+// The lookup allocates nothing and costs about a microsecond of host time; caching it per device
+// would hand a stale address to a call made under another context of the same device, or after
+// the device was reset and its context re-created.
 __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[kMaxDevices] = {nullptr};
-
 mla_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return MLA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MLA_ERR_CUDA;
+  *out = p;
   return MLA_OK;
 }
 
@@ -647,3 +640,5 @@ extern "C" mla_status mla_decode_attn_noalloc(const mla_bf16* q_full, const mla_
   return mla_decode_attn(q_full, cache, block_table, seq_lens, desc, batch, softmax_scale, num_splits, scratch,
                          MLA_NOALLOC_SCRATCH_BYTES, out_lat, lse, stream);
 }
+
+extern "C" size_t mla_noalloc_scratch_bytes(void) { return MLA_NOALLOC_SCRATCH_BYTES; }

@@ -47,7 +47,19 @@ def test_status_strings(mla):
 FAKE = 0x10000  # never dereferenced: validation fails first
 
 
-def test_append_validation(mla):
+@pytest.fixture
+def host_only(mla):
+    """The tests below pass never-dereferenced addresses and check that host validation refuses
+    them before any device call.  They run only where no GPU is visible, so that a regression in
+    the validation could never hand such an address to a kernel."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-validation test with placeholder addresses: runs only without a GPU")
+    return mla
+
+
+def test_append_validation(host_only):
+    mla = host_only
     lib = mla.lib
     good = mla.contiguous_desc(4, 128)
     assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, None, None, good, 4, 10000.0, None) == 1  # null cache
@@ -66,7 +78,8 @@ def test_append_validation(mla):
     assert lib.mla_cache_append(FAKE, FAKE, None, FAKE, FAKE, None, too_few_rows, 1, 10000.0, None) == 1
 
 
-def test_projection_validation(mla):
+def test_projection_validation(host_only):
+    mla = host_only
     lib = mla.lib
     assert lib.mla_absorb_q(FAKE, FAKE, None, FAKE, FAKE, 0, 10000.0, None) == 0
     assert lib.mla_absorb_q(FAKE, FAKE, None, FAKE, FAKE, -1, 10000.0, None) == 1
@@ -79,7 +92,8 @@ def test_projection_validation(mla):
     assert lib.mla_unabsorb_v(FAKE, FAKE, FAKE + 4, 4, None) == 1
 
 
-def test_decode_validation_and_workspace(mla):
+def test_decode_validation_and_workspace(host_only):
+    mla = host_only
     lib = mla.lib
     d = mla.contiguous_desc(8, 4096)
     S = lib.mla_decode_num_splits(8, 4096, 16)
@@ -104,7 +118,8 @@ def test_decode_validation_and_workspace(mla):
     assert lib.mla_get_device_error(None) == 1
 
 
-def test_prefill_validation(mla):
+def test_prefill_validation(host_only):
+    mla = host_only
     """Host checks of mla_prefill_attn (no kernel is launched on any of these paths): the query
     rows may outnumber the cache's sequences (several rows read one sequence), the map is required."""
     lib = mla.lib
@@ -119,7 +134,8 @@ def test_prefill_validation(mla):
     assert lib.mla_prefill_attn(*args(FAKE, need, n=16385)) == 2     # beyond the plan's limit
 
 
-def test_wait_selftest_validates_arguments(mla):
+def test_wait_selftest_validates_arguments(host_only):
+    mla = host_only
     """Host-side checks of the bounded-wait self-test (no launch, no GPU needed)."""
     import ctypes
     lib = ctypes.CDLL(mla.LIB_PATH)
@@ -129,3 +145,21 @@ def test_wait_selftest_validates_arguments(mla):
     assert lib.mla_selftest_wait_timeout(0, bogus, None) == 1           # MLA_ERR_INVALID_ARG
     assert lib.mla_selftest_wait_timeout(2000001, bogus, None) == 1
     assert lib.mla_selftest_wait_timeout(1000, None, None) == 1
+
+
+def test_noalloc_scratch_size_and_refusal(host_only):
+    """The static buffer's size as the header states it, as the library reports it and as the binding
+    uses it agree; a problem whose partials exceed it is refused before any device call."""
+    mla = host_only
+    src = open(os.path.join(ROOT, "include", "mla.h")).read()
+    m = re.search(r"#define\s+MLA_NOALLOC_SCRATCH_BYTES\s+\(([^)]*)\)", src)
+    header_bytes = eval(m.group(1).replace("u", ""))   # e.g. "48u * 1024u * 1024u"
+    assert header_bytes == mla.lib.mla_noalloc_scratch_bytes() == mla.NOALLOC_SCRATCH_BYTES
+    d = mla.contiguous_desc(4, 131072)
+    assert mla.decode_workspace_size(4, 131072, 1024) > mla.NOALLOC_SCRATCH_BYTES
+    rc = mla.lib.mla_decode_attn_noalloc(FAKE, FAKE, None, FAKE, d, 4, ctypes.c_float(0.07), 1024, FAKE, None, None)
+    assert rc == 3   # MLA_ERR_WORKSPACE
+    assert mla.lib.mla_decode_attn_noalloc(FAKE, FAKE, None, FAKE, d, -1, ctypes.c_float(0.07), 0, FAKE, None,
+                                           None) == 1
+    assert mla.lib.mla_decode_attn_noalloc(FAKE, FAKE, None, FAKE, d, 0, ctypes.c_float(0.07), 0, FAKE, None,
+                                           None) == 0   # empty batch: a no-op
