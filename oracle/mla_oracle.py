@@ -29,6 +29,13 @@ Readings where the pages are silent:
     plain linear projection W^KR h_t (the pages draw the branch h_t -> k^R without naming its
     matrix), rotated by RoPE before it is cached.
 
+  * FP8 latent cache ([DR] §4.2 效率证据 reports FP8 serving with the KV cache at about 6 bits per
+    element, without a format): each cached row (the 576 values [c | RoPE(k^R)], taken before any
+    bf16 rounding) is stored as 576 OCP E4M3 codes plus one fp32 scale per token, s = amax / 448
+    (amax the row's largest magnitude; s = 1 for an all-zero row); a value x is coded as the E4M3
+    value nearest (ties to even, saturating at +-448) to the fp32 rounding of x / s; it decodes
+    to code_value * s.
+
 Pins: every function here is checked by ``tests/test_oracle_pins.py`` against values that
 do not come from this file (closed forms, library routines, brute-force scalar loops,
 invariants).  No function is "parity unpinned".
@@ -296,3 +303,71 @@ def decode_step(q_nope, q_pe, cs, krs_raw, w_uk, w_uv, scale, base=ROPE_BASE,
             qa = r["q_abs"]
         outs.append(r["out"]); lats.append(r["out_lat"]); lses.append(r["lse"]); qas.append(qa)
     return dict(out=np.stack(outs), out_lat=np.stack(lats), lse=np.stack(lses), q_abs=np.stack(qas))
+
+
+# ----------------------------------------------------------------------------------------
+# FP8 (E4M3) latent cache ([DR] §4.2: FP8 serving, KV cache at about 6 bits per element).
+# E4M3 (OCP 8-bit floating point, E4M3 variant): 1 sign bit, 4 exponent bits with bias 7,
+# 3 mantissa bits; exponent field 0 holds the subnormals m * 2^-9; no infinities; the largest
+# finite magnitude is 1.75 * 2^8 = 448 (exponent field 15, mantissa 6); field 15 with mantissa 7
+# is NaN.
+# ----------------------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each E4M3 code (uint8) in float64, from the bit fields."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_encode_rne(v) -> np.ndarray:
+    """The E4M3 code of each float32 value: round to the nearest representable magnitude, ties to
+    the even mantissa, magnitudes at or beyond 448 saturate to 448; the sign is kept (also for
+    zero).  NaN inputs are not handled."""
+    v = np.asarray(v, dtype=np.float32).astype(np.float64)
+    a = np.abs(v)
+    sat = a >= E4M3_MAX
+    # quantum of the binade: 2^(E - 3) for a in [2^E, 2^(E+1)), E >= -6; 2^-9 below 2^-6
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))          # a = f * 2^ex, f in [0.5, 1)
+    E = np.maximum(ex - 1, -6)
+    q = np.exp2(E - 3.0)
+    n = np.rint(a / q)                                 # a / q is exact (q a power of two); rint is ties-to-even
+    mag = np.where(sat, E4M3_MAX, n * q)
+    # code of a representable magnitude: exponent field and mantissa from the value
+    _, ex2 = np.frexp(np.where(mag > 0, mag, 1.0))
+    E2 = ex2 - 1
+    normal = mag >= 2.0 ** -6
+    efield = np.where(normal, E2 + 7, 0)
+    mfield = np.where(normal, np.rint((mag / np.exp2(E2) - 1.0) * 8.0), np.rint(mag / 2.0 ** -9))
+    code = (efield.astype(np.int64) << 3) | mfield.astype(np.int64)
+    code = np.where(mag == 0, 0, code)
+    return (code | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
+
+
+def quantize_rows(rows):
+    """Per-token FP8 rows: rows [n, w] (values in any precision) -> (codes uint8 [n, w], scales fp32 [n]).
+
+    s_t = fp32(amax_t / 448) (1 for an all-zero row); code = E4M3 RNE of fp32(x / s_t), the division
+    done in fp64 and rounded once to fp32."""
+    r = np.asarray(rows, dtype=np.float64)
+    amax = np.max(np.abs(r), axis=-1)
+    s = np.where(amax > 0, amax / E4M3_MAX, 1.0).astype(np.float32)
+    v = (r / s.astype(np.float64)[..., None]).astype(np.float32)
+    return e4m3_encode_rne(v), s
+
+
+def dequantize_rows(codes, scales) -> np.ndarray:
+    """code value * scale, in float64."""
+    return e4m3_decode(codes) * np.asarray(scales, np.float64)[..., None]
+
+
+def fp8_cache_rows(c, kr_raw, pos, base: float = ROPE_BASE):
+    """The FP8 cached row of a token: the row [c^KV | RoPE(k^R, pos)] (fp64 rotation, no bf16 step)
+    quantized per token."""
+    return quantize_rows(cache_rows(c, kr_raw, pos, base))

@@ -610,3 +610,150 @@ def test_pins_catch_planted_decode_step_mistakes():
 
     for bad in (keys_one_late, keys_unrotated, query_unrotated, query_at_length, query_negated_angle):
         assert _fails(check_decode_step_positions, bad), bad.__name__
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) latent cache
+# 《DeepSeek-V2》深度解读报告 §4.2 效率证据: FP8 serving with the KV cache at about 6 bits per element.
+# The format pinned here is OCP E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits,
+# subnormals m * 2^-9, largest finite 448, S.1111.111 NaN, no infinities).
+E4M3_ANCHORS = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x0F: 1.875 * 2.0 ** -6,
+                0x38: 1.0, 0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0x48: 4.0, 0x77: 240.0, 0x78: 256.0,
+                0x7E: 448.0, 0x80: -0.0, 0xB8: -1.0, 0xFE: -448.0}
+
+
+def check_e4m3_decode(e4m3_decode):
+    codes = np.array(list(E4M3_ANCHORS), dtype=np.uint8)
+    got = e4m3_decode(codes)
+    for c, g in zip(codes, got):
+        assert g == E4M3_ANCHORS[int(c)] and math.copysign(1, g) == math.copysign(1, E4M3_ANCHORS[int(c)]), hex(c)
+    assert np.isnan(e4m3_decode(np.array([0x7F, 0xFF], np.uint8))).all()
+    assert not np.isnan(e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))).any()
+
+
+def bf_e4m3_nearest(v):
+    """Brute force: the non-negative finite code whose value (from the anchors' rule written out
+    as scalar arithmetic) is nearest to |v|, ties to the even code, 448 for |v| >= 448; sign bit
+    from v."""
+    a = abs(float(v))
+    best, bestd = None, None
+    for c in range(0x7F):
+        e, m = c >> 3, c & 7
+        val = m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+        d = abs(val - a)
+        if best is None or d < bestd or (d == bestd and c % 2 == 0):
+            best, bestd = c, d
+    if a >= 448.0:
+        best = 0x7E
+    return best | (0x80 if math.copysign(1, float(v)) < 0 else 0)
+
+
+def check_e4m3_encode(e4m3_encode_rne, e4m3_decode):
+    # every finite code round-trips
+    codes = np.arange(256, dtype=np.uint8)
+    vals = e4m3_decode(codes)
+    fin = ~np.isnan(vals)
+    assert np.array_equal(e4m3_encode_rne(vals[fin].astype(np.float32)), codes[fin])
+    # exact midpoints between neighbours, just above and below them, saturation, tiny values
+    pos = np.sort(np.unique(np.abs(vals[fin])))
+    mids = (pos[:-1] + pos[1:]) / 2
+    rng = np.random.default_rng(71)
+    probe = np.concatenate([mids, np.nextafter(mids.astype(np.float32), np.float32(0)),
+                            np.nextafter(mids.astype(np.float32), np.float32(1000)),
+                            [448.0, 460.0, 479.99, 480.0, 1e6, 2.0 ** -10, 2.0 ** -11, 1e-30, 0.0],
+                            rng.standard_normal(300) * 3, rng.standard_normal(100) * 200]).astype(np.float32)
+    probe = np.concatenate([probe, -probe])
+    got = e4m3_encode_rne(probe)
+    want = np.array([bf_e4m3_nearest(x) for x in probe], dtype=np.uint8)
+    assert np.array_equal(got, want), probe[got != want][:5]
+
+
+def check_quantize_rows(quantize_rows, e4m3_decode):
+    rng = np.random.default_rng(72)
+    rows = rng.standard_normal((6, 576)) * np.array([1, 0.01, 100, 3, 1e-3, 1])[:, None]
+    codes, s = quantize_rows(rows)
+    assert codes.dtype == np.uint8 and codes.shape == rows.shape and s.dtype == np.float32
+    amax = np.abs(rows).max(axis=1)
+    assert np.array_equal(s, (amax / 448.0).astype(np.float32))                   # the scale from the row max
+    top = np.abs(rows).argmax(axis=1)
+    assert all((codes[i, top[i]] & 0x7F) == 0x7E for i in range(6))               # the max codes to 448
+    xh = e4m3_decode(codes) * s.astype(np.float64)[:, None]
+    bound = 2.0 ** -4 * np.abs(rows) + 2.0 ** -10 * s.astype(np.float64)[:, None]   # half a step: normal / subnormal
+    assert (np.abs(xh - rows) <= bound * (1 + 1e-6)).all()
+    assert np.array_equal(np.sign(xh[xh != 0]), np.sign(rows[xh != 0]))
+    # rows of representable values times a power of two come back exactly, scale included
+    k = rng.integers(0, 0x7E, size=(3, 576)).astype(np.uint8)
+    k[:, 5] = 0x7E
+    vals = e4m3_decode(k) * (2.0 ** np.array([-3.0, 0.0, 5.0]))[:, None]
+    c2, s2 = quantize_rows(vals)
+    assert np.array_equal(c2, k) and np.array_equal(s2, np.float32([2.0 ** -3, 1.0, 2.0 ** 5]))
+    # sign symmetry and the all-zero row
+    c3, s3 = quantize_rows(-rows)
+    assert np.array_equal(c3, codes ^ 0x80) and np.array_equal(s3, s)
+    c4, s4 = quantize_rows(np.zeros((1, 576)))
+    assert not c4.any() and s4[0] == 1.0
+
+
+def test_e4m3_and_fp8_quantizer_pins():
+    check_e4m3_decode(oracle.e4m3_decode)
+    check_e4m3_encode(oracle.e4m3_encode_rne, oracle.e4m3_decode)
+    check_quantize_rows(oracle.quantize_rows, oracle.e4m3_decode)
+
+
+def test_fp8_cache_rows_pin():
+    """fp8_cache_rows quantizes the fp64 row [c | RoPE(k^R, pos)]: checked against the scalar-loop
+    rotation and the brute-force nearest code, element by element."""
+    rng = np.random.default_rng(73)
+    c = rng.standard_normal((3, 8))
+    kr = rng.standard_normal((3, 4)) * 3
+    pos = [0, 5, 1000]
+    codes, s = oracle.fp8_cache_rows(c, kr, pos)
+    for t in range(3):
+        row = list(c[t]) + list(bf_rotate(kr[t], pos[t]))
+        amax = max(abs(x) for x in row)
+        st = np.float32(amax / 448.0)
+        assert s[t] == st
+        want = [bf_e4m3_nearest(np.float32(x / float(st))) for x in row]
+        assert list(codes[t]) == want
+
+
+def test_pins_catch_planted_fp8_mistakes():
+    def truncating(v):                       # rounds toward zero instead of to nearest
+        v = np.asarray(v, np.float32)
+        out = oracle.e4m3_encode_rne(v)
+        dec = oracle.e4m3_decode(out)
+        over = np.abs(dec) > np.abs(v.astype(np.float64))
+        return np.where(over & ((out & 0x7F) > 0), out - 1, out).astype(np.uint8)
+
+    def ties_away(v):                        # ties away from zero
+        v = np.asarray(v, np.float32).astype(np.float64)
+        a = np.abs(v)
+        _, ex = np.frexp(np.where(a > 0, a, 1.0))
+        q = np.exp2(np.maximum(ex - 1, -6) - 3.0)
+        mag = np.minimum(np.floor(a / q + 0.5) * q, 448.0)
+        return oracle.e4m3_encode_rne(np.copysign(mag, v).astype(np.float32))
+
+    def no_saturation(v):                    # wraps past 448 into the NaN code
+        out = oracle.e4m3_encode_rne(v)
+        big = np.abs(np.asarray(v, np.float32)) >= 480
+        return np.where(big, out | 0x7F, out).astype(np.uint8)
+
+    for bad in (truncating, ties_away, no_saturation):
+        assert _fails(check_e4m3_encode, bad, oracle.e4m3_decode), bad.__name__
+
+    def bias_six(codes):                     # exponent bias 6 instead of 7
+        return oracle.e4m3_decode(codes) * 2.0
+
+    assert _fails(check_e4m3_decode, bias_six)
+
+    def scale_from_240(rows):                # the E4M3-FNUZ maximum instead of 448
+        r = np.asarray(rows, np.float64)
+        s = (np.abs(r).max(axis=-1) / 240.0).astype(np.float32)
+        return oracle.e4m3_encode_rne((r / s.astype(np.float64)[..., None]).astype(np.float32)), s
+
+    def scale_from_mean(rows):               # the row's mean magnitude instead of its max
+        r = np.asarray(rows, np.float64)
+        s = (np.abs(r).mean(axis=-1) / 448.0 * 8).astype(np.float32)
+        return oracle.e4m3_encode_rne((r / s.astype(np.float64)[..., None]).astype(np.float32)), s
+
+    for bad in (scale_from_240, scale_from_mean):
+        assert _fails(check_quantize_rows, bad, oracle.e4m3_decode), bad.__name__
