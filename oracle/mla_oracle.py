@@ -31,10 +31,11 @@ Readings where the pages are silent:
 
   * FP8 latent cache ([DR] §4.2 效率证据 reports FP8 serving with the KV cache at about 6 bits per
     element, without a format): each cached row (the 576 values [c | RoPE(k^R)], taken before any
-    bf16 rounding) is stored as 576 OCP E4M3 codes plus one fp32 scale per token, s = amax / 448
-    (amax the row's largest magnitude; s = 1 for an all-zero row); a value x is coded as the E4M3
-    value nearest (ties to even, saturating at +-448) to the fp32 rounding of x / s; it decodes
-    to code_value * s.
+    bf16 rounding) is stored as 576 OCP E4M3 codes plus one scale per token, the power of two
+    s = 2^k with k the smallest integer for which amax <= 448 * 2^k (amax the row's largest
+    magnitude; s = 1 for an all-zero row); a value x is coded as the E4M3 value nearest (ties to
+    even, saturating at +-448) to the fp32 rounding of x / s, and decodes to code_value * s, which
+    a power-of-two scale keeps exact in bf16 and fp32.
 
 Pins: every function here is checked by ``tests/test_oracle_pins.py`` against values that
 do not come from this file (closed forms, library routines, brute-force scalar loops,
@@ -350,14 +351,24 @@ def e4m3_encode_rne(v) -> np.ndarray:
     return (code | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
 
 
+def fp8_row_scale(amax):
+    """The per-token scale: the power of two 2^k with k the smallest integer such that
+    amax <= 448 * 2^k (1 for amax = 0).  Float32."""
+    a = np.asarray(amax, dtype=np.float64)
+    _, e = np.frexp(np.where(a > 0, a / E4M3_MAX, 1.0))      # a / 448 = f 2^e, f in [0.5, 1)
+    k = e.astype(np.int64)                                   # 2^e >= a / 448 > 2^(e-1) up to the division's rounding
+    k = np.where(a > E4M3_MAX * np.exp2(k), k + 1, k)        # settle k by exact comparisons with 448 * 2^k
+    k = np.where(a <= E4M3_MAX * np.exp2(k - 1), k - 1, k)
+    return np.where(a > 0, np.exp2(k), 1.0).astype(np.float32)
+
+
 def quantize_rows(rows):
     """Per-token FP8 rows: rows [n, w] (values in any precision) -> (codes uint8 [n, w], scales fp32 [n]).
 
-    s_t = fp32(amax_t / 448) (1 for an all-zero row); code = E4M3 RNE of fp32(x / s_t), the division
-    done in fp64 and rounded once to fp32."""
+    s_t = fp8_row_scale(amax_t); code = E4M3 RNE of fp32(x / s_t) (x / s_t is exact: s_t is a power
+    of two)."""
     r = np.asarray(rows, dtype=np.float64)
-    amax = np.max(np.abs(r), axis=-1)
-    s = np.where(amax > 0, amax / E4M3_MAX, 1.0).astype(np.float32)
+    s = fp8_row_scale(np.max(np.abs(r), axis=-1))
     v = (r / s.astype(np.float64)[..., None]).astype(np.float32)
     return e4m3_encode_rne(v), s
 

@@ -667,18 +667,30 @@ def check_e4m3_encode(e4m3_encode_rne, e4m3_decode):
     assert np.array_equal(got, want), probe[got != want][:5]
 
 
+def bf_pow2_scale(amax):
+    """Brute force: the smallest power of two p (as 2^k, k an integer) with amax <= 448 p."""
+    if amax == 0:
+        return 1.0
+    k = -200
+    while amax > 448.0 * 2.0 ** k:
+        k += 1
+    return 2.0 ** k
+
+
 def check_quantize_rows(quantize_rows, e4m3_decode):
     rng = np.random.default_rng(72)
     rows = rng.standard_normal((6, 576)) * np.array([1, 0.01, 100, 3, 1e-3, 1])[:, None]
+    rows[5, 7] = 448.0 * 2.0 ** -2                                               # amax exactly 448 * 2^k
     codes, s = quantize_rows(rows)
     assert codes.dtype == np.uint8 and codes.shape == rows.shape and s.dtype == np.float32
     amax = np.abs(rows).max(axis=1)
-    assert np.array_equal(s, (amax / 448.0).astype(np.float32))                   # the scale from the row max
+    assert [float(x) for x in s] == [bf_pow2_scale(float(a)) for a in amax]      # power-of-two scale from the row max
     top = np.abs(rows).argmax(axis=1)
-    assert all((codes[i, top[i]] & 0x7F) == 0x7E for i in range(6))               # the max codes to 448
+    assert all(0x76 <= (codes[i, top[i]] & 0x7F) <= 0x7E for i in range(6))     # the max codes into (224, 448]
+    assert (codes[5, 7] & 0x7F) == 0x7E
     xh = e4m3_decode(codes) * s.astype(np.float64)[:, None]
     bound = 2.0 ** -4 * np.abs(rows) + 2.0 ** -10 * s.astype(np.float64)[:, None]   # half a step: normal / subnormal
-    assert (np.abs(xh - rows) <= bound * (1 + 1e-6)).all()
+    assert (np.abs(xh - rows) <= bound * (1 + 1e-12)).all()
     assert np.array_equal(np.sign(xh[xh != 0]), np.sign(rows[xh != 0]))
     # rows of representable values times a power of two come back exactly, scale included
     k = rng.integers(0, 0x7E, size=(3, 576)).astype(np.uint8)
@@ -686,6 +698,9 @@ def check_quantize_rows(quantize_rows, e4m3_decode):
     vals = e4m3_decode(k) * (2.0 ** np.array([-3.0, 0.0, 5.0]))[:, None]
     c2, s2 = quantize_rows(vals)
     assert np.array_equal(c2, k) and np.array_equal(s2, np.float32([2.0 ** -3, 1.0, 2.0 ** 5]))
+    # a code times its scale is exact in bf16 (8 significant bits): decoded values have <= 4
+    dec = (e4m3_decode(codes) * s.astype(np.float64)[:, None]).astype(np.float32)
+    assert np.array_equal(dec.view(np.uint32) & 0xFFFF, np.zeros_like(dec.view(np.uint32)))
     # sign symmetry and the all-zero row
     c3, s3 = quantize_rows(-rows)
     assert np.array_equal(c3, codes ^ 0x80) and np.array_equal(s3, s)
@@ -709,8 +724,7 @@ def test_fp8_cache_rows_pin():
     codes, s = oracle.fp8_cache_rows(c, kr, pos)
     for t in range(3):
         row = list(c[t]) + list(bf_rotate(kr[t], pos[t]))
-        amax = max(abs(x) for x in row)
-        st = np.float32(amax / 448.0)
+        st = bf_pow2_scale(max(abs(x) for x in row))
         assert s[t] == st
         want = [bf_e4m3_nearest(np.float32(x / float(st))) for x in row]
         assert list(codes[t]) == want
@@ -747,13 +761,14 @@ def test_pins_catch_planted_fp8_mistakes():
 
     def scale_from_240(rows):                # the E4M3-FNUZ maximum instead of 448
         r = np.asarray(rows, np.float64)
-        s = (np.abs(r).max(axis=-1) / 240.0).astype(np.float32)
+        s = np.exp2(np.ceil(np.log2(np.maximum(np.abs(r).max(axis=-1), 1e-300) / 240.0))).astype(np.float32)
         return oracle.e4m3_encode_rne((r / s.astype(np.float64)[..., None]).astype(np.float32)), s
 
-    def scale_from_mean(rows):               # the row's mean magnitude instead of its max
+    def scale_not_pow2(rows):                # amax / 448 itself
         r = np.asarray(rows, np.float64)
-        s = (np.abs(r).mean(axis=-1) / 448.0 * 8).astype(np.float32)
+        s = (np.abs(r).max(axis=-1) / 448.0).astype(np.float32)
+        s = np.where(s > 0, s, 1).astype(np.float32)
         return oracle.e4m3_encode_rne((r / s.astype(np.float64)[..., None]).astype(np.float32)), s
 
-    for bad in (scale_from_240, scale_from_mean):
+    for bad in (scale_from_240, scale_not_pow2):
         assert _fails(check_quantize_rows, bad, oracle.e4m3_decode), bad.__name__
