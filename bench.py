@@ -1,6 +1,7 @@
 """Benchmark of one MLA decode step (append -> absorb -> decode attention -> un-absorb).
 
-python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--splits P]
+                [--extra-workloads A,B,...] [--impl ours|reference]
 
 A step is one pass of the whole hot path over one batch of synthetic input: append the batch's
 new token (RoPE on k^R) into the latent cache, absorb W_UK into the queries, split-KV decode
@@ -10,6 +11,14 @@ device time).  Inputs are resident in HBM before the timed region; the caches ar
 between steps (several copies, together larger than the 126 MB L2) so no step reads a cache
 the previous step left in L2.  N > 1 runs independent replicas (weak scaling): the decode of
 disjoint batches needs no data exchange.
+
+The headline workload is batch 128 with lengths uniform in [1024, 8192] over a 64-token paged
+cache at permuted physical blocks (the B = 128, ~4K-context decode class).  The timed region is
+K steps, bracketed by a barrier and a device synchronisation on both sides; when K steps last
+less than MIN_TIMED_S, further K-step brackets follow back to back until the brackets together
+last that long, so the clock samples come from timed work, and the reported time per step is
+the total device time of all brackets over all their steps.  The other workloads are measured
+the same way in the same run and reported under `by_workload`.
 """
 from __future__ import annotations
 
@@ -35,7 +44,11 @@ ROW_BYTES = 576 * 2
 FLOP_PER_TOKEN = 2 * 128 * 576 + 2 * 128 * 512          # QK^T over [c|k_R] plus P.V over c
 GEMM_FLOP_PER_SEQ = 2 * (2 * 128 * 128 * 512)           # absorb + un-absorb
 L2_BYTES = 126 * 1024 * 1024
-DEFAULT_WORKLOAD = "b32_l4096"
+DEFAULT_WORKLOAD = "b128_u1024_8192_paged"
+# measured after the headline in the same run (name, forced work ranges or 0 for the auto plan)
+DEFAULT_EXTRAS = "b32_l4096,b4_l131072@512,l60_b256_log64_32768_paged"
+MIN_TIMED_S = 1.0
+NOMINAL_HBM_GBS, NOMINAL_BF16_TFLOPS = 8000.0, 2250.0   # B200 data-sheet figures (context)
 
 
 def load_peaks():
@@ -127,31 +140,47 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------- oracle
-def time_oracle(lens, budget_tokens=4096, seed=4242):
-    """The fp64 oracle (explicit form, as it stands) on one sequence of the workload's first
-    length, truncated to `budget_tokens` tokens.  Returns (tokens, seconds)."""
+def time_oracle(lens, budget_tokens=8192, seed=4242, form="explicit", index=0):
+    """The fp64 oracle, as it stands, on one sequence of the workload: length lens[index]
+    (truncated to `budget_tokens`), `form` = "explicit" (per-head K and V decompressed, textbook
+    softmax) or "absorbed" (W_UK folded into the query, W_UV after attention).  Returns
+    (tokens, seconds)."""
     import oracle
-    L = int(min(int(lens[0]), budget_tokens))
+    L = int(min(int(lens[index % len(lens)]), budget_tokens))
     b = mi.decode_batch(seed, [L])
     w = mi.layer_weights(seed + 1)
     f = mi.bf16_to_f64
     args = (f(b.q_nope), f(b.q_pe), [f(x) for x in b.c], [f(x) for x in b.kr], f(w.w_uk), f(w.w_uv),
             1.0 / math.sqrt(192.0))
     t0 = time.perf_counter()
-    oracle.decode_step(*args, form="explicit")
+    oracle.decode_step(*args, q_pos=[L - 1], form=form)
     dt = time.perf_counter() - t0
     return L, dt
 
 
-def time_oracle_sample(lens, min_seconds=12.0, max_seqs=64):
-    """Bounded CPU baseline: sequences of the workload (first length, at most 4096 tokens each,
-    distinct seeds) through the oracle until about `min_seconds` of work.  Returns
+def time_oracle_sample(lens, min_seconds=12.0, max_seqs=64, form="explicit"):
+    """Bounded CPU baseline: sequences of the workload in its own order (each truncated to 8192
+    tokens, distinct seeds) through the oracle until about `min_seconds` of work.  Returns
     (tokens, seconds, sequences)."""
     tok, secs, n = 0, 0.0, 0
     while n < max_seqs and (n == 0 or secs < min_seconds):
-        L, dt = time_oracle(lens, seed=4242 + n)
+        L, dt = time_oracle(lens, seed=4242 + n, form=form, index=n)
         tok, secs, n = tok + L, secs + dt, n + 1
     return tok, secs, n
+
+
+def time_oracle_layers(lens, n_layers, n_seqs=8, n_sample_layers=2):
+    """The whole-model workload's CPU sample: `n_sample_layers` layers x the first `n_seqs`
+    sequences (full lengths) through the absorbed fp64 oracle, each layer with its own seeded
+    weights and inputs, extrapolated to all layers and sequences of a step by cached tokens.
+    Returns (sampled tokens, seconds, extrapolated seconds per step)."""
+    tok, secs = 0, 0.0
+    for layer in range(n_sample_layers):
+        for i in range(n_seqs):
+            L, dt = time_oracle(lens, budget_tokens=1 << 30, seed=8000 + 97 * layer + i, form="absorbed", index=i)
+            tok, secs = tok + L, secs + dt
+    step_tokens = int(np.sum(lens)) * n_layers
+    return tok, secs, secs * step_tokens / max(tok, 1)
 
 
 def cpu_threads():
@@ -171,12 +200,13 @@ def run_reference(args, rank, world):
         time_oracle(lens, budget_tokens=256)
     tok, secs = 0, 0.0
     for i in range(args.steps):
-        L, dt = time_oracle(lens, seed=4242 + i)
+        L, dt = time_oracle(lens, seed=4242 + i, index=i)
         tok += L
         secs += dt
     gbs = tok * ROW_BYTES / secs / 1e9
     threads, cores = cpu_threads()
-    sample = f"{args.steps} steps x one sequence of {L} tokens (explicit fp64 form), extrapolated per cached token"
+    sample = (f"{args.steps} steps, each one sequence of the workload in its order ({tok} cached tokens in all, "
+              f"each at most 8192; explicit fp64 form), GB/s of cached rows processed")
     line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -242,7 +272,7 @@ def _layer_on_device(name, layer, device, chunk_tokens=1 << 18):
                 w_uv=normal((128, 512, 128), 1 / math.sqrt(512)), host=None, dev=dev)
 
 
-def setup_replica(name, device):
+def setup_replica(name, device, splits=0):
     import torch
     import mla_latent_kv_20_b200 as m
     w, lens = workload_shape(name)
@@ -262,7 +292,7 @@ def setup_replica(name, device):
         layers = [_layer_on_device(name, l, device) for l in range(n_layers)]
     last = np.asarray(lens, np.int32) - 1
     base = layers[0]["caches"][0]
-    splits = 0   # the auto work plan (ranges = resident CTA pairs)
+    # splits = 0: the auto work plan (ranges = resident CTA pairs); else that many forced ranges
     ws_bytes = m.decode_workspace_size(B, base.capacity(), splits)
     st = dict(B=B, lens=lens, w=w, layers=layers, splits=splits,
               n_splits=m.decode_num_splits(B, base.capacity(), splits),
@@ -296,14 +326,12 @@ def traffic_sources_digest():
     return h.hexdigest()
 
 
-def recorded_traffic(workload):
-    rec = MEASURED_TRAFFIC.get(workload)
+def recorded_traffic(workload, splits=0):
+    rec = MEASURED_TRAFFIC.get(workload if not splits else f"{workload}@{splits}")
     if rec is None or rec["sha256"] != traffic_sources_digest():
         return None
     return rec["bytes"]
 
-
-CLOCK_WINDOW_S = 1.0     # clock-sampling replay window when the timed region is too short to sample
 
 LAUNCHES_PER_LAYER = 4   # append + absorb GEMM (with the q_pe rotation), decode ranges, combine, un-absorb GEMM
 
@@ -571,20 +599,48 @@ def hz_bits(t):
     return hz.bf16_bits(t)
 
 
-def run_ours(args, rank, world, local_rank):
+def partial_segments(lens, P):
+    """Range partials one decode call writes (and its combine reads back) under the work plan:
+    with the per-sequence plan (every non-empty sequence has at least T/P of the T tiles) sequence
+    b gets r_b = min(floor(P tiles_b / T), tiles_b) ranges and contributes r_b partials when r_b > 1;
+    otherwise the tiles are laid end to end and range p takes [floor(pT/P), floor((p+1)T/P)),
+    and every range that does not cover the whole of a sequence it meets writes a partial of
+    that sequence.  Used only to report the partials' bytes."""
+    tiles = [(int(L) + 127) // 128 for L in lens]
+    T = sum(tiles)
+    if T == 0:
+        return 0
+    nz = [t for t in tiles if t > 0]
+    if min(nz) * P >= T:
+        n = 0
+        for t in nz:
+            r = min(P * t // T, t)
+            n += r if r > 1 else 0
+        return n
+    n, run = 0, 0
+    starts = [p * T // P for p in range(P + 1)]
+    for t in tiles:
+        if t == 0:
+            continue
+        first = next(p for p in range(P) if starts[p] <= run < starts[p + 1])
+        last = next(p for p in range(P) if starts[p] <= run + t - 1 < starts[p + 1])
+        if last > first:
+            n += last - first + 1
+        run += t
+    return n
+
+
+PARTIAL_BYTES = 128 * (512 + 2) * 4    # one range partial of one sequence: fp32 O rows, m and l of 128 heads
+
+
+def measure_workload(name, splits, args, world, dev, barrier):
+    """Set up one replica of a workload, time its step, its phases and its end-to-end loop.
+    Returns the raw per-rank numbers and the facts of the workload (nothing reduced yet)."""
     import torch
-    import torch.distributed as dist
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
     import mla_latent_kv_20_b200 as m
-    st = setup_replica(args.workload, dev)
+    st = setup_replica(name, dev, splits)
     torch.cuda.synchronize()
     assert m.get_device_error() == 0
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
     for i in range(args.warmup):
         run_step(st, i)
     torch.cuda.synchronize()
@@ -608,39 +664,37 @@ def run_ours(args, rank, world, local_rank):
     for i in range(args.warmup):
         step_graphs[i % n_rot].replay()
     torch.cuda.synchronize()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local_rank)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
     sampler.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
+    # K-step brackets, each between a barrier and a synchronisation on both sides, back to back
+    # until they add up to MIN_TIMED_S of device time (every rank runs the same number: rank 0's
+    # count is broadcast through the max-over-ranks reduction of a flag after each bracket).
+    total_ms, brackets, host_ms = 0.0, 0, 0.0
     m0 = time.monotonic()
-    t_start.record()
-    h0 = time.perf_counter()
-    for i in range(args.steps):
-        step_graphs[i % n_rot].replay()
-    host_ms = (time.perf_counter() - h0) * 1e3 / args.steps
-    t_end.record()
-    torch.cuda.synchronize()
-    m1 = time.monotonic()
-    barrier()
-    ms = t_start.elapsed_time(t_end) / args.steps
-    clocks = sampler.summary(m0, m1)
-    clocks["window"] = "timed region (%.1f ms)" % ((m1 - m0) * 1e3)
-    if clocks["samples"] < 5:
-        # The timed region is shorter than the sampler's resolution: the same step graphs replay
-        # for another ~CLOCK_WINDOW_S seconds right after it, untimed, and the clocks of that window
-        # stand for the load of the timed region.
-        n_win = max(1, int(CLOCK_WINDOW_S / max(ms * 1e-3, 1e-6)))
-        w0 = time.monotonic()
-        for i in range(n_win):
-            step_graphs[i % n_rot].replay()
+    while True:
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
         torch.cuda.synchronize()
-        w1 = time.monotonic()
-        clocks = sampler.summary(w0, w1)
-        clocks["window"] = ("%d replays of the timed step right after the timed region (%.2f s; the timed "
-                            "region itself lasted %.1f ms)" % (n_win, w1 - w0, (m1 - m0) * 1e3))
+        t_start.record()
+        h0 = time.perf_counter()
+        for i in range(args.steps):
+            step_graphs[(brackets * args.steps + i) % n_rot].replay()
+        host_ms += (time.perf_counter() - h0) * 1e3
+        t_end.record()
+        torch.cuda.synchronize()
+        barrier()
+        total_ms += t_start.elapsed_time(t_end)
+        brackets += 1
+        more = 1.0 if (total_ms < args.min_timed_s * 1e3 and brackets < 100000) else 0.0
+        if reduce_max_over_ranks([more], world, device=dev)[0] == 0.0:
+            break
+    m1 = time.monotonic()
     sampler.stop()
+    ms = total_ms / (brackets * args.steps)
+    clocks = sampler.summary(m0, m1)
+    clocks["window"] = "timed region: %d bracket%s of %d steps (%.2f s)" % (
+        brackets, "" if brackets == 1 else "s", args.steps, m1 - m0)
     # per-phase timing loop
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(len(GRAPH_PHASES) + 1)] for _ in range(n_layers)]
            for _ in range(args.steps)]
@@ -742,58 +796,148 @@ def run_ours(args, rank, world, local_rank):
     rt.destroy(in_ready + step_done + out_read)
     assert m.get_device_error() == 0
     assert np.array_equal(hz_bits(out_host[(args.steps - 1) % 2]), hz_bits(st["out"]))   # the read-back is the result
+    return dict(st=st, n_layers=n_layers, ms=ms, e2e_ms=e2e_ms, dec_ms=dec_ms, phase_ms=phase_ms, clocks=clocks,
+                host_ms=host_ms / (brackets * args.steps), brackets=brackets, h2d=h2d, d2h=d2h)
 
-    next_rows = {"project_append": measure_project_append(st, args.steps, args.warmup),
-                 "output_proj": measure_output_proj(st, args.steps, args.warmup),
-                 "prefill": measure_prefill(args.steps, args.warmup)}
-    ms, e2e_ms, dec_ms = reduce_max_over_ranks([ms, e2e_ms, dec_ms], world, device=dev)
-    if rank != 0:
-        return
+
+def summarize(name, splits, r, world, peaks):
+    """The reported numbers of one measured workload (times already reduced over ranks)."""
+    st, n_layers = r["st"], r["n_layers"]
+    hbm, tc, tc_sus, peak_kind = peaks
     tokens, cache_bytes, flops, dec_bytes = step_work(st["lens"])
-    tokens, cache_bytes, flops = tokens * n_layers, cache_bytes * n_layers, flops * n_layers
-    hbm, tc, tc_sus, peak_kind = load_peaks()
-    value = job_throughput(cache_bytes, world, ms)
+    step_tokens, step_bytes, step_flops = tokens * n_layers, cache_bytes * n_layers, flops * n_layers
+    ms, e2e_ms, dec_ms = r["ms"], r["e2e_ms"], r["dec_ms"]
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
-    roofline_s = max(cache_bytes / (hbm * 1e9), flops / (tc * 1e12))
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) latents/keys/queries, "
-                                                     "N(0,1/512) weights)",
-        "config": {"workload": args.workload, "batch": st["B"], "seq_len": int(np.max(st["lens"])),
-                   "layers": n_layers, "tokens_per_layer": tokens // n_layers, "paged": bool(st["w"]["paged"]),
-                   "work_ranges": st["n_splits"],
-                   "l2": "inputs larger than L2: %d cache cop%s rotated, %.0f MB each" % (
-                       len(st["layers"][0]["caches"]) * n_layers, "y" if n_layers * len(st["layers"][0]["caches"]) == 1 else "ies",
-                       cache_bytes / n_layers / 1e6),
-                   "parallelism": f"replicas x{world}"},
-        "tflops": world * flops / (ms * 1e-3) / 1e12,
+    dec_flops = tokens * FLOP_PER_TOKEN
+    roofline_s = max(step_bytes / (hbm * 1e9), step_flops / (tc * 1e12))
+    n_part = partial_segments(st["lens"], st["n_splits"])
+    cfg = {"workload": name, "batch": st["B"], "seq_len": int(np.max(st["lens"])), "layers": n_layers,
+           "tokens_per_layer": tokens, "paged": bool(st["w"]["paged"]), "work_ranges": st["n_splits"],
+           "work_ranges_forced": bool(splits),
+           "l2": "inputs larger than L2: %d cache cop%s rotated, %.0f MB each" % (
+               len(st["layers"][0]["caches"]) * n_layers,
+               "y" if n_layers * len(st["layers"][0]["caches"]) == 1 else "ies", cache_bytes / 1e6),
+           "parallelism": f"replicas x{world}"}
+    return {
+        "value": job_throughput(step_bytes, world, ms), "ms_per_step": ms, "config": cfg,
+        "tflops": world * step_flops / (ms * 1e-3) / 1e12,
         "tokens_per_s": world * st["B"] / (ms * 1e-3),
-        "decode_layer_ms": dec_ms,
-        "phase_ms_per_layer": phase_ms,
-        "host_issue_ms_per_step": host_ms,
-        "timed_step": "one CUDA graph replay per step (all launches of the step); e2e uses plain API calls with "
-                      "one packed input copy and one read-back per step on a second stream, double-buffered and "
-                      "overlapping the neighbouring steps' kernels; "
-                      "phase and decode times from a second loop of per-phase graph replays with events",
+        "decode_layer_ms": dec_ms, "phase_ms_per_layer": r["phase_ms"],
+        "host_issue_ms_per_step": r["host_ms"],
         "roofline_step_frac": roofline_s / (ms * 1e-3),
         "roofline": {"kernel": "mla_decode_attn (split-KV decode + combine)", "bound": "hbm",
                      "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "peak_kind": peak_kind, "traffic": recorded_traffic(args.workload), "avg_launch_ms": dec_ms,
-                     "algorithmic_bytes_per_launch": dec_bytes},
-        "e2e": {"value": job_throughput(cache_bytes, world, e2e_ms), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": LAUNCHES_PER_LAYER * n_layers * args.steps,
-        "clocks": clocks,
-        "next_rows": next_rows,
+                     "peak_kind": peak_kind, "traffic": recorded_traffic(name, splits), "avg_launch_ms": dec_ms,
+                     "algorithmic_bytes_per_launch": dec_bytes,
+                     "tensor": {"achieved_tflops": dec_flops / (dec_ms * 1e-3) / 1e12, "peak": tc,
+                                "frac": dec_flops / (dec_ms * 1e-3) / 1e12 / tc},
+                     "nominal": {"hbm_peak": NOMINAL_HBM_GBS, "frac": achieved / NOMINAL_HBM_GBS,
+                                 "bf16_peak_tflops": NOMINAL_BF16_TFLOPS},
+                     "split_partials": {"segments": n_part, "bytes_written": n_part * PARTIAL_BYTES,
+                                        "bytes_read_by_combine": n_part * PARTIAL_BYTES,
+                                        "note": "not algorithmic bytes: reported beside them"}},
+        "e2e": {"value": job_throughput(step_bytes, world, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"], "ms_per_step": e2e_ms},
+        "clocks": r["clocks"], "timed_brackets": r["brackets"],
+        "gpu_launches": LAUNCHES_PER_LAYER * n_layers * r["brackets"],   # per K steps: times K below
     }
+
+
+def parse_extras(spec):
+    out = []
+    for item in (spec or "").split(","):
+        item = item.strip()
+        if not item:
+            continue
+        name, _, sp = item.partition("@")
+        if name not in mi.WORKLOADS:
+            raise SystemExit(f"unknown workload {name!r} in --extra-workloads")
+        out.append((name, int(sp) if sp else 0))
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import gc
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    import mla_latent_kv_20_b200 as m
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    peaks = load_peaks()
+    r = measure_workload(args.workload, args.splits, args, world, dev, barrier)
+    r["ms"], r["e2e_ms"], r["dec_ms"] = reduce_max_over_ranks([r["ms"], r["e2e_ms"], r["dec_ms"]], world, device=dev)
+    head = summarize(args.workload, args.splits, r, world, peaks)
+    st = r["st"]
+    next_rows = None if args.no_next_rows else {
+        "project_append": measure_project_append(st, args.steps, args.warmup),
+        "output_proj": measure_output_proj(st, args.steps, args.warmup),
+        "prefill": measure_prefill(args.steps, args.warmup)}
+    del r, st
+    gc.collect()
+    torch.cuda.empty_cache()
+    by_workload = {}
+    for name, splits in parse_extras(args.extra_workloads):
+        if name == args.workload and splits == args.splits:
+            continue
+        rx = measure_workload(name, splits, args, world, dev, barrier)
+        rx["ms"], rx["e2e_ms"], rx["dec_ms"] = reduce_max_over_ranks([rx["ms"], rx["e2e_ms"], rx["dec_ms"]], world,
+                                                                     device=dev)
+        sx = summarize(name, splits, rx, world, peaks)
+        sx["gpu_launches"] *= args.steps
+        key = name if not splits else f"{name}@{splits}"
+        if rank == 0 and not args.no_cpu_baseline and int(mi.WORKLOADS[name].get("layers", 1)) > 1:
+            tok, dt, step_s = time_oracle_layers(rx["st"]["lens"], rx["n_layers"])
+            threads, cores = cpu_threads()
+            sx["cpu_baseline"] = {"value": tok * ROW_BYTES / dt / 1e9, "unit": UNIT, "cores": threads,
+                                  "kind": "oracle", "form": "absorbed", "affinity_cores": cores,
+                                  "extrapolated_s_per_step": step_s,
+                                  "sample": f"2 layers x the first 8 sequences ({tok} cached tokens, full lengths) "
+                                            f"through the absorbed fp64 oracle ({dt:.1f} s); GB/s of cached rows "
+                                            f"processed, and the step time extrapolated by cached tokens to "
+                                            f"{rx['n_layers']} layers x {len(rx['st']['lens'])} sequences"}
+        by_workload[key] = sx
+        del rx
+        gc.collect()
+        torch.cuda.empty_cache()
+    assert m.get_device_error() == 0
+    if rank != 0:
+        return
+    head["gpu_launches"] *= args.steps
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) latents/keys/queries, "
+                                                     "N(0,1/512) weights)",
+        "config": head["config"],
+        "timed_step": "one CUDA graph replay per step (all launches of the step), K-step brackets back to back until "
+                      "%.1f s; e2e uses plain API calls with one packed input copy and one read-back per step on a "
+                      "second stream, double-buffered and overlapping the neighbouring steps' kernels; phase and "
+                      "decode times from a second loop of per-phase graph replays with events" % args.min_timed_s,
+    }
+    for k in ("tflops", "tokens_per_s", "decode_layer_ms", "phase_ms_per_layer", "host_issue_ms_per_step",
+              "roofline_step_frac", "roofline", "e2e", "gpu_launches", "clocks", "timed_brackets"):
+        line[k] = head[k]
+    line["next_rows"] = next_rows
+    line["by_workload"] = by_workload
     if not args.no_cpu_baseline:
-        tok, dt, nseq = time_oracle_sample(st["lens"])
+        lens = mi.workload_lengths(args.workload)
+        tok, dt, nseq = time_oracle_sample(lens)
+        tok_a, dt_a, nseq_a = time_oracle_sample(lens, min_seconds=4.0, form="absorbed")
         threads, cores = cpu_threads()
         line["cpu_baseline"] = {"value": tok * ROW_BYTES / dt / 1e9, "unit": UNIT, "cores": threads,
-                                "kind": "oracle", "affinity_cores": cores,
-                                "sample": f"{nseq} sequences of {tok // nseq} tokens of this workload, explicit "
-                                          f"fp64 form ({dt:.1f} s of CPU work), GB/s of cached rows processed"}
+                                "kind": "oracle", "form": "explicit", "affinity_cores": cores,
+                                "sample": f"the first {nseq} sequences of this workload ({tok} cached tokens, each "
+                                          f"at most 8192), explicit fp64 form ({dt:.1f} s of CPU work), GB/s of "
+                                          f"cached rows processed",
+                                "absorbed": {"value": tok_a * ROW_BYTES / dt_a / 1e9, "unit": UNIT,
+                                             "sample": f"the first {nseq_a} sequences ({tok_a} cached tokens), "
+                                                       f"absorbed fp64 form ({dt_a:.1f} s)"}}
     print(json.dumps(line), flush=True)
 
 
@@ -804,7 +948,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(mi.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--splits", type=int, default=0, help="forced work ranges of the decode (0: the auto plan)")
+    ap.add_argument("--extra-workloads", default=DEFAULT_EXTRAS,
+                    help="comma-separated NAME or NAME@RANGES measured after the headline (empty: none)")
+    ap.add_argument("--min-timed-s", type=float, default=MIN_TIMED_S)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true", help="skip the built next rows (profiling runs)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -156,7 +156,7 @@ WORKLOADS = {
     "b1_l256": dict(batch=1, lens="fixed", L=256, paged=False, seed=1001),
     "b32_l4096": dict(batch=32, lens="fixed", L=4096, paged=False, seed=1002),
     "b128_u1024_8192_paged": dict(batch=128, lens="uniform", lo=1024, hi=8192, paged=True, seed=1003),
-    "b4_l131072": dict(batch=4, lens="fixed", L=131072, paged=False, seed=1004, test_ranges=128),
+    "b4_l131072": dict(batch=4, lens="fixed", L=131072, paged=False, seed=1004, test_ranges=512),
     "l60_b256_log64_32768_paged": dict(batch=256, lens="loguniform", lo=64, hi=32768, paged=True,
                                        seed=1005, layers=60),
 }

@@ -62,3 +62,22 @@ def test_step_work_counts_bytes_and_flops():
     assert tokens == 8 and cache_bytes == 8 * 1152
     assert flops == 8 * 2 * 128 * (576 + 512) + 2 * 2 * (2 * 128 * 128 * 512)
     assert dec_bytes == cache_bytes + 2 * 128 * (576 + 512) * 2
+
+
+def test_partial_segments_follow_the_plan():
+    """Range partials a decode call writes: per-sequence plan (r_b ranges of sequence b, partials
+    only when r_b > 1) and the balanced plan (tiles end to end, a partial for every range that
+    meets only part of a sequence), on hand-worked cases."""
+    import bench
+    assert bench.partial_segments([4096] * 32, 74) == 64             # 32 tiles each: 2 ranges per sequence
+    assert bench.partial_segments([131072] * 4, 512) == 512          # 128 ranges of 8 tiles per sequence
+    assert bench.partial_segments([1280, 1280], 4) == 4              # tiles 10, 10: 2 ranges each
+    assert bench.partial_segments([256, 128, 384], 4) == 4           # balanced: ranges [0,1) [1,3) [3,4) [4,6)
+    assert bench.partial_segments([128, 128], 2) == 0                # one range per sequence: no partials
+    assert bench.partial_segments([0, 0], 4) == 0
+
+
+def test_extra_workloads_spec():
+    import bench
+    assert bench.parse_extras("b32_l4096, b4_l131072@512") == [("b32_l4096", 0), ("b4_l131072", 512)]
+    assert bench.parse_extras("") == []

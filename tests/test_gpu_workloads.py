@@ -1,6 +1,7 @@
 """Parity at the full workload sizes, in the launch configuration bench.py times (the auto work
-plan), or with 128 forced work ranges for the long-context workload (so each of its sequences is
-merged from 32 partials), checked on sampled sequences that the fp64 oracle computes one by one."""
+plan), or with 512 forced work ranges for the long-context workload (each of its 4 sequences of
+131072 tokens is cut into 128 ranges of 8 tiles and merged from 128 partials), checked on sampled
+sequences that the fp64 oracle computes one by one."""
 import numpy as np
 import pytest
 
@@ -55,8 +56,41 @@ def test_b128_paged_uniform_lengths():
     _run_workload("b128_u1024_8192_paged", [int(np.argmin(lens)), int(np.argmax(lens)), 64])
 
 
-def test_b4_l131072_128_ranges():
-    _run_workload("b4_l131072", [2], explicit_first=False)
+def test_b4_l131072_128_ranges_per_sequence():
+    """The long-context workload split 128 ways per sequence (512 forced work ranges): the whole
+    step against the oracle on two of the four sequences."""
+    assert mi.WORKLOADS["b4_l131072"]["test_ranges"] == 512
+    _run_workload("b4_l131072", [0, 2], explicit_first=False)
+
+
+def test_b4_l131072_decode_kernel_128_partials():
+    """The decode call alone on the same workload with 512 forced ranges, the query being the bf16
+    rounding of the oracle's absorbed query: out_lat and lse of two sequences against the oracle's
+    absorbed attention at the decode kernel's bound (each is merged from 128 range partials)."""
+    import torch
+    from mla_latent_kv_20_b200 import get_device_error
+    from mla_latent_kv_20_b200 import harness as hz
+    from gpu_common import assert_lse, assert_out_lat
+    name = "b4_l131072"
+    w = mi.WORKLOADS[name]
+    lens = mi.workload_lengths(name)
+    batch = mi.decode_batch(w["seed"], lens)
+    wts = mi.layer_weights(w["seed"] + 1)
+    cache = hz.Cache(lens, False, fill_value=None)
+    cache.fill(batch.c, batch.kr)
+    qa = oracle.absorb_q(f64(batch.q_nope), f64(wts.w_uk))
+    qf_bits = mi.f64_to_bf16(oracle.q_full(qa, f64(batch.q_pe)))
+    out_lat, lse = hz.decode(hz.bf16_tensor(qf_bits), cache, num_splits=512)
+    torch.cuda.synchronize()
+    assert get_device_error() == 0
+    g_lat = f64(hz.bf16_bits(out_lat))
+    g_lse = lse.cpu().numpy()
+    for i in (1, 3):
+        L = int(lens[i])
+        rows = oracle.cache_rows(f64(batch.c[i]), f64(batch.kr[i]), np.arange(L))
+        ref = oracle.attend_rows(f64(qf_bits[i]), rows, SCALE, mi.D_LATENT)
+        assert_out_lat(g_lat[i], ref["out_lat"])
+        assert_lse(g_lse[i], ref["lse"])
 
 
 def test_l60_one_layer_full_size():
