@@ -462,6 +462,64 @@ def measure_output_proj(st, steps, warmup):
             "frac": gbs / hbm, "l2": "weight (168 MB) larger than L2 (median of %d back-to-back calls)" % n}
 
 
+FP8_ROW_BYTES = 576 + 1   # E4M3 codes + the E8M0 scale byte of a token
+
+
+def measure_fp8_decode(name, steps, warmup):
+    """The FP8-cache row: the same workload's rows (the seeded host generator) appended as E4M3
+    codes with power-of-two row scales (mla_cache_append_fp8), then mla_decode_attn_fp8 timed per
+    call with CUDA events (median) over two rotated cache copies (larger than L2 together), with
+    the workload's bf16 decode call timed the same way beside it.  Algorithmic bytes: 577 per
+    cached token plus q_full in and out_lat out."""
+    import torch
+    import mla_latent_kv_20_b200 as m
+    from mla_latent_kv_20_b200 import harness as hz
+    w, lens = workload_shape(name)
+    batch = mi.decode_batch(w["seed"], lens)
+    table, nblk = mi.block_permutation(w["seed"] + 2, lens) if w["paged"] else (None, 0)
+    caches = []
+    for _ in range(2):
+        c = hz.Fp8Cache(lens, w["paged"], table, nblk, fill_byte=None)
+        c.fill(batch.c, batch.kr)
+        caches.append(c)
+    del batch
+    B = len(lens)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(9004)
+    qf = torch.randn((B, mi.N_HEADS, mi.D_ROW), device="cuda", generator=gen).to(torch.bfloat16)
+    out_lat = torch.empty((B, mi.N_HEADS, mi.D_LATENT), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, mi.N_HEADS), dtype=torch.float32, device="cuda")
+    ws = torch.empty((m.decode_workspace_size(B, caches[0].capacity(), 0),), dtype=torch.uint8, device="cuda")
+
+    def call(i):
+        c = caches[i % 2]
+        m.decode_attn_fp8(qf, c.data, c.scales, c.seq_lens, c.desc, ws, out_lat, lse=lse, block_table=c.block_table)
+
+    for i in range(max(warmup, 2)):
+        call(i)
+    torch.cuda.synchronize()
+    n = min(max(steps, 2), 200)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i, (e0, e1) in enumerate(ev):
+        e0.record()
+        call(i)
+        e1.record()
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+    ms = sorted(e0.elapsed_time(e1) for e0, e1 in ev)[n // 2]
+    tokens = int(np.sum(lens))
+    nbytes = tokens * FP8_ROW_BYTES + B * mi.N_HEADS * (mi.D_ROW + mi.D_LATENT) * 2
+    hbm, tc = load_peaks()[0], load_peaks()[1]
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    tf = tokens * FLOP_PER_TOKEN / (ms * 1e-3) / 1e12
+    del caches, qf, out_lat, lse, ws
+    return {"kernel": "decode_tc_kernel<false, true> (FP8 codes expanded to bf16 in shared memory) + combine_kernel",
+            "workload": name, "us_per_call": ms * 1e3, "bound": "hbm", "algorithmic_bytes_per_launch": nbytes,
+            "bytes_per_token": FP8_ROW_BYTES, "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+            "tensor": {"achieved_tflops": tf, "peak": tc, "frac": tf / tc},
+            "l2": "two cache copies rotated (%.0f MB each), median of %d calls" % (tokens * FP8_ROW_BYTES / 1e6, n)}
+
+
 PREFILL_SEQS, PREFILL_PREFIX, PREFILL_CHUNK = 4, 3072, 1024
 
 
@@ -879,6 +937,11 @@ def run_ours(args, rank, world, local_rank):
         "output_proj": measure_output_proj(st, args.steps, args.warmup),
         "prefill": measure_prefill(args.steps, args.warmup)}
     del r, st
+    gc.collect()
+    torch.cuda.empty_cache()
+    if next_rows is not None:
+        next_rows["fp8_decode"] = measure_fp8_decode(args.workload, args.steps, args.warmup)
+        next_rows["fp8_decode"]["bf16_decode_us_same_workload"] = head["decode_layer_ms"] * 1e3
     gc.collect()
     torch.cuda.empty_cache()
     by_workload = {}

@@ -104,6 +104,26 @@ mla_status mla_cache_append(const mla_bf16* c_new, const mla_bf16* kr_new, const
                             mla_cache_desc desc, int32_t n_tokens, float rope_base, void* stream);
 
 /*
+ * (1-fp8) Cache append into an FP8 latent cache — [DR] §4.2 效率证据 (FP8 serving with the KV cache
+ *     at about 6 bits per element; the pages give no format, this library's reading follows).
+ * For each new token i, the row r = [c_new[i] (512) | RoPE(kr_new[i], pos[i]) (64)] is formed in
+ * fp64 (the latent exactly, the key rotated in fp64 with no bf16 rounding) and stored as
+ *     k = the smallest integer with max_j |r_j| <= 448 * 2^k   (0 for an all-zero row)
+ *     scales[row] = k + 127                        (E8M0: the byte e stands for the scale 2^(e - 127))
+ *     cache[row * 576 + j] = E4M3 code of fp32(r_j * 2^-k)   (OCP E4M3, round to nearest even,
+ *                                                             saturating at +-448)
+ * so r_j is approximated by code_value * 2^k, which is exact in bf16: 577 bytes per token, against
+ * 1152 for the bf16 row.
+ *   cache  [num_rows, 576] uint8 (E4M3 codes; contiguous or paged exactly as the bf16 cache, with
+ *          the row index of the descriptor)              scales [num_rows] uint8 (E8M0, written)
+ *   other arguments, checks and device errors as mla_cache_append.  cache 16-byte aligned.
+ * Rows whose largest magnitude is below about 1e-33 lose their smallest codes when expanded to bf16.
+ */
+mla_status mla_cache_append_fp8(const mla_bf16* c_new, const mla_bf16* kr_new, const int32_t* seq_ids,
+                                const int32_t* pos, uint8_t* cache, uint8_t* scales, const int32_t* block_table,
+                                mla_cache_desc desc, int32_t n_tokens, float rope_base, void* stream);
+
+/*
  * (1') Down-projection + cache append — [DR] §2.2 (c^KV = W_D^KV h_t), §3.1 (k^R, the shared
  *      64-wide key of the RoPE branch, is projected from h_t too; c^KV and k^R are the only cached
  *      objects), §2.4 (RoPE on that branch only), §3.3 (model width d = 5120).
@@ -215,6 +235,22 @@ mla_status mla_prefill_attn(const mla_bf16* q_full, const mla_bf16* cache, const
                             const int32_t* q_seq, const int32_t* q_len, mla_cache_desc desc, int32_t n_queries,
                             float softmax_scale, int32_t num_splits, void* workspace, size_t workspace_bytes,
                             mla_bf16* out_lat, float* lse, void* stream);
+
+/*
+ * (3-fp8) Decode attention over an FP8 latent cache — [DR] §4.2 效率证据 (FP8 KV cache) with the
+ *     attention of (3): every cached row is taken as code_value * 2^(scales[row] - 127), the rows
+ *     mla_cache_append_fp8 writes, and attended exactly as mla_decode_attn attends bf16 rows (the
+ *     decoded values are exact in bf16, so the result is that of mla_decode_attn on a bf16 cache
+ *     holding them).
+ *   cache  [num_rows, 576] uint8 E4M3 codes   scales [num_rows] uint8 E8M0 exponents (16-byte aligned)
+ *   every other argument, output, workspace and error as mla_decode_attn (mla_decode_workspace_size
+ *   applies unchanged).  A contiguous cache needs max_seq_len % 16 == 0 (the scale bytes of a
+ *   64-row box are copied from a 16-byte boundary), else MLA_ERR_INVALID_ARG.
+ */
+mla_status mla_decode_attn_fp8(const mla_bf16* q_full, const uint8_t* cache, const uint8_t* scales,
+                               const int32_t* block_table, const int32_t* seq_lens, mla_cache_desc desc,
+                               int32_t batch, float softmax_scale, int32_t num_splits, void* workspace,
+                               size_t workspace_bytes, mla_bf16* out_lat, float* lse, void* stream);
 
 /*
  * Decode attention that allocates nothing and takes no workspace (the pages have no counterpart:

@@ -51,6 +51,8 @@ def _load():
         "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "mla_version": (I32, []),
         "mla_cache_append": (ctypes.c_int, [P, P, P, P, P, P, CacheDesc, I32, F32, P]),
+        "mla_cache_append_fp8": (ctypes.c_int, [P, P, P, P, P, P, P, CacheDesc, I32, F32, P]),
+        "mla_decode_attn_fp8": (ctypes.c_int, [P, P, P, P, P, CacheDesc, I32, F32, I32, P, SZ, P, P, P]),
         "mla_project_append": (ctypes.c_int, [P, P, P, P, P, P, P, CacheDesc, I32, F32, P]),
         "mla_output_proj": (ctypes.c_int, [P, P, P, I32, P]),
         "mla_append_absorb": (ctypes.c_int, [P, P, P, P, P, P, CacheDesc, I32, P, P, P, P, P, I32, F32, P]),
@@ -108,6 +110,15 @@ def cache_append(c_new, kr_new, pos, cache, desc: CacheDesc, *, seq_ids=None, bl
                                 _ptr(block_table), desc, n, rope_base, _stream(stream)), "mla_cache_append")
 
 
+def cache_append_fp8(c_new, kr_new, pos, cache, scales, desc: CacheDesc, *, seq_ids=None, block_table=None,
+                     rope_base: float = 10000.0, stream=None, n_tokens: int | None = None):
+    """mla_cache_append_fp8: rows as E4M3 codes (cache, uint8 [rows, 576]) with E8M0 row scales
+    (scales, uint8 [rows])."""
+    n = c_new.shape[0] if n_tokens is None else n_tokens
+    _check(lib.mla_cache_append_fp8(_ptr(c_new), _ptr(kr_new), _ptr(seq_ids), _ptr(pos), _ptr(cache), _ptr(scales),
+                                    _ptr(block_table), desc, n, rope_base, _stream(stream)), "mla_cache_append_fp8")
+
+
 def project_append(h, w_dkv, w_kr, pos, cache, desc: CacheDesc, *, seq_ids=None, block_table=None,
                    rope_base: float = 10000.0, stream=None, n_tokens: int | None = None):
     n = h.shape[0] if n_tokens is None else n_tokens
@@ -156,6 +167,17 @@ def decode_attn(q_full, cache, seq_lens, desc: CacheDesc, workspace, out_lat, *,
     _check(lib.mla_decode_attn(_ptr(q_full), _ptr(cache), _ptr(block_table), _ptr(seq_lens), desc, b,
                                softmax_scale, num_splits, _ptr(workspace), wb, _ptr(out_lat), _ptr(lse),
                                _stream(stream)), "mla_decode_attn")
+
+
+def decode_attn_fp8(q_full, cache, scales, seq_lens, desc: CacheDesc, workspace, out_lat, *, lse=None,
+                    block_table=None, softmax_scale: float = 1.0 / 192 ** 0.5, num_splits: int = 0, stream=None,
+                    batch: int | None = None, workspace_bytes: int | None = None):
+    """mla_decode_attn_fp8: decode over an FP8 cache (E4M3 codes + E8M0 row scales)."""
+    b = q_full.shape[0] if batch is None else batch
+    wb = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(lib.mla_decode_attn_fp8(_ptr(q_full), _ptr(cache), _ptr(scales), _ptr(block_table), _ptr(seq_lens), desc,
+                                   b, softmax_scale, num_splits, _ptr(workspace), wb, _ptr(out_lat), _ptr(lse),
+                                   _stream(stream)), "mla_decode_attn_fp8")
 
 
 def prefill_attn(q_full, cache, q_seq, q_len, desc: CacheDesc, workspace, out_lat, *, lse=None,

@@ -95,4 +95,108 @@ __global__ void __launch_bounds__(96) cache_append_kernel(const uint4* __restric
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// FP8 (E4M3) latent cache rows (《DeepSeek-V2》深度解读报告 §4.2 效率证据: FP8 serving with the KV cache
+// at about 6 bits per element; the format is this library's reading).  A token's row is the 576
+// values [c^KV | RoPE(k^R, pos)], taken in fp64 (the latent exactly from its bf16 input, the key
+// rotated in fp64 and never rounded to bf16), stored as 576 OCP E4M3 codes plus one fp32 scale per
+// token: the power of two 2^k, k the smallest integer with amax <= 448 * 2^k (amax the row's
+// largest magnitude, k = 0 for an all-zero row), kept as its E8M0 byte k + 127.  A value x is
+// coded as the E4M3 value nearest to the fp32 rounding of x * 2^-k (ties to even, saturating at
+// +-448).  A code times its scale is exact in bf16, so the decode expands FP8 tiles into exact bf16
+// MMA operands.
+// ------------------------------------------------------------------------------------------
+constexpr double kE4m3Max = 448.0;
+
+// Two E4M3 codes (round to nearest even, saturating to +-448) of lo and hi; lo in the low byte.
+__device__ __forceinline__ uint16_t e4m3x2_rn_sat(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// k of the row scale 2^k: the smallest integer with amax <= 448 * 2^k (0 for amax = 0).
+__device__ __forceinline__ int fp8_scale_exp(double amax) {
+  if (!(amax > 0.0)) return 0;
+  int e = 0;
+  (void)frexp(amax / kE4m3Max, &e);   // amax / 448 = f 2^e, f in [0.5, 1): 2^e bounds it up to rounding
+  int k = e;
+  if (amax > kE4m3Max * ldexp(1.0, k)) ++k;          // settle k by exact comparisons
+  if (amax <= kE4m3Max * ldexp(1.0, k - 1)) --k;
+  return k;
+}
+
+// One CTA of 96 threads per new token: threads 0..63 hold 8 latent values each, threads 64..95
+// one rotated pair each (fp64); the CTA reduces the row's largest magnitude, then every thread
+// codes its values and writes them, and thread 0 writes the token's scale.
+__global__ void __launch_bounds__(96) cache_append_fp8_kernel(const uint4* __restrict__ c_new,
+                                                              const __nv_bfloat162* __restrict__ kr_new,
+                                                              const int32_t* __restrict__ seq_ids,
+                                                              const int32_t* __restrict__ pos, uint8_t* cache,
+                                                              uint8_t* scales, CacheView v, RopeFreq f) {
+  __shared__ double red[3];
+  pdl_trigger();
+  pdl_wait();
+  const int i = blockIdx.x;
+  const int seq = seq_ids ? seq_ids[i] : i;
+  const int p = pos[i];
+  const int capacity = v.page_size == 0 ? v.max_seq_len : v.max_blocks * kPage;
+  if (p < 0 || p >= capacity || seq < 0 || seq >= v.num_seqs) {   // the same for every thread of the CTA
+    if (threadIdx.x == 0) set_dev_error(0x1);
+    return;
+  }
+  const int64_t row = cache_row(v, seq, p);
+  if (row < 0) return;
+  const int t = threadIdx.x;
+  double x[8];
+  int nv = 2;
+  if (t < 64) {
+    const uint4 u = c_new[static_cast<int64_t>(i) * (kDLat / 8) + t];
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      x[2 * j] = static_cast<double>(__low2float(h[j]));
+      x[2 * j + 1] = static_cast<double>(__high2float(h[j]));
+    }
+    nv = 8;
+  } else {
+    const int pr = t - 64;   // pair index 0..31
+    double sn, cs;
+    sincos(static_cast<double>(p) * f.inv_freq[pr], &sn, &cs);
+    const __nv_bfloat162 k2 = kr_new[static_cast<int64_t>(i) * (kDRope / 2) + pr];
+    const double xe = static_cast<double>(__low2float(k2));
+    const double xo = static_cast<double>(__high2float(k2));
+    x[0] = xe * cs - xo * sn;
+    x[1] = xe * sn + xo * cs;
+#pragma unroll
+    for (int j = 2; j < 8; ++j) x[j] = 0.0;
+  }
+  double am = 0.0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) am = fmax(am, fabs(x[j]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmax(am, __shfl_xor_sync(0xffffffffu, am, o));
+  if ((t & 31) == 0) red[t >> 5] = am;
+  __syncthreads();
+  const double amax = fmax(fmax(red[0], red[1]), red[2]);
+  // The E8M0 byte holds k in [-127, 127]; bf16 inputs keep amax within it.
+  const int k = min(max(fp8_scale_exp(amax), -127), 127);
+  const double inv = ldexp(1.0, -k);   // x * 2^-k is exact in fp64
+  uint8_t* dst = cache + row * kDRow;
+  if (nv == 8) {
+    uint32_t w[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t lo = e4m3x2_rn_sat(static_cast<float>(x[4 * j] * inv), static_cast<float>(x[4 * j + 1] * inv));
+      const uint32_t hi = e4m3x2_rn_sat(static_cast<float>(x[4 * j + 2] * inv), static_cast<float>(x[4 * j + 3] * inv));
+      w[j] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint2*>(dst + 8 * t) = make_uint2(w[0], w[1]);
+  } else {
+    *reinterpret_cast<uint16_t*>(dst + kDLat + 2 * (t - 64)) =
+        e4m3x2_rn_sat(static_cast<float>(x[0] * inv), static_cast<float>(x[1] * inv));
+  }
+  if (t == 0) scales[row] = static_cast<uint8_t>(k + 127);
+}
+
 }  // namespace mla

@@ -38,9 +38,19 @@
 // quadrant, each owning half of the S columns), warp 8 work plan and TMA producer, and in the
 // even CTA only: warp 9 QK^T part A (warp 9 also allocates TMEM in both CTAs), warp 11 QK^T part
 // B, warps 10 and 12 PV for the two latent halves.
+//
+// FP8 cache (kFp8, 544 threads).  Rows are 576 E4M3 codes with a power-of-two scale per token (an
+// E8M0 exponent byte, 2^(e - 127)): code * scale is exact in bf16, so the MMAs, the softmax and
+// the epilogue are those of the bf16 cache.  The producer copies a box's codes into the upper half
+// of the bf16 buffer it will become, and the box's 64 scale bytes to the buffer's start, on a
+// CTA-local barrier; four converter warps (13-16) read both into registers, and after a barrier
+// among themselves write the exact bf16 values of code * scale over the whole buffer in the
+// swizzled layout the MMAs read (zeroing V rows past the segment end), then publish the buffer to
+// the pair barrier the MMA waits on.
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <climits>
 
@@ -83,6 +93,15 @@ constexpr int kTcPvWarp = 10;     // PV issue, first latent half (even CTA)
 constexpr int kTcMmaBWarp = 11;   // QK^T part B issue (even CTA)
 constexpr int kTcPv1Warp = 12;    // PV issue, second latent half (even CTA)
 constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 5);
+// FP8 cache: four converter warps after the others.
+constexpr int kTcConvWarp0 = kTcSoftmaxWarps + 5;
+constexpr int kTcConvThreads = 128;
+constexpr int kTcThreadsFp8 = kTcThreads + kTcConvThreads;
+__host__ __device__ constexpr int tc_threads(bool fp8) { return fp8 ? kTcThreadsFp8 : kTcThreads; }
+// Where the codes of a box wait for conversion: the upper half of the bf16 buffer they become.
+constexpr int kTcFp8OffA = kTcKSlabsA * kTcSlab / 2;
+constexpr int kTcFp8OffB = kTcKSlabsB * kTcSlab / 2;
+constexpr int kTcFp8OffV = kTcVBox / 2;
 
 struct DecodeTcArgs {
   CacheView v;
@@ -95,6 +114,7 @@ struct DecodeTcArgs {
   __nv_bfloat16* out_lat;
   float* lse;
   const uint8_t* cache;   // the cache buffer (L2 prefetch addresses)
+  int row_bytes;          // bytes of one cached row: 1152 (bf16) or 576 (FP8 codes)
   const int32_t* seq_map; // query row -> cache sequence (chunked prefill), or null: row b reads sequence b
 };
 
@@ -121,6 +141,8 @@ struct TcBars {
   uint64_t o_free;               // both: every softmax warp of both CTAs has read O of a segment
   uint64_t q_full;               // even CTA only: Q of both CTAs landed (one phase per segment)
   uint64_t q_empty;              // both: QK^T of a segment's last tile done (two commits)
+  uint64_t kraw[2];              // FP8, per CTA and part: this CTA's K codes and scales landed (+ tx)
+  uint64_t vraw[kTcVSlots];      // FP8, per CTA and slot: this CTA's V codes and scales landed (+ tx)
 };
 static_assert(sizeof(TcBars) <= 256, "barrier block");
 static_assert(kTcSmemBytes <= 232448, "shared memory budget");
@@ -144,6 +166,42 @@ __device__ __forceinline__ int tc_cache_seq(const DecodeTcArgs& a, int b, bool r
   if (s >= 0 && s < a.v.num_seqs) return s;
   if (report) set_dev_error(0x2);
   return -1;
+}
+
+// Block ids of a paged cache for the producer warp, so that the row of a copy needs no dependent
+// load of the block table on the way to the copy (211 instead of 223 us for the batch-128 paged
+// workload, A/B on identical inputs): lane l holds the ids of pages wp + l (cur) and wp + 32 + l
+// (nxt) of cache sequence b.  A lookup past wp + 48 slides the window by 32 pages and requests the
+// next 32 ids then, 16 pages (8 tiles) before they are needed; lookups stay within 16 pages behind
+// the furthest one (the V copies of a tile follow the K copy of the next one).
+struct PageWindow {
+  int b = -1, wp = 0, cur = -1, nxt = -1;
+};
+__device__ __forceinline__ int pw_entry(const CacheView& v, int b, int p) {
+  return (p >= 0 && p < v.max_blocks) ? v.block_table[static_cast<int64_t>(b) * v.max_blocks + p] : -1;
+}
+// TMA row of token t of cache sequence b (every lane calls it with the same arguments and gets the
+// same row), or -kTcTile (a fully out-of-bounds box) with the error word set for a bad block id.
+__device__ __forceinline__ int pw_row(PageWindow& w, const CacheView& v, int b, int t, int lane) {
+  const int p = t / kPage;
+  if (b != w.b || p < w.wp || p >= w.wp + 64) {
+    w.b = b;
+    w.wp = p & ~31;
+    w.cur = pw_entry(v, b, w.wp + lane);
+    w.nxt = pw_entry(v, b, w.wp + 32 + lane);
+  } else if (p >= w.wp + 48) {
+    w.cur = w.nxt;
+    w.wp += 32;
+    w.nxt = pw_entry(v, b, w.wp + 32 + lane);
+  }
+  const int d = p - w.wp;
+  const int blk = __shfl_sync(0xffffffffu, d < 32 ? w.cur : w.nxt, d & 31);
+  const int64_t r = static_cast<int64_t>(blk) * kPage + (t % kPage);
+  if (blk < 0 || r >= v.num_rows) {
+    if (lane == 0) set_dev_error(0x2);
+    return -kTcTile;
+  }
+  return static_cast<int>(r);
 }
 
 // 3-D TMA load (x: element in a 64-wide dim-slab, y: cache row, z: dim-slab) into this CTA's
@@ -220,10 +278,11 @@ __device__ __noinline__ bool tc_load_ragged_v(uint8_t* box, const CUtensorMap* t
   return true;
 }
 
-template <bool kMapped>
+template <bool kMapped, bool kFp8>
 __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, const CUtensorMap* tm_v,
-                            const CUtensorMap* tm_q, const DecodeTcArgs& a, const TcPlan& plan, uint8_t* smem,
-                            TcBars* bars, uint32_t rank, int pair, volatile int* abort_flag) {
+                            const CUtensorMap* tm_q, const CUtensorMap* tm_sc, const DecodeTcArgs& a,
+                            const TcPlan& plan, uint8_t* smem, TcBars* bars, uint32_t rank, int pair,
+                            volatile int* abort_flag) {
   const int lane = threadIdx.x & 31;
   const bool l0 = lane == 0;
   const bool leader = rank == 0;
@@ -240,6 +299,8 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
   int k = 0;    // segment index
   uint32_t fix_phase = 0;
   bool ok = true;
+  PageWindow pw;
+  const bool paged = a.v.page_size != 0;
   while (ok && cur.next(a.seq_lens, a.capacity, sg)) {
     const int b = sg.b, t_begin = sg.tok_begin, t_end = sg.tok_end, n_tiles = sg.n_tiles;
     // Q of sequence b.  The buffer is free once both QK^T parts have finished the previous segment.
@@ -256,10 +317,12 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
       else
         mbar_arrive_relaxed(lbar(&bars->q_full));
     }
-    // TMA row of token t of query row b's sequence (a fully out-of-bounds box for a bad map entry)
+    // TMA row of token t of query row b's sequence (a fully out-of-bounds box for a bad map entry).
+    // Every lane calls it (the paged lookup shares the block ids across the warp).
+    const int cb = tc_cache_seq<kMapped>(a, b, true);
     auto row_of = [&](int t) -> int {
-      const int cb = tc_cache_seq<kMapped>(a, b, true);
-      return (kMapped && cb < 0) ? -kTcTile : tma_row(a.v, cb, t);
+      if (kMapped && cb < 0) return -kTcTile;
+      return paged ? pw_row(pw, a.v, cb, t, lane) : tma_row(a.v, cb, t);
     };
     auto issue_k = [&](int i) -> bool {
       const int gi = g + i;
@@ -268,13 +331,22 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
 #pragma unroll 1
       for (int part = 0; part < 2; ++part) {
         if (gi >= 1 && !wait0(&bars->k_empty[part], static_cast<uint32_t>(gi - 1) & 1u, 0x10 + part)) return false;
+        uint8_t* slot = smem + kTcOffK + tc_part_slab0(part) * kTcSlab;
         if (l0) {
-          tma_load_3d_pair(smem + kTcOffK + tc_part_slab0(part) * kTcSlab, part ? tm_kb : tm_ka,
-                           lbar(&bars->k_full[part]), 0, y, tc_part_slab0(part));
-          if (leader)
-            mbar_arrive_expect_tx_relaxed(lbar(&bars->k_full[part]), 2u * tc_part_slabs(part) * kTcSlab);
-          else
-            mbar_arrive_relaxed(lbar(&bars->k_full[part]));
+          if constexpr (kFp8) {
+            // codes to the slot's upper half, the 64 rows' scale bytes to its start (this CTA only;
+            // the converter warps publish the converted slot to k_full)
+            mbar_arrive_expect_tx(&bars->kraw[part], static_cast<uint32_t>(tc_part_slabs(part) * kTcSlab / 2 + 64));
+            tma_load_3d(slot + (part ? kTcFp8OffB : kTcFp8OffA), part ? tm_kb : tm_ka, &bars->kraw[part], 0, y,
+                        tc_part_slab0(part));
+            tma_load_1d(slot, tm_sc, &bars->kraw[part], y);
+          } else {
+            tma_load_3d_pair(slot, part ? tm_kb : tm_ka, lbar(&bars->k_full[part]), 0, y, tc_part_slab0(part));
+            if (leader)
+              mbar_arrive_expect_tx_relaxed(lbar(&bars->k_full[part]), 2u * tc_part_slabs(part) * kTcSlab);
+            else
+              mbar_arrive_relaxed(lbar(&bars->k_full[part]));
+          }
         }
       }
       return true;
@@ -291,16 +363,31 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
         uint8_t* box = smem + kTcOffV + s * kTcVBox;
         const int tok0 = t_begin + i * kTcTile + 64 * h;
         const int vcount = min(max(t_end - tok0, 0), 64);
+        const int row = vcount > 0 ? row_of(tok0) : 0;
+        if constexpr (kFp8) {
+          // The converter warps zero the rows past the segment end; a box with none in the
+          // segment is not copied, its barrier completes on the arrival alone.
+          if (l0) {
+            if (vcount > 0) {
+              mbar_arrive_expect_tx(&bars->vraw[s], static_cast<uint32_t>(kTcVBox / 2 + 64));
+              tma_load_4d_local(box + kTcFp8OffV, tm_v, &bars->vraw[s], 0, row, 2 * static_cast<int>(rank), 0);
+              tma_load_1d(box, tm_sc, &bars->vraw[s], row);
+            } else {
+              mbar_arrive(&bars->vraw[s]);
+            }
+          }
+          continue;
+        }
         if (vcount == 64) {
           if (l0) {
-            tma_load_4d_pair(box, tm_v, lbar(&bars->v_full[s]), 0, row_of(tok0), 2 * static_cast<int>(rank), 0);
+            tma_load_4d_pair(box, tm_v, lbar(&bars->v_full[s]), 0, row, 2 * static_cast<int>(rank), 0);
             if (leader)
               mbar_arrive_expect_tx_relaxed(lbar(&bars->v_full[s]), 2u * kTcVBox);
             else
               mbar_arrive_relaxed(lbar(&bars->v_full[s]));
           }
         } else {
-          if (!tc_load_ragged_v(box, tm_v, &bars->fix, fix_phase, vcount > 0 ? row_of(tok0) : 0,
+          if (!tc_load_ragged_v(box, tm_v, &bars->fix, fix_phase, row,
                                 static_cast<int>(rank), vcount, lbar(&bars->v_full[s]), abort_flag))
             return false;
           if (vcount > 0) fix_phase ^= 1u;
@@ -308,7 +395,9 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
       }
       return true;
     };
-    // K(i) then V(i - 1): one call site each (the loop runs one step past the last K).
+    // K(i) then V(i - 1): one call site each (the loop runs one step past the last K).  (Paged rows
+    // pulled into L2 two tiles ahead by this warp's lanes measured slower: 211 -> 232 us for the
+    // batch-128 paged workload, A/B on identical inputs.)
     for (int i = 0; ok && i <= n_tiles; ++i) {
       if (i < n_tiles) ok = issue_k(i);
       if (i > 0 && ok) ok = issue_v(i - 1);
@@ -424,6 +513,103 @@ __device__ bool tc_mma_pv(uint8_t* smem, TcBars* bars, uint32_t tmem, int nh, co
   return ok;
 }
 
+// ------------------------------------------------------------------------------ FP8 converter warps
+// 2^(e - 127) of an E8M0 scale byte (e = 255, not written by the FP8 append, is read as 2^128 = inf).
+__device__ __forceinline__ float e8m0_value(uint32_t e) {
+  return e == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(e << 23);
+}
+
+// 16 E4M3 codes (one 16-byte chunk) times the row scale, as 16 exact bf16 values in two 16-byte
+// chunks (codes 0-7, codes 8-15).
+__device__ __forceinline__ void e4m3x16_to_bf16(const uint4& c, float mult, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const uint32_t f2 = e4m3x2_to_f16x2(static_cast<uint16_t>(w[q] >> (16 * hh)));
+      const __half2 h2 = *reinterpret_cast<const __half2*>(&f2);
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(__low2float(h2) * mult, __high2float(h2) * mult);
+      o[2 * q + hh] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// One box: wait for its codes and scale bytes (a CTA-local barrier), read this thread's chunks and
+// its two rows' scales, meet the other converter threads (the buffer is then free to overwrite),
+// write the bf16 values into the 128-byte-swizzled slab layout of the buffer (rows at or past
+// `vcount` as zeros), and publish the buffer on the even CTA's barrier `done`.  The staged codes
+// are laid out [slab][row][64 bytes], so converter thread ct takes chunk ct + 128 j: piece ct & 3
+// of row (ct >> 2) + 32 (j & 1) of slab j >> 1.  False (the same in every converter thread) if
+// the wait failed or the kernel is aborting.
+template <int kSlabs>
+__device__ __forceinline__ bool tc_convert_box(uint8_t* buf, int codes_off, int vcount, uint64_t* raw, uint32_t parity,
+                                               uint32_t done, volatile int* abort_flag, int ct) {
+  const bool got = mbar_wait(raw, parity, 0x17) && !*abort_flag;
+  if (!named_bar_red_and(3, kTcConvThreads, got)) return false;
+  const int pc = ct & 3;
+  const int rb = ct >> 2;
+  uint4 c[2 * kSlabs];
+#pragma unroll
+  for (int j = 0; j < 2 * kSlabs; ++j)
+    c[j] = *reinterpret_cast<const uint4*>(buf + codes_off + 16 * (ct + kTcConvThreads * j));
+  const float m0 = e8m0_value(buf[rb]);
+  const float m1 = e8m0_value(buf[rb + 32]);
+  named_bar_sync(3, kTcConvThreads);   // every staged byte has been read
+#pragma unroll
+  for (int j = 0; j < 2 * kSlabs; ++j) {
+    const int row = rb + 32 * (j & 1);
+    uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+    if (row < vcount) e4m3x16_to_bf16(c[j], (j & 1) ? m1 : m0, lo, hi);
+    uint8_t* dst = buf + (j >> 1) * kTcSlab + row * 128;
+    *reinterpret_cast<uint4*>(dst + (((2 * pc) ^ (row & 7)) << 4)) = lo;
+    *reinterpret_cast<uint4*>(dst + (((2 * pc + 1) ^ (row & 7)) << 4)) = hi;
+  }
+  fence_proxy_async_smem();
+  named_bar_sync(3, kTcConvThreads);
+  if (ct == 0) {
+    fence_release_smem_to_cluster();
+    mbar_arrive_relaxed(done);
+  }
+  return true;
+}
+
+// The converter warps walk the boxes in the producer's order: K(0), K(1), V(0), K(2), V(1), ...
+// (both parts of a K tile, then both 64-token V boxes of a tile).
+template <bool kMapped>
+__device__ bool tc_convert(const DecodeTcArgs& a, const TcPlan& plan, int pair, uint8_t* smem, TcBars* bars,
+                           volatile int* abort_flag) {
+  const int ct = static_cast<int>(threadIdx.x) - 32 * kTcConvWarp0;
+  SegmentCursor cur{plan.b0, plan.off0, plan.start, plan.end, plan.b_end, pair, true, plan.len0};
+  Segment sg;
+  int g = 0, vn = 0;
+  bool ok = true;
+  while (ok && cur.next(a.seq_lens, a.capacity, sg)) {
+    const int t_begin = sg.tok_begin, t_end = sg.tok_end, n_tiles = sg.n_tiles;
+    for (int i = 0; ok && i <= n_tiles; ++i) {
+      if (i < n_tiles) {
+        const uint32_t par = static_cast<uint32_t>(g + i) & 1u;
+        ok = tc_convert_box<kTcKSlabsA>(smem + kTcOffK, kTcFp8OffA, 64, &bars->kraw[0], par, lbar(&bars->k_full[0]),
+                                        abort_flag, ct) &&
+             tc_convert_box<kTcKSlabsB>(smem + kTcOffK + kTcKSlabsA * kTcSlab, kTcFp8OffB, 64, &bars->kraw[1], par,
+                                        lbar(&bars->k_full[1]), abort_flag, ct);
+      }
+      for (int h = 0; ok && i > 0 && h < 2; ++h, ++vn) {
+        const int s = vn % kTcVSlots;
+        const int tok0 = t_begin + (i - 1) * kTcTile + 64 * h;
+        const int vcount = min(max(t_end - tok0, 0), 64);
+        ok = tc_convert_box<4>(smem + kTcOffV + s * kTcVBox, kTcFp8OffV, vcount, &bars->vraw[s],
+                               static_cast<uint32_t>(vn / kTcVSlots) & 1u, lbar(&bars->v_full[s]), abort_flag, ct);
+      }
+    }
+    g += n_tiles;
+  }
+  return ok;
+}
+
 // Each lane holds 128 bytes (w[0..31]) of its own row r = lane of a 32-row block whose rows lie
 // row_stride bytes apart from row0.  Written through a 4 KB per-warp staging buffer (16-byte
 // chunks XOR-swizzled by row, so both passes are free of bank conflicts beyond the 4 wavefronts
@@ -465,8 +651,9 @@ __device__ __forceinline__ void tc_prefetch_tile(const DecodeTcArgs& a, int b, i
   if (r < 0) return;
   int n = min(64, t_end - tok0);
   if (a.v.num_rows - r < n) n = static_cast<int>(a.v.num_rows - r);   // rows of the buffer only
-  const uint8_t* base = a.cache + r * (kDRow * 2);
-  for (int L = threadIdx.x; L < n * (kDRow * 2 / 128); L += 32 * kTcSoftmaxWarps)
+  const uint8_t* base = a.cache + r * a.row_bytes;
+  const int lines = (n * a.row_bytes + 127) / 128;
+  for (int L = threadIdx.x; L < lines; L += 32 * kTcSoftmaxWarps)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(base + 128 * L));
 }
 
@@ -843,11 +1030,13 @@ __device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacit
 // ------------------------------------------------------------------------------ kernel
 // grid = 2 * P CTAs, clusters of 2 along x: blockIdx.x = 2 * pair + rank.  kMapped: query rows
 // read the cache sequences of a.seq_map (chunked prefill); the decode instance carries none of it.
-template <bool kMapped>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
+// kFp8: the cache holds E4M3 codes with E8M0 row scales (tm_ka, tm_kb, tm_v are byte maps of the
+// codes, tm_sc the 1-D byte map of the scales; unused otherwise).
+template <bool kMapped, bool kFp8 = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc_threads(kFp8), 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_ka, const __grid_constant__ CUtensorMap tm_kb,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
-                     const DecodeTcArgs a) {
+                     const __grid_constant__ CUtensorMap tm_sc, const DecodeTcArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   TcBars* bars = reinterpret_cast<TcBars*>(smem + kTcOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kTcOffMisc);
@@ -887,6 +1076,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     mbar_init(&bars->o_free, 2 * kTcSoftmaxWarps);   // every softmax warp of both CTAs
     mbar_init(&bars->q_full, 2);
     mbar_init(&bars->q_empty, 2);   // one commit per QK^T part
+    if (kFp8) {
+      for (int part = 0; part < 2; ++part) mbar_init(&bars->kraw[part], 1);   // this CTA's producer (plus bytes)
+      for (int s = 0; s < kTcVSlots; ++s) mbar_init(&bars->vraw[s], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -899,6 +1092,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     tma_prefetch_desc(&tm_kb);
     tma_prefetch_desc(&tm_v);
     tma_prefetch_desc(&tm_q);
+    if (kFp8) tma_prefetch_desc(&tm_sc);
   }
   // The barrier inits and the TMEM allocation reach the peer CTA through the cluster barrier, whose
   // wait comes after the plan.
@@ -912,9 +1106,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
     const TcPlan w = tc_make_plan(a.seq_lens, a.capacity, a.batch, a.P, a.ws.off, pair, pair == 0 && rank == 0);
     if ((threadIdx.x & 31) == 0) *plan = w;
     __syncwarp();
-    named_bar_arrive(2, kTcThreads);
+    named_bar_arrive(2, tc_threads(kFp8));
   } else {
-    named_bar_sync(2, kTcThreads);
+    named_bar_sync(2, tc_threads(kFp8));
   }
   cluster_wait_acquire();
   tc_fence_after();
@@ -927,8 +1121,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
   } else if (warp < kTcSoftmaxWarps) {
     tc_softmax<kMapped>(a, pl, pair, smem, bars, red, tmem, rank, abort_flag);
   } else if (warp == kTcProducerWarp) {
-    if (!tc_producer<kMapped>(&tm_ka, &tm_kb, &tm_v, &tm_q, a, pl, smem, bars, rank, pair, abort_flag) &&
+    if (!tc_producer<kMapped, kFp8>(&tm_ka, &tm_kb, &tm_v, &tm_q, &tm_sc, a, pl, smem, bars, rank, pair,
+                                    abort_flag) &&
         (threadIdx.x & 31) == 0)
+      *abort_flag = 1;
+  } else if (kFp8 && warp >= kTcConvWarp0) {
+    if (!tc_convert<kMapped>(a, pl, pair, smem, bars, abort_flag) && threadIdx.x == 32 * kTcConvWarp0)
       *abort_flag = 1;
   } else if (rank == 0 && (threadIdx.x & 31) == 0) {
     bool ok = true;

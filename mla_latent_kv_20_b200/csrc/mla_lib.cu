@@ -145,6 +145,39 @@ bool make_map_vbox(CUtensorMap* map, const void* base, uint64_t rows) {
   return r == CUDA_SUCCESS;
 }
 
+// Byte views of an FP8 cache (E4M3 codes, rows of 576 bytes) with the same box shapes as the bf16
+// maps above, no swizzle (the converter warps write the swizzled bf16 layout): boxes of 64 bytes x
+// 64 rows x box_slabs slabs, laid out [slab][row][64 B]; the V box [half][chunk][row][64 B]; and
+// the scale bytes as a 1-D map with boxes of 64 rows.
+bool make_map_u8(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                 const cuuint32_t* box) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+bool make_map_u8_slabs(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_slabs) {
+  const cuuint64_t dims[3] = {64, rows, 9};
+  const cuuint64_t strides[2] = {mla::kDRow, 64};
+  const cuuint32_t box[3] = {64, 64, box_slabs};
+  return make_map_u8(map, base, 3, dims, strides, box);
+}
+bool make_map_u8_vbox(CUtensorMap* map, const void* base, uint64_t rows) {
+  const cuuint64_t dims[4] = {64, rows, 4, 2};
+  const cuuint64_t strides[3] = {mla::kDRow, 64, 256};
+  const cuuint32_t box[4] = {64, 64, 2, 2};
+  return make_map_u8(map, base, 4, dims, strides, box);
+}
+bool make_map_u8_rows(CUtensorMap* map, const void* base, uint64_t rows) {
+  const cuuint64_t dims[1] = {rows};
+  const cuuint64_t strides[1] = {1};   // not read for a rank-1 map
+  const cuuint32_t box[1] = {64};
+  return make_map_u8(map, base, 1, dims, strides, box);
+}
+
 // Validates a cache descriptor; on success fills the kernel-side view.
 mla_status check_cache(const mla_cache_desc& d, const void* cache, const int32_t* block_table, CacheView* v) {
   if (cache == nullptr || !aligned16(cache)) return MLA_ERR_INVALID_ARG;
@@ -356,6 +389,23 @@ mla_status mla_cache_append(const mla_bf16* c_new, const mla_bf16* kr_new, const
                         seq_ids, pos, reinterpret_cast<uint4*>(cache), v, rope_freq(rope_base));
 }
 
+mla_status mla_cache_append_fp8(const mla_bf16* c_new, const mla_bf16* kr_new, const int32_t* seq_ids,
+                                const int32_t* pos, uint8_t* cache, uint8_t* scales, const int32_t* block_table,
+                                mla_cache_desc desc, int32_t n_tokens, float rope_base, void* stream) {
+  if (n_tokens < 0 || !(rope_base > 0.f) || !std::isfinite(rope_base)) return MLA_ERR_INVALID_ARG;
+  CacheView v;
+  const mla_status st = check_cache(desc, cache, block_table, &v);
+  if (st != MLA_OK) return st;
+  if (n_tokens == 0) return MLA_OK;
+  if (scales == nullptr) return MLA_ERR_INVALID_ARG;
+  if (c_new == nullptr || kr_new == nullptr || pos == nullptr || !aligned16(c_new) || !aligned16(kr_new))
+    return MLA_ERR_INVALID_ARG;
+  if (seq_ids == nullptr && n_tokens > desc.num_seqs) return MLA_ERR_INVALID_ARG;
+  if (n_tokens > INT_MAX / 2) return MLA_ERR_UNSUPPORTED;
+  return launch_chained(mla::cache_append_fp8_kernel, dim3(n_tokens), dim3(96), 0, as_stream(stream),
+                        reinterpret_cast<const uint4*>(c_new), reinterpret_cast<const __nv_bfloat162*>(kr_new),
+                        seq_ids, pos, cache, scales, v, rope_freq(rope_base));
+}
 
 mla_status mla_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const mla_bf16* w_kr,
                               const int32_t* seq_ids, const int32_t* pos, mla_bf16* cache,
@@ -527,10 +577,11 @@ namespace {
 // The decode kernel and its combine over `rows` query rows: row b attends to the first
 // lens[b] cached tokens of sequence b, or of sequence seq_map[b] when a map is given (chunked
 // prefill).  Host checks shared by both entry points.
-mla_status launch_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,
+mla_status launch_attn(const mla_bf16* q_full, const void* cache, const int32_t* block_table,
                        const int32_t* lens, const int32_t* seq_map, mla_cache_desc desc, int32_t rows,
                        float softmax_scale, int32_t num_splits, void* workspace, size_t workspace_bytes,
-                       mla_bf16* out_lat, float* lse, void* stream) {
+                       mla_bf16* out_lat, float* lse, void* stream, const uint8_t* fp8_scales = nullptr) {
+  const bool fp8 = fp8_scales != nullptr;
   if (rows < 0 || num_splits < 0) return MLA_ERR_INVALID_ARG;
   if (rows > mla::kMaxDecodeBatch) return MLA_ERR_UNSUPPORTED;
   if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
@@ -539,6 +590,10 @@ mla_status launch_attn(const mla_bf16* q_full, const mla_bf16* cache, const int3
   if (st != MLA_OK) return st;
   if (rows == 0) return MLA_OK;
   if (seq_map == nullptr && rows > desc.num_seqs) return MLA_ERR_INVALID_ARG;
+  // FP8: the scale bytes of a 64-row box are copied from row y, which must be a multiple of 16
+  // (pages start at multiples of 64; a contiguous cache needs max_seq_len % 16 == 0).
+  if (fp8 && (!aligned16(fp8_scales) || (desc.page_size == 0 && desc.max_seq_len % 16 != 0)))
+    return MLA_ERR_INVALID_ARG;
   if (q_full == nullptr || lens == nullptr || out_lat == nullptr) return MLA_ERR_INVALID_ARG;
   if (!aligned16(q_full) || !aligned16(out_lat) || (lse != nullptr && !aligned16(lse))) return MLA_ERR_INVALID_ARG;
   const int capacity = cache_capacity(desc);
@@ -559,17 +614,28 @@ mla_status launch_attn(const mla_bf16* q_full, const mla_bf16* cache, const int3
   a.out_lat = reinterpret_cast<__nv_bfloat16*>(out_lat);
   a.lse = lse;
   a.cache = reinterpret_cast<const uint8_t*>(cache);
+  a.row_bytes = fp8 ? mla::kDRow : 2 * mla::kDRow;
   a.seq_map = seq_map;
-  CUtensorMap tka, tkb, tv, tq;
-  if (!make_map_slabs(&tka, cache, desc.num_rows, mla::kTcKSlabsA) ||
-      !make_map_slabs(&tkb, cache, desc.num_rows, mla::kTcKSlabsB) || !make_map_vbox(&tv, cache, desc.num_rows) ||
-      !make_map_slabs(&tq, q_full, static_cast<uint64_t>(rows) * mla::kHeads, 9))
-    return MLA_ERR_CUDA;
-  auto kernel = seq_map != nullptr ? mla::decode_tc_kernel<true> : mla::decode_tc_kernel<false>;
+  CUtensorMap tka, tkb, tv, tq, tsc;
+  if (!make_map_slabs(&tq, q_full, static_cast<uint64_t>(rows) * mla::kHeads, 9)) return MLA_ERR_CUDA;
+  if (fp8) {
+    if (!make_map_u8_slabs(&tka, cache, desc.num_rows, mla::kTcKSlabsA) ||
+        !make_map_u8_slabs(&tkb, cache, desc.num_rows, mla::kTcKSlabsB) ||
+        !make_map_u8_vbox(&tv, cache, desc.num_rows) || !make_map_u8_rows(&tsc, fp8_scales, desc.num_rows))
+      return MLA_ERR_CUDA;
+  } else {
+    if (!make_map_slabs(&tka, cache, desc.num_rows, mla::kTcKSlabsA) ||
+        !make_map_slabs(&tkb, cache, desc.num_rows, mla::kTcKSlabsB) || !make_map_vbox(&tv, cache, desc.num_rows))
+      return MLA_ERR_CUDA;
+    tsc = tq;   // unused by the bf16 instances
+  }
+  if (fp8 && seq_map != nullptr) return MLA_ERR_UNSUPPORTED;
+  auto kernel = fp8 ? mla::decode_tc_kernel<false, true>
+                    : (seq_map != nullptr ? mla::decode_tc_kernel<true> : mla::decode_tc_kernel<false>);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mla::kTcSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
-  mla_status ls = launch_chained(kernel, dim3(2 * P), dim3(mla::kTcThreads), static_cast<size_t>(mla::kTcSmemBytes), s,
-                                 tka, tkb, tv, tq, a);
+  mla_status ls = launch_chained(kernel, dim3(2 * P), dim3(mla::tc_threads(fp8)),
+                                 static_cast<size_t>(mla::kTcSmemBytes), s, tka, tkb, tv, tq, tsc, a);
   if (ls != MLA_OK) return ls;
   // Many rows (a prefill): each warp takes 8 heads of its row, so the plan is read by 8x fewer blocks.
   if (rows > 512)
@@ -589,6 +655,15 @@ mla_status mla_decode_attn(const mla_bf16* q_full, const mla_bf16* cache, const 
                            float* lse, void* stream) {
   return launch_attn(q_full, cache, block_table, seq_lens, nullptr, desc, batch, softmax_scale, num_splits, workspace,
                      workspace_bytes, out_lat, lse, stream);
+}
+
+mla_status mla_decode_attn_fp8(const mla_bf16* q_full, const uint8_t* cache, const uint8_t* scales,
+                               const int32_t* block_table, const int32_t* seq_lens, mla_cache_desc desc,
+                               int32_t batch, float softmax_scale, int32_t num_splits, void* workspace,
+                               size_t workspace_bytes, mla_bf16* out_lat, float* lse, void* stream) {
+  if (scales == nullptr) return MLA_ERR_INVALID_ARG;
+  return launch_attn(q_full, cache, block_table, seq_lens, nullptr, desc, batch, softmax_scale, num_splits, workspace,
+                     workspace_bytes, out_lat, lse, stream, scales);
 }
 
 mla_status mla_prefill_attn(const mla_bf16* q_full, const mla_bf16* cache, const int32_t* block_table,

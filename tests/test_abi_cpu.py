@@ -163,3 +163,20 @@ def test_noalloc_scratch_size_and_refusal(host_only):
                                            None) == 1
     assert mla.lib.mla_decode_attn_noalloc(FAKE, FAKE, None, FAKE, d, 0, ctypes.c_float(0.07), 0, FAKE, None,
                                            None) == 0   # empty batch: a no-op
+
+
+def test_fp8_validation(host_only):
+    """Host checks of the FP8 cache entry points (nothing is launched on these paths)."""
+    mla = host_only
+    lib = mla.lib
+    d = mla.contiguous_desc(4, 128)
+    assert lib.mla_cache_append_fp8(FAKE, FAKE, None, FAKE, FAKE, None, None, d, 4, 10000.0, None) == 1   # no scales
+    assert lib.mla_cache_append_fp8(FAKE, FAKE, None, FAKE, FAKE, FAKE, None, d, 0, 10000.0, None) == 0   # no-op
+    assert lib.mla_cache_append_fp8(FAKE, FAKE, None, FAKE, FAKE + 8, FAKE, None, d, 4, 10000.0, None) == 1
+    need = lib.mla_decode_workspace_size(4, 128, 0)
+    args = lambda desc, scales=FAKE, ws=FAKE, nbytes=need: (  # noqa: E731
+        FAKE, FAKE, scales, None, FAKE, desc, 4, 0.072, 0, ws, nbytes, FAKE, None, None)
+    assert lib.mla_decode_attn_fp8(*args(d, scales=None)) == 1               # scales are required
+    assert lib.mla_decode_attn_fp8(*args(d, scales=FAKE + 4)) == 1           # scales 16-byte aligned
+    assert lib.mla_decode_attn_fp8(*args(mla.contiguous_desc(4, 100))) == 1  # max_seq_len % 16 != 0
+    assert lib.mla_decode_attn_fp8(*args(d, nbytes=need - 16)) == 3          # workspace too small
