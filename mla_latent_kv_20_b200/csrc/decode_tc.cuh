@@ -640,7 +640,9 @@ __device__ __forceinline__ void store_rows_128b(uint8_t* stage, const uint32_t (
 // copies): this CTA's 64 rows of the tile are one contiguous 72 KB run, 576 lines over 256
 // threads, once per tile.  Contiguous caches only: with pages at permuted addresses the
 // prefetches measured slower (b32 x 4096 paged 65.6 -> 66.6 us, 128 mixed lengths paged 219 ->
-// 223 us), against 61.8 -> 58.6 and 200 -> 195 us for the same batches contiguous.
+// 223 us), against 61.8 -> 58.6 and 200 -> 195 us for the same batches contiguous; and slower
+// still with the page rows handed over by the producer from its block-id window, so that no
+// thread waits for the block table (212 -> 225 us for the batch-128 paged workload).
 constexpr int kTcPfDist = 2;
 template <bool kMapped>
 __device__ __forceinline__ void tc_prefetch_tile(const DecodeTcArgs& a, int b, int tok0, int t_end) {

@@ -28,8 +28,8 @@ constexpr int kGemmThreads = 224;    // warps 0-3: epilogue, warp 4: TMA produce
 constexpr int kGemmIssuers = 2;      // MMA-issuing warps, each with its own accumulator (summed at the end)
 constexpr int kGemmKS = 128;         // contraction rows per stage
 
-// Stage bytes: weight KS x 128 (two 64-wide M chunks) + activation nt x KS, bf16.
-__host__ __device__ constexpr int gemm_stage_bytes(int nt) { return kGemmKS * 256 + nt * kGemmKS * 2; }
+// Stage bytes: weight KS x 128 MT (2 MT 64-wide M chunks) + activation nt x KS, bf16.
+__host__ __device__ constexpr int gemm_stage_bytes(int nt, int mt = 1) { return kGemmKS * 256 * mt + nt * kGemmKS * 2; }
 
 // New tokens' cache rows written by the query-side launch (cache == nullptr: none): the rows of
 // mla_cache_append, row = [c_new[i] | RoPE(kr_new[i], pos[i])] at (seq_ids ? seq_ids[i] : i, pos[i]).
@@ -54,8 +54,12 @@ struct AppendJob {
 // null), and write the new tokens' cache rows of `app` (if any), while the MMAs run: CTA c (linear
 // index) takes work units c, c + #CTAs, ... (a unit is one new token's cache row and one group of
 // heads of one query row).
-// At most 72 registers a thread, so that four CTAs fit an SM (the absorption's 512 CTAs are one wave).
-template <int KTOT, int NSTAGE>
+// MT: 128-row M tiles per CTA.  MT = 1: the two issuing warps split the K steps into two
+// accumulators (summed in the epilogue).  MT = 2: issuing warp j computes M tile j over all K
+// steps; one CTA then loads the activation once for 256 output rows, and half as many CTAs with
+// the same TMEM per CTA (2 nt columns) fit one wave where MT = 1 needs two.
+// At most 72 registers a thread, so that four CTAs fit an SM.
+template <int KTOT, int NSTAGE, int MT = 1>
 __global__ void __launch_bounds__(kGemmThreads, 4)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      __nv_bfloat16* __restrict__ out, int batch, int nt, int64_t out_bstride,
@@ -66,7 +70,8 @@ __global__ void __launch_bounds__(kGemmThreads, 4)
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms.
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int stage_bytes = gemm_stage_bytes(nt);
+  static_assert(MT == 1 || MT == 2, "M tiles per CTA");
+  const int stage_bytes = gemm_stage_bytes(nt, MT);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + NSTAGE * stage_bytes);
   uint64_t* empty = full + NSTAGE;
   uint64_t* done = empty + NSTAGE;
@@ -75,7 +80,7 @@ __global__ void __launch_bounds__(kGemmThreads, 4)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 128;
+  const int m0 = blockIdx.x * 128 * MT;
   const int h = blockIdx.y;
   const int n0 = blockIdx.z * nt;
   const uint32_t acc_cols = nt <= 32 ? 32u : (nt <= 64 ? 64u : (nt <= 128 ? 128u : 256u));
@@ -121,7 +126,7 @@ __global__ void __launch_bounds__(kGemmThreads, 4)
       }
       if (*reinterpret_cast<volatile int*>(abort_flag)) break;
       uint8_t* sa = smem + s * stage_bytes;
-      uint8_t* sb = sa + kGemmKS * 256;
+      uint8_t* sb = sa + kGemmKS * 256 * MT;
       mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(stage_bytes));
       const int krow = h * KTOT + ks * kGemmKS;
       tma_load_3d(sa, &tmA, &full[s], 0, krow, m0 / 64);
@@ -147,11 +152,15 @@ __global__ void __launch_bounds__(kGemmThreads, 4)
       }
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + s * stage_bytes);
-      const uint32_t sb = sa + kGemmKS * 256;
+      const uint32_t sb = sa + kGemmKS * 256 * MT;
+      // MT = 1: this warp's K steps (kk = j, j + 2, ...); MT = 2: every K step of M tile j, whose
+      // two 64-wide M chunks start 2 j chunks into the stage.
+      const uint32_t sa_t = MT == 1 ? sa : sa + j * 2 * kGemmKS * 128;
+      constexpr int kStep = MT == 1 ? kGemmIssuers : 1;
 #pragma unroll
-      for (int kk = j; kk < kGemmKS / 16; kk += kGemmIssuers) {
+      for (int kk = (MT == 1 ? j : 0); kk < kGemmKS / 16; kk += kStep) {
         // A (MN-major): 16 K rows per MMA = 2 swizzle atoms of 1024 B; M chunks KS * 128 B apart.
-        const uint64_t adesc = sdesc_sw128(sa + kk * 2048, kGemmKS * 128, 1024);
+        const uint64_t adesc = sdesc_sw128(sa_t + kk * 2048, kGemmKS * 128, 1024);
         // B (K-major): slab kk / 4 of nt rows x 128 B; 16 K elements = 32 B into each row.
         const uint64_t bdesc = sdesc_sw128(sb + (kk >> 2) * nt * 128 + (kk & 3) * 32, 16, 1024);
         umma_bf16_ss(acc, adesc, bdesc, idesc, first ? 0u : 1u);
@@ -250,24 +259,29 @@ __global__ void __launch_bounds__(kGemmThreads, 4)
     if (ok && !*reinterpret_cast<volatile int*>(abort_flag)) {
       const uint32_t trow = tmem_d + (static_cast<uint32_t>(warp * 32) << 16);
       __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem + warp * nt * 64);
-      for (int c = 0; c < nt; c += 16) {
-        uint32_t r0[16], r1[16];
-        tmem_ld16(trow + c, r0);
-        tmem_ld16(trow + acc_cols + c, r1);
-        tmem_ld_wait();
+#pragma unroll 1
+      for (int mtile = 0; mtile < MT; ++mtile) {
+        if (mtile > 0) __syncwarp();   // the previous tile's stores have read the stage
+        for (int c = 0; c < nt; c += 16) {
+          uint32_t r0[16], r1[16];
+          tmem_ld16(trow + (MT == 1 ? 0u : mtile * acc_cols) + c, r0);
+          if (MT == 1) tmem_ld16(trow + acc_cols + c, r1);
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          stage[(c + i) * 32 + lane] = __float2bfloat16_rn(__uint_as_float(r0[i]) + __uint_as_float(r1[i]));
-      }
-      __syncwarp();
-      const int q = lane & 3;   // 16-byte piece (8 outputs) of a 64-byte row
-      for (int n8 = 0; n8 < nt; n8 += 8) {
-        const int nl = n8 + (lane >> 2);
-        const int n = n0 + nl;
-        if (n < batch) {
-          const uint4 v = *reinterpret_cast<const uint4*>(stage + nl * 32 + 8 * q);
-          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * out_bstride + static_cast<int64_t>(h) * out_hstride +
-                                    m0 + warp * 32 + 8 * q) = v;
+          for (int i = 0; i < 16; ++i)
+            stage[(c + i) * 32 + lane] =
+                __float2bfloat16_rn(MT == 1 ? __uint_as_float(r0[i]) + __uint_as_float(r1[i]) : __uint_as_float(r0[i]));
+        }
+        __syncwarp();
+        const int q = lane & 3;   // 16-byte piece (8 outputs) of a 64-byte row
+        for (int n8 = 0; n8 < nt; n8 += 8) {
+          const int nl = n8 + (lane >> 2);
+          const int n = n0 + nl;
+          if (n < batch) {
+            const uint4 v = *reinterpret_cast<const uint4*>(stage + nl * 32 + 8 * q);
+            *reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * out_bstride +
+                                      static_cast<int64_t>(h) * out_hstride + m0 + 128 * mtile + warp * 32 + 8 * q) = v;
+          }
         }
       }
     }

@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -449,21 +450,21 @@ mla_status mla_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y
 
 namespace {
 
-template <int KTOT, int NSTAGE>
+template <int KTOT, int NSTAGE, int MT = 1>
 mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, int batch, __nv_bfloat16* out,
                             int64_t out_bstride, int out_hstride, cudaStream_t stream, const void* qpe = nullptr,
                             const int32_t* q_pos = nullptr, float rope_base = 10000.f,
-                            const mla::AppendJob* app = nullptr) {
+                            const mla::AppendJob* app = nullptr, int nt_cap = 256) {
   // Weight viewed as [heads * KTOT rows][m_total cols]: 3-D (64-element M chunk, row, M chunk index),
   // box {64, KS, 2}.  Activation as [batch rows][heads * KTOT cols]: 3-D (64-element K slab, batch
   // row, slab index), box {64, nt, KS / 64}.
-  const int nt = batch >= 256 ? 256 : ((batch + 15) / 16) * 16;
+  const int nt = std::min(batch >= 256 ? 256 : ((batch + 15) / 16) * 16, nt_cap);
   const uint64_t krows = static_cast<uint64_t>(mla::kHeads) * KTOT;
   CUtensorMap ta, tb;
   {
     const cuuint64_t dims[3] = {64, krows, static_cast<cuuint64_t>(m_total / 64)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(m_total) * 2, 128};
-    const cuuint32_t box[3] = {64, mla::kGemmKS, 2};
+    const cuuint32_t box[3] = {64, mla::kGemmKS, 2 * MT};
     if (!make_map_3d(&ta, weight, dims, strides, box)) return MLA_ERR_CUDA;
   }
   {
@@ -473,15 +474,30 @@ mla_status launch_proj_gemm(const void* weight, int m_total, const void* act, in
     if (!make_map_3d(&tb, act, dims, strides, box)) return MLA_ERR_CUDA;
   }
   // ring, barriers, TMEM slot and flag, then the 32 (cos, sin) pairs of the q_pe rotation
-  const size_t smem = 1024 + NSTAGE * mla::gemm_stage_bytes(nt) + (2 * NSTAGE + 1) * 8 + 16 + 32 * 16;
-  auto kern = mla::proj_gemm_kernel<KTOT, NSTAGE>;
+  const size_t smem = 1024 + NSTAGE * mla::gemm_stage_bytes(nt, MT) + (2 * NSTAGE + 1) * 8 + 16 + 32 * 16;
+  auto kern = mla::proj_gemm_kernel<KTOT, NSTAGE, MT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return MLA_ERR_CUDA;
-  dim3 grid(m_total / 128, mla::kHeads, (batch + nt - 1) / nt);
+  dim3 grid(m_total / (128 * MT), mla::kHeads, (batch + nt - 1) / nt);
   return launch_chained(kern, grid, dim3(mla::kGemmThreads), smem, stream, ta, tb, out, batch, nt, out_bstride,
                         out_hstride, reinterpret_cast<const uint4*>(qpe), q_pos, rope_freq(rope_base),
                         app != nullptr ? *app : mla::AppendJob{nullptr, nullptr, nullptr, nullptr, nullptr, {}, 0});
+}
+
+// The W_UK GEMM of the query absorption (optionally with the cache append of `app`): two 128-row M
+// tiles per CTA for batches of 65..128 rows (256 CTAs in one wave where 512 of one tile took two:
+// 16.2 -> 14.8 us at 128 rows, weights cold), one otherwise (at 64 rows and below two tiles per
+// CTA measured no faster).
+mla_status launch_absorb(const mla_bf16* w_uk, const mla_bf16* q_nope, int batch, mla_bf16* q_full, cudaStream_t s,
+                         const mla_bf16* q_pe, const int32_t* q_pos, float rope_base, const mla::AppendJob* app) {
+  auto* qf = reinterpret_cast<__nv_bfloat16*>(q_full);
+  const int64_t bstride = static_cast<int64_t>(mla::kHeads) * mla::kDRow;
+  if (batch > 64 && batch <= 128)
+    return launch_proj_gemm<mla::kDHead, 1, 2>(w_uk, mla::kDLat, q_nope, batch, qf, bstride, mla::kDRow, s, q_pe, q_pos,
+                                               rope_base, app);
+  return launch_proj_gemm<mla::kDHead, 1, 1>(w_uk, mla::kDLat, q_nope, batch, qf, bstride, mla::kDRow, s, q_pe, q_pos,
+                                             rope_base, app);
 }
 
 }  // namespace
@@ -497,11 +513,9 @@ mla_status mla_absorb_q(const mla_bf16* q_nope, const mla_bf16* q_pe, const int3
   if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(w_uk) || !aligned16(q_full)) return MLA_ERR_INVALID_ARG;
   if (q_pos != nullptr && (!(rope_base > 0.f) || !std::isfinite(rope_base))) return MLA_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
-  // One launch: the W_UK GEMM fills q_full[:, :, 0:512] and its M-tile-0 CTAs rotate q_pe into
-  // q_full[:, :, 512:576].
-  return launch_proj_gemm<mla::kDHead, 1>(w_uk, mla::kDLat, q_nope, batch, reinterpret_cast<__nv_bfloat16*>(q_full),
-                                          static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow, s, q_pe, q_pos,
-                                          rope_base);
+  // One launch: the W_UK GEMM fills q_full[:, :, 0:512] and its CTAs rotate q_pe into
+  // q_full[:, :, 512:576] meanwhile.
+  return launch_absorb(w_uk, q_nope, batch, q_full, s, q_pe, q_pos, rope_base, nullptr);
 }
 
 mla_status mla_append_absorb(const mla_bf16* c_new, const mla_bf16* kr_new, const int32_t* seq_ids,
@@ -527,9 +541,7 @@ mla_status mla_append_absorb(const mla_bf16* c_new, const mla_bf16* kr_new, cons
   if (!aligned16(q_nope) || !aligned16(q_pe) || !aligned16(w_uk) || !aligned16(q_full)) return MLA_ERR_INVALID_ARG;
   const mla::AppendJob app{reinterpret_cast<const uint4*>(c_new), reinterpret_cast<const __nv_bfloat162*>(kr_new),
                            seq_ids, pos, reinterpret_cast<uint4*>(cache), v, n_tokens};
-  return launch_proj_gemm<mla::kDHead, 1>(w_uk, mla::kDLat, q_nope, batch, reinterpret_cast<__nv_bfloat16*>(q_full),
-                                          static_cast<int64_t>(mla::kHeads) * mla::kDRow, mla::kDRow,
-                                          as_stream(stream), q_pe, q_pos, rope_base, &app);
+  return launch_absorb(w_uk, q_nope, batch, q_full, as_stream(stream), q_pe, q_pos, rope_base, &app);
 }
 
 mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf16* out, int32_t batch,
@@ -540,7 +552,8 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
   if (!aligned16(out_lat) || !aligned16(w_uv) || !aligned16(out)) return MLA_ERR_INVALID_ARG;
   // One CTA per head streams that head's 128 KB of W_UV in four 128-row stages: with a batch of up
   // to 64 rows all four stages fit in shared memory and are requested at once (one HBM round trip);
-  // larger batches (larger stages) go through a two-stage ring.
+  // larger batches (larger stages) go through a two-stage ring.  (Two 64-row N tiles per head for
+  // batches of 65..128 rows, 256 CTAs, measured no faster.)
   if (batch <= 64)
     return launch_proj_gemm<mla::kDLat, 4>(w_uv, mla::kDHead, out_lat, batch, reinterpret_cast<__nv_bfloat16*>(out),
                                            static_cast<int64_t>(mla::kHeads) * mla::kDHead, mla::kDHead,
