@@ -89,7 +89,7 @@ def test_append_out_of_range_is_reported_not_written(env):
 
 
 # ----------------------------------------------------------------------------- projections
-@pytest.mark.parametrize("batch", [1, 5, 32, 300])
+@pytest.mark.parametrize("batch", [1, 5, 32, 100, 128, 300])   # 65..128 rows take two M tiles per CTA
 def test_absorb_q(env, batch):
     m, hz, torch = env
     w = mi.layer_weights(200)
@@ -224,7 +224,8 @@ def test_full_step_vs_explicit_oracle(env, lens, paged):
 
 
 # ----------------------------------------------------------------------------- fused append + absorb
-@pytest.mark.parametrize("paged,n_tokens,batch", [(False, 4, 4), (True, 4, 4), (False, 7, 3), (True, 2, 33)])
+@pytest.mark.parametrize("paged,n_tokens,batch", [(False, 4, 4), (True, 4, 4), (False, 7, 3), (True, 2, 33),
+                                                   (True, 40, 128)])
 def test_append_absorb_equals_separate_calls(env, paged, n_tokens, batch):
     """mla_append_absorb writes exactly the rows of mla_cache_append and the q_full of mla_absorb_q."""
     m, hz, torch = env
