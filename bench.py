@@ -310,7 +310,8 @@ def setup_replica(name, device, splits=0):
 # ncu capture per workload, keyed by the SHA-256 of the sources that build those kernels and
 # choose their launch shape.  A digest that no longer matches means the kernels changed since the
 # counters were taken, and the traffic is reported as null.
-TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh", "csrc/mla_lib.cu")
+TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh", "csrc/append.cuh",
+                   "csrc/decode_launch.cuh")
 MEASURED_TRAFFIC = {   # workload -> {"bytes": int, "sha256": str, "profile": str}
     "b32_l4096": {"bytes": 155800320 + 3449344 + 16858880, "sha256": "d2d222cae8eb16d5ba01634a13f5b483c3a047b20bbfdaf4e77e73e9e52a37bb",
                   "profile": "profiles/decode_tc_b32_l4096.md (decode + combine, ncu cache flush per kernel)"},
