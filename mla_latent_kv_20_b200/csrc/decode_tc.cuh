@@ -36,8 +36,9 @@
 //
 // Warp roles (416 threads): warps 0-7 softmax / O correction / epilogue (two warps per TMEM lane
 // quadrant, each owning half of the S columns), warp 8 work plan and TMA producer, and in the
-// even CTA only: warp 9 QK^T part A (warp 9 also allocates TMEM in both CTAs), warp 11 QK^T part
-// B, warps 10 and 12 PV for the two latent halves.
+// even CTA only: warps 9 and 11 QK^T, each the 16-deep K steps of its parity into its own S
+// accumulator (warp 9 also allocates TMEM in both CTAs), warps 10 and 12 PV for the two latent
+// halves.
 //
 // FP8 cache (kFp8, 544 threads).  Rows are 576 E4M3 codes with a power-of-two scale per token (an
 // E8M0 exponent byte, 2^(e - 127)): code * scale is exact in bf16, so the MMAs, the softmax and
@@ -81,16 +82,17 @@ constexpr int kTcOffBar = kTcOffV + kTcVSlots * kTcVBox;
 constexpr int kTcOffMisc = kTcOffBar + 256;
 constexpr int kTcSmemBytes = kTcOffMisc + 64 + 2 * 256 * 4;   // the dynamic base is 1024-aligned (checked)
 
-// TMEM columns of each CTA (512 allocated): S part A (2 buffers x 64), S part B (2 x 64), O (256).
+// TMEM columns of each CTA (512 allocated): S of QK^T issuer 0 (2 buffers x 64), of issuer 1
+// (2 x 64), O (256).
 constexpr uint32_t kTcColSA = 0;
 constexpr uint32_t kTcColSB = 128;
 constexpr uint32_t kTcColO = 256;
 
 constexpr int kTcSoftmaxWarps = 8;
 constexpr int kTcProducerWarp = 8;
-constexpr int kTcMmaWarp = 9;     // TMEM allocation (both CTAs); QK^T part A issue (even CTA)
+constexpr int kTcMmaWarp = 9;     // TMEM allocation (both CTAs); QK^T even K steps (even CTA)
 constexpr int kTcPvWarp = 10;     // PV issue, first latent half (even CTA)
-constexpr int kTcMmaBWarp = 11;   // QK^T part B issue (even CTA)
+constexpr int kTcMmaBWarp = 11;   // QK^T odd K steps (even CTA)
 constexpr int kTcPv1Warp = 12;    // PV issue, second latent half (even CTA)
 constexpr int kTcThreads = 32 * (kTcSoftmaxWarps + 5);
 // FP8 cache: four converter warps after the others.
@@ -128,7 +130,7 @@ struct TcPlan {
 
 struct TcBars {
   uint64_t k_full[2];            // even CTA only, per QK^T part: both CTAs' K boxes landed (one arrival per CTA + tx)
-  uint64_t k_empty[2];           // both CTAs, per part: K box consumed by the MMAs
+  uint64_t k_empty[2];           // both CTAs, per part: K box consumed by the MMAs (one commit per QK^T issuer)
   uint64_t v_full[kTcVSlots];    // even CTA only: both CTAs' V box landed (one arrival per CTA + tx)
   uint64_t v_empty[kTcVSlots];   // both CTAs: V box consumed (one commit per PV warp)
   uint64_t fix;                  // per CTA: local load of a ragged V box
@@ -420,38 +422,42 @@ __device__ bool tc_producer(const CUtensorMap* tm_ka, const CUtensorMap* tm_kb, 
 // never carries out of the field.
 __device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
-// S_part(g) = Q[:, dims of part] . K(g)[:, dims of part]^T into S buffer g & 1 of the part, for
-// every global tile g of the range; Q is reloaded for each segment.
-__device__ bool tc_mma_qk(uint8_t* smem, TcBars* bars, uint32_t tmem, int part, const int32_t* seq_lens,
-                          int capacity, SegmentCursor cur, volatile int* abort_flag) {
+// S_j(g) = the sum over the 16-deep K steps (slab c, step kk) with kk % 2 == j of Q . K(g)^T, into
+// S buffer g & 1 of issuer j (the softmax adds S_0 + S_1), for every global tile g of the range; Q
+// is reloaded for each segment.  Both issuers walk the part-A slabs (0-4) first and then part B's
+// (5-8), so part A's K slot is released halfway through the tile's QK^T (its next copy then
+// overlaps the second half and PV) and QK^T of the next tile needs part B's copy only halfway in.
+__device__ bool tc_mma_qk(uint8_t* smem, TcBars* bars, uint32_t tmem, int j, const int32_t* seq_lens, int capacity,
+                          SegmentCursor cur, volatile int* abort_flag) {
   const uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-  const int slab0 = tc_part_slab0(part);
-  const int nslabs = tc_part_slabs(part);
-  const uint64_t dq = sdesc_sw128(smem_u32(smem + kTcOffQ + slab0 * kTcSlab), 16, 1024);
-  const uint64_t dk = sdesc_sw128(smem_u32(smem + kTcOffK + slab0 * kTcSlab), 16, 1024);
-  const uint32_t scol = tmem + (part ? kTcColSB : kTcColSA);
+  const uint64_t dq = sdesc_sw128(smem_u32(smem + kTcOffQ), 16, 1024);
+  const uint64_t dk = sdesc_sw128(smem_u32(smem + kTcOffK), 16, 1024);
+  const uint32_t scol = tmem + (j ? kTcColSB : kTcColSA);
   Segment sg;
   int g = 0, k = 0;
   while (cur.next(seq_lens, capacity, sg)) {
     if (!mbar_wait_cluster(&bars->q_full, static_cast<uint32_t>(k) & 1u, 0x20)) return false;
     for (int i = 0; i < sg.n_tiles; ++i, ++g) {
-      const int j = g & 1;
-      // S buffer j last held tile g - 2: every softmax warp of both CTAs must have read it.
-      if (g >= 2 && !mbar_wait_cluster(&bars->s_empty[j], static_cast<uint32_t>((g - 2) >> 1) & 1u, 0x24))
+      const uint32_t sb = scol + 64 * (g & 1);
+      // S buffer g & 1 last held tile g - 2: every softmax warp of both CTAs must have read it.
+      if (g >= 2 && !mbar_wait_cluster(&bars->s_empty[g & 1], static_cast<uint32_t>((g - 2) >> 1) & 1u, 0x24))
         return false;
-      if (!mbar_wait_cluster(&bars->k_full[part], static_cast<uint32_t>(g) & 1u, 0x21)) return false;
-      tc_fence_after();
-      // Fully unrolled (the issue rate of this thread bounds the tensor pipe here): every
-      // descriptor is a constant offset from the part's base.
 #pragma unroll
-      for (int c = 0; c < kTcKSlabsA; ++c)
+      for (int part = 0; part < 2; ++part) {
+        if (!mbar_wait_cluster(&bars->k_full[part], static_cast<uint32_t>(g) & 1u, 0x21)) return false;
+        tc_fence_after();
+        // Fully unrolled (the issue rate of this thread bounds the tensor pipe here): every
+        // descriptor is a constant offset from the base.
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          if (c < nslabs)
-            umma_bf16_pair(scol + 64 * j, sdesc_add(dq, c * kTcSlab + 32 * kk), sdesc_add(dk, c * kTcSlab + 32 * kk),
-                           idesc_qk, (c | kk) != 0 ? 1u : 0u);
-      umma_commit_pair_mc(&bars->k_empty[part], 3);
-      umma_commit_pair_mc(&bars->s_full[j], 3);
+        for (int c = tc_part_slab0(part); c < tc_part_slab0(part) + tc_part_slabs(part); ++c)
+#pragma unroll
+          for (int kk = 0; kk < 4; kk += 2) {
+            const uint32_t off = c * kTcSlab + 32 * (kk + j);
+            umma_bf16_pair(sb, sdesc_add(dq, off), sdesc_add(dk, off), idesc_qk, (c | kk) != 0 ? 1u : 0u);
+          }
+        umma_commit_pair_mc(&bars->k_empty[part], 3);
+      }
+      umma_commit_pair_mc(&bars->s_full[g & 1], 3);
       if (*abort_flag) return false;
     }
     umma_commit_pair_mc(&bars->q_empty, 3);   // Q of this segment no longer read
@@ -775,7 +781,7 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
       break;
     }
     tc_fence_after();
-    // S = S_A + S_B (the two QK^T parts over disjoint dims).
+    // S = S_0 + S_1 (the two QK^T issuers' sums over disjoint K steps).
     float sc[32];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -1060,7 +1066,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc_threads(kFp8), 1)
   if (threadIdx.x == 0) {
     for (int part = 0; part < 2; ++part) {
       mbar_init(&bars->k_full[part], 2);   // one arrival per CTA of the pair (plus the copies' bytes)
-      mbar_init(&bars->k_empty[part], 1);
+      mbar_init(&bars->k_empty[part], 2);   // one commit per QK^T issuer
     }
     for (int s = 0; s < kTcVSlots; ++s) {
       mbar_init(&bars->v_full[s], 2);   // one arrival per CTA of the pair (plus the copies' bytes)
