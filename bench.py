@@ -312,9 +312,15 @@ def setup_replica(name, device, splits=0):
 # counters were taken, and the traffic is reported as null.
 TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh", "csrc/append.cuh",
                    "csrc/decode_launch.cuh")
-MEASURED_TRAFFIC = {   # workload -> {"bytes": int, "sha256": str, "profile": str}
-    "b32_l4096": {"bytes": 155800320 + 3449344 + 16858880, "sha256": "d2d222cae8eb16d5ba01634a13f5b483c3a047b20bbfdaf4e77e73e9e52a37bb",
-                  "profile": "profiles/decode_tc_b32_l4096.md (decode + combine, ncu cache flush per kernel)"},
+MEASURED_TRAFFIC = {   # workload[@ranges] -> {"bytes": int, "sha256": str, "profile": str}
+    "b128_u1024_8192_paged": {
+        "bytes": 693064192 + 27741184 + 37912832,
+        "sha256": "86b9eb1ac8b66e99ad9405569e62e03a92b23b9a3adebbfdf528ddb344c3adf3",
+        "profile": "profiles/decode_tc_b128_u1024_8192_paged.md (decode + combine, ncu cache flush per kernel)"},
+    "b32_l4096": {
+        "bytes": 155815936 + 3915776 + 16858624,
+        "sha256": "86b9eb1ac8b66e99ad9405569e62e03a92b23b9a3adebbfdf528ddb344c3adf3",
+        "profile": "profiles/decode_tc_b32_l4096.md (decode + combine, ncu cache flush per kernel)"},
 }
 
 
