@@ -664,13 +664,39 @@ def hz_bits(t):
     return hz.bf16_bits(t)
 
 
+SEG_COST = 2   # tiles' worth of cost a segment start adds in the balanced plan (the decode plan's kSegCost)
+
+
+def plan_bounds(tiles, P):
+    """First global tile of each of the P ranges of the balanced plan, and T: the tiles of the
+    batch laid end to end, a non-empty sequence costing SEG_COST + its tiles on a cost line that
+    is cut into P pieces of equal cost; a cut inside a sequence's segment charge moves to the
+    sequence's first tile."""
+    T = sum(tiles)
+    C = sum(t + SEG_COST for t in tiles if t > 0)
+    bounds = []
+    for p in range(P + 1):
+        x = p * C // P
+        W, off, b = 0, 0, T
+        for t in tiles:
+            if t == 0:
+                continue
+            if x < W + SEG_COST + t:
+                b = off + max(0, x - W - SEG_COST)
+                break
+            W += SEG_COST + t
+            off += t
+        bounds.append(b)
+    return bounds
+
+
 def partial_segments(lens, P):
     """Range partials one decode call writes (and its combine reads back) under the work plan:
     with the per-sequence plan (every non-empty sequence has at least T/P of the T tiles) sequence
     b gets r_b = min(floor(P tiles_b / T), tiles_b) ranges and contributes r_b partials when r_b > 1;
-    otherwise the tiles are laid end to end and range p takes [floor(pT/P), floor((p+1)T/P)),
-    and every range that does not cover the whole of a sequence it meets writes a partial of
-    that sequence.  Used only to report the partials' bytes."""
+    otherwise the balanced plan (plan_bounds) cuts the tiles laid end to end into P ranges, and
+    every range that does not cover the whole of a sequence it meets writes a partial of that
+    sequence.  Used only to report the partials' bytes."""
     tiles = [(int(L) + 127) // 128 for L in lens]
     T = sum(tiles)
     if T == 0:
@@ -682,15 +708,15 @@ def partial_segments(lens, P):
             r = min(P * t // T, t)
             n += r if r > 1 else 0
         return n
+    starts = plan_bounds(tiles, P)
     n, run = 0, 0
-    starts = [p * T // P for p in range(P + 1)]
     for t in tiles:
         if t == 0:
             continue
-        first = next(p for p in range(P) if starts[p] <= run < starts[p + 1])
-        last = next(p for p in range(P) if starts[p] <= run + t - 1 < starts[p + 1])
+        first = max(p for p in range(P) if starts[p] <= run)
+        last = max(p for p in range(P) if starts[p] <= run + t - 1)
         if last > first:
-            n += last - first + 1
+            n += sum(1 for p in range(first, last + 1) if starts[p] < starts[p + 1])
         run += t
     return n
 

@@ -12,7 +12,14 @@
 //    r_b = floor(P tiles_b / T) >= 1 ranges that split its tiles evenly, so every range holds one
 //    piece of one sequence (pairs beyond sum r_b stay idle);
 //  * balanced (otherwise): the tiles of the batch are laid end to end (sequence b owns global
-//    tiles [off_b, off_b + tiles_b)) and range p takes [floor(p T / P), floor((p + 1) T / P));
+//    tiles [off_b, off_b + tiles_b)) and the ranges cut that line into P pieces of equal cost,
+//    where a non-empty sequence costs kSegCost + tiles_b: a range spends a few tiles' worth of
+//    time at each segment it starts (the new Q, the pipeline refill, the epilogue of the previous
+//    segment), so a range that meets more sequences takes fewer tiles.  On the cost line sequence
+//    b spans [W_b, W_b + kSegCost + tiles_b) (W_b the sum over earlier non-empty sequences); the
+//    boundary x_p = floor(p C / P) (C the total cost) falls in one such span and becomes global
+//    tile off_b + max(0, x_p - W_b - kSegCost) (off_b itself when it falls in the sequence's
+//    segment charge), or T when p = P.  Range p takes tiles [bound_p, bound_{p+1}) (possibly none);
 //    the part of each sequence a range touches is a segment.
 // A segment that covers its whole sequence is finished by the decode kernel; otherwise (in the
 // balanced plan at most the first and the last segment of a range) its partial goes to
@@ -28,35 +35,44 @@
 namespace mla {
 
 constexpr int kTile = 128;               // tokens per tile of the work plan and of the decode kernel
+// What a segment start costs a range in the balanced plan, in tiles: the decode kernel's range
+// time fits 5.1 us per segment against 2.7 us per steady-state tile (per-tile timestamps, batch
+// 128 with lengths uniform in [1024, 8192]).
+constexpr int kSegCost = 2;
 constexpr int kMaxDecodeBatch = 16384;   // sequences per decode call (the plan's prefix fits in smem)
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // Workspace layout for P work ranges and `batch` sequences:
-//   O    [2P][128][512] fp32   (unnormalised partial sums of c)
-//   m    [2P][128]      fp32   (running max, log2 domain)
-//   l    [2P][128]      fp32   (running sum of exp2(s - m))
-//   plan [batch + 2]    int32  (balanced: global tile offset of each sequence, [batch] = T;
-//                               per sequence: first range of each sequence, [batch] = ranges used;
-//                               [batch + 1] = the plan kind)
+//   O      [2P][128][512] fp32   (unnormalised partial sums of c)
+//   m      [2P][128]      fp32   (running max, log2 domain)
+//   l      [2P][128]      fp32   (running sum of exp2(s - m))
+//   bounds [P + 1]        int32  (balanced plan: first global tile of each range, [P] = T;
+//                                 written by the decode kernel; padded to a multiple of 4)
+//   plan   [batch + 2]    int32  (balanced: global tile offset of each sequence, [batch] = T;
+//                                 per sequence: first range of each sequence, [batch] = ranges used;
+//                                 [batch + 1] = the plan kind)
 struct Workspace {
   float* o;
   float* m;
   float* l;
-  int32_t* off;
+  int32_t* off;   // the plan table; the range bounds sit just before it (ws_bounds)
 };
+__host__ __device__ __forceinline__ int ws_bounds_ints(int P) { return (P + 1 + 3) / 4 * 4; }
 __host__ __device__ __forceinline__ Workspace ws_carve(void* base, int P) {
   Workspace w;
   w.o = reinterpret_cast<float*>(base);
   w.m = w.o + static_cast<int64_t>(2 * P) * kHeads * kDLat;
   w.l = w.m + static_cast<int64_t>(2 * P) * kHeads;
-  w.off = reinterpret_cast<int32_t*>(w.l + static_cast<int64_t>(2 * P) * kHeads);
+  w.off = reinterpret_cast<int32_t*>(w.l + static_cast<int64_t>(2 * P) * kHeads) + ws_bounds_ints(P);
   return w;
 }
+__host__ __device__ __forceinline__ int32_t* ws_bounds(const Workspace& w, int P) { return w.off - ws_bounds_ints(P); }
 __host__ __device__ __forceinline__ size_t ws_bytes(int batch, int P) {
   const size_t partials = static_cast<size_t>(2 * P) * kHeads * (kDLat + 2) * sizeof(float);
-  return partials + ((static_cast<size_t>(batch) + 2) * sizeof(int32_t) + 15) / 16 * 16;
+  return partials + static_cast<size_t>(ws_bounds_ints(P)) * sizeof(int32_t) +
+         ((static_cast<size_t>(batch) + 2) * sizeof(int32_t) + 15) / 16 * 16;
 }
 
 // Effective length of sequence b: seq_lens[b] clamped to [0, capacity] (error word set if it
@@ -80,14 +96,15 @@ __host__ __device__ __forceinline__ int muldiv(int x, int y, int z) {
   return muldiv_wide(p, static_cast<uint32_t>(z));
 }
 
-// First global tile of work range p (of P) over T tiles.
-__host__ __device__ __forceinline__ int range_start(int p, int P, int T) { return muldiv(p, T, P); }
-// The (non-empty) range that holds global tile t: the last p with range_start(p) <= t.
-__host__ __device__ __forceinline__ int range_of_tile(int t, int P, int T) {
-  // ceil((t + 1) P / T) - 1
-  const uint64_t x = static_cast<uint64_t>(t + 1) * static_cast<uint32_t>(P) + static_cast<uint32_t>(T - 1);
-  if (x <= 0xffffffffull) return static_cast<int>(static_cast<uint32_t>(x) / static_cast<uint32_t>(T)) - 1;
-  return muldiv_wide(x, static_cast<uint32_t>(T)) - 1;
+// The (non-empty) range of the balanced plan that holds global tile t (0 <= t < T): the last p
+// with bounds[p] <= t, by bisection over the P + 1 ascending bounds.
+__device__ __forceinline__ int range_of_tile(const int32_t* bounds, int t, int P) {
+  int lo = 0, hi = P - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (bounds[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 constexpr int kPlanBalanced = 0;
@@ -158,7 +175,6 @@ __global__ void __launch_bounds__(128, hpw == 1 ? 8 : 4) combine_kernel(Workspac
   const int lane = threadIdx.x & 31;
   const int B = gridDim.x;
   const bool per_seq = ws.off[B + 1] == kPlanPerSequence;
-  const int T = ws.off[B];
   const int off = ws.off[b];
   const int span = ws.off[b + 1] - off;   // tiles (balanced) or ranges (per sequence) of b
   if (span == 0) {
@@ -170,68 +186,77 @@ __global__ void __launch_bounds__(128, hpw == 1 ? 8 : 4) combine_kernel(Workspac
     return;
   }
   // Ranges [p0, p1] that hold pieces of b; in the per-sequence plan each holds one (slot 2p).
-  const int p0 = per_seq ? off : range_of_tile(off, P, T);
-  const int p1 = per_seq ? off + span - 1 : range_of_tile(off + span - 1, P, T);
+  const int p0 = per_seq ? off : range_of_tile(ws_bounds(ws, P), off, P);
+  const int p1 = per_seq ? off + span - 1 : range_of_tile(ws_bounds(ws, P), off + span - 1, P);
   if (p0 == p1) return;
-  auto slot_of = [&](int p) { return (!per_seq && range_start(p, P, T) < off) ? 2 * p + 1 : 2 * p; };
-  auto nonempty = [&](int p) { return per_seq || range_start(p, P, T) < range_start(p + 1, P, T); };
+  // The merge over the ranges, with the slot and emptiness of range p given by the plan kind (two
+  // copies of the loop, so that each keeps only what its kind needs live).
+  auto merge_rows = [&](auto slot_of, auto nonempty) {
 #pragma unroll 1
-  for (int h = h0; h < h0 + hpw; ++h) {
-    __nv_bfloat16* dst = out_lat + (static_cast<int64_t>(b) * kHeads + h) * kDLat;
-    // Online merge in ascending range order: after each range, (M, den, acc) hold the merge of the
-    // ranges so far relative to M.  Two ranges are fetched per step so their loads overlap (every
-    // partial's m is finite: a non-empty range holds at least one valid token of b).
-    float M = -INFINITY, den = 0.f;
-    float acc[16];
+    for (int h = h0; h < h0 + hpw; ++h) {
+      __nv_bfloat16* dst = out_lat + (static_cast<int64_t>(b) * kHeads + h) * kDLat;
+      // Online merge in ascending range order: after each range, (M, den, acc) hold the merge of the
+      // ranges so far relative to M.  Two ranges are fetched per step so their loads overlap (every
+      // partial's m is finite: a non-empty range holds at least one valid token of b).
+      float M = -INFINITY, den = 0.f;
+      float acc[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-    auto fetch = [&](int p, float& m, float& l, float4 (&o)[4]) -> bool {
-      if (p > p1 || !nonempty(p)) return false;
-      const int64_t ml = static_cast<int64_t>(slot_of(p)) * kHeads + h;
-      m = ws.m[ml];
-      l = ws.l[ml];
-      const float4* src = reinterpret_cast<const float4*>(ws.o + ml * kDLat);
+      for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+      auto fetch = [&](int p, float& m, float& l, float4 (&o)[4]) -> bool {
+        if (p > p1 || !nonempty(p)) return false;
+        const int64_t ml = static_cast<int64_t>(slot_of(p)) * kHeads + h;
+        m = ws.m[ml];
+        l = ws.l[ml];
+        const float4* src = reinterpret_cast<const float4*>(ws.o + ml * kDLat);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) o[i] = src[lane + 32 * i];
-      return true;
-    };
-    auto merge = [&](float m, float l, const float4 (&o)[4]) {
-      const float Mn = fmaxf(M, m);
-      const float sa = M == -INFINITY ? 0.f : exp2f(M - Mn);
-      const float w = exp2f(m - Mn);
-      den = den * sa + w * l;
+        for (int i = 0; i < 4; ++i) o[i] = src[lane + 32 * i];
+        return true;
+      };
+      auto merge = [&](float m, float l, const float4 (&o)[4]) {
+        const float Mn = fmaxf(M, m);
+        const float sa = M == -INFINITY ? 0.f : exp2f(M - Mn);
+        const float w = exp2f(m - Mn);
+        den = den * sa + w * l;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[4 * i + 0] = acc[4 * i + 0] * sa + w * o[i].x;
+          acc[4 * i + 1] = acc[4 * i + 1] * sa + w * o[i].y;
+          acc[4 * i + 2] = acc[4 * i + 2] * sa + w * o[i].z;
+          acc[4 * i + 3] = acc[4 * i + 3] * sa + w * o[i].w;
+        }
+        M = Mn;
+      };
+      constexpr int kStep = 2;
+      for (int p = p0; p <= p1; p += kStep) {
+        float m[kStep], l[kStep];
+        float4 o[kStep][4];
+        bool has[kStep];
+#pragma unroll
+        for (int u = 0; u < kStep; ++u) has[u] = fetch(p + u, m[u], l[u], o[u]);
+#pragma unroll
+        for (int u = 0; u < kStep; ++u)
+          if (has[u]) merge(m[u], l[u], o[u]);
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        acc[4 * i + 0] = acc[4 * i + 0] * sa + w * o[i].x;
-        acc[4 * i + 1] = acc[4 * i + 1] * sa + w * o[i].y;
-        acc[4 * i + 2] = acc[4 * i + 2] * sa + w * o[i].z;
-        acc[4 * i + 3] = acc[4 * i + 3] * sa + w * o[i].w;
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc[4 * i + 0] * inv, acc[4 * i + 1] * inv);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc[4 * i + 2] * inv, acc[4 * i + 3] * inv);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(dst)[lane + 32 * i] = pk;
       }
-      M = Mn;
-    };
-    constexpr int kStep = 2;
-    for (int p = p0; p <= p1; p += kStep) {
-      float m[kStep], l[kStep];
-      float4 o[kStep][4];
-      bool has[kStep];
-#pragma unroll
-      for (int u = 0; u < kStep; ++u) has[u] = fetch(p + u, m[u], l[u], o[u]);
-#pragma unroll
-      for (int u = 0; u < kStep; ++u)
-        if (has[u]) merge(m[u], l[u], o[u]);
+      if (lse != nullptr && lane == 0)
+        lse[static_cast<int64_t>(b) * kHeads + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
     }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __nv_bfloat162 lo = __floats2bfloat162_rn(acc[4 * i + 0] * inv, acc[4 * i + 1] * inv);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(acc[4 * i + 2] * inv, acc[4 * i + 3] * inv);
-      uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t*>(&lo);
-      pk.y = *reinterpret_cast<uint32_t*>(&hi);
-      reinterpret_cast<uint2*>(dst)[lane + 32 * i] = pk;
-    }
-    if (lse != nullptr && lane == 0)
-      lse[static_cast<int64_t>(b) * kHeads + h] = den > 0.f ? (M + log2f(den)) * kLn2 : -INFINITY;
+  };
+  if (per_seq) {
+    merge_rows([](int p) { return 2 * p; }, [](int) { return true; });   // one piece per range: slot 2p
+  } else {
+    const int32_t* bounds = ws_bounds(ws, P);
+    merge_rows([&](int p) { return bounds[p] < off ? 2 * p + 1 : 2 * p; },
+               [&](int p) { return bounds[p] < bounds[p + 1]; });
   }
 }
 

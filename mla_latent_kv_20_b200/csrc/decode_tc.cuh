@@ -916,25 +916,47 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
 }
 
 // ------------------------------------------------------------------------------ work plan
-// One warp computes the plan; every CTA computes it for itself (it only reads seq_lens), and the
-// even CTA of range 0 also writes the table the combine reads.  Lane l walks the contiguous chunk
-// of sequences [l per, (l + 1) per): three passes over it (tile totals and the smallest sequence;
-// per-chunk sums of the prefix counts; the prefix itself, the table and this pair's piece), with
-// one warp reduction or scan between passes.  Every lane returns the same plan.
+// One warp computes the plan; every CTA computes it for itself (it only reads seq_lens), the even
+// CTA of range 0 also writes the table the combine reads, and the even CTA of every range writes
+// its first tile to bounds (the balanced plan; range P - 1 also writes bounds[P] = T).  Lane l
+// walks the contiguous chunk of sequences [l per, (l + 1) per): three passes over it (tile totals,
+// the smallest and largest sequence and the non-empty count; per-chunk sums of the prefix counts
+// and, balanced, of the costs; the prefixes themselves, the table and this pair's piece), with warp
+// reductions or scans between passes.  Every lane returns the same plan.  For batches of up to 128
+// sequences (per <= 4) the lane's lengths are loaded once, all loads in flight together, and kept
+// in registers for the three passes.
+constexpr int kTcPlanCached = 4;
 __device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacity, int B, int P, int32_t* table,
-                                               int pair, bool write_table) {
+                                               int32_t* bounds, int pair, bool write_table, bool write_bound) {
   const int lane = threadIdx.x & 31;
   const int per = (B + 31) / 32;
   const int lo = min(B, lane * per), hi = min(B, lo + per);
-  // pass 1: total tiles T and the smallest non-empty sequence (and the largest)
-  int sum = 0, mn = INT_MAX, mx = 0;
-  #pragma unroll 1
-  for (int bb = lo; bb < hi; ++bb) {
-    const int t = tiles_of(seq_len_checked(seq_lens, bb, capacity));
+  const bool cached = per <= kTcPlanCached;
+  int lens[kTcPlanCached];
+#pragma unroll
+  for (int u = 0; u < kTcPlanCached; ++u) lens[u] = (cached && lo + u < hi) ? seq_len_checked(seq_lens, lo + u, capacity) : 0;
+  // fn(bb, L) for every sequence bb of this lane's chunk, in order, with its checked length L
+  auto for_chunk = [&](auto&& fn) {
+    if (cached) {
+#pragma unroll
+      for (int u = 0; u < kTcPlanCached; ++u)
+        if (lo + u < hi) fn(lo + u, lens[u]);
+    } else {
+#pragma unroll 1
+      for (int bb = lo; bb < hi; ++bb) fn(bb, seq_len_checked(seq_lens, bb, capacity));
+    }
+  };
+  // pass 1: total tiles T, the smallest non-empty sequence, the largest, the non-empty count
+  int sum = 0, mn = INT_MAX, mx = 0, nne = 0;
+  for_chunk([&](int, int L) {
+    const int t = tiles_of(L);
     sum += t;
     mx = max(mx, t);
-    if (t > 0) mn = min(mn, t);
-  }
+    if (t > 0) {
+      mn = min(mn, t);
+      ++nne;
+    }
+  });
   const int T = __reduce_add_sync(0xffffffffu, sum);
   mn = __reduce_min_sync(0xffffffffu, mn);
   mx = __reduce_max_sync(0xffffffffu, mx);
@@ -972,30 +994,37 @@ __device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacit
     const int r = muldiv(P, t, T);
     return r < t ? r : t;
   };
-  // pass 2: this lane's share of the prefix
+  // pass 2: this lane's share of the prefix, and (balanced) of the cost line
   int csum = sum;
   if (per_seq) {
     csum = 0;
-    #pragma unroll 1
-    for (int bb = lo; bb < hi; ++bb) csum += count_of(tiles_of(seq_len_checked(seq_lens, bb, capacity)));
+    for_chunk([&](int, int L) { csum += count_of(tiles_of(L)); });
   }
-  int incl = csum;
+  const int wsum = sum + kSegCost * nne;
+  int incl = csum, wincl = wsum;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
     const int u = __shfl_up_sync(0xffffffffu, incl, d);
-    if (lane >= d) incl += u;
+    const int uw = __shfl_up_sync(0xffffffffu, wincl, d);
+    if (lane >= d) {
+      incl += u;
+      wincl += uw;
+    }
   }
   const int total = __shfl_sync(0xffffffffu, incl, 31);
-  // pass 3: the prefix of each sequence, the table, and the piece of this pair
-  const int start_g = T > 0 ? range_start(pair, P, T) : 0;   // the balanced plan's range
-  const int end_g = T > 0 ? range_start(pair + 1, P, T) : 0;
+  const int C = __shfl_sync(0xffffffffu, wincl, 31);
+  // pass 3: the prefixes, the table, and the piece of this pair.  Balanced: the range's cost
+  // interval [x0, x1) of the cost line; the lane whose sequence span holds x0 finds the start
+  // (and the first sequence), the one whose span holds x1 the end (none: x1 = C, the end is T).
+  const int x0 = (T > 0 && !per_seq) ? muldiv(pair, C, P) : 0;
+  const int x1 = (T > 0 && !per_seq) ? muldiv(pair + 1, C, P) : 0;
   TcPlan pl;
   pl.start = pl.end = 0;
   pl.b0 = pl.off0 = pl.b_end = pl.len0 = 0;
+  bool found_start = false, found_end = false;
   int run = incl - csum;
-  #pragma unroll 1
-  for (int bb = lo; bb < hi; ++bb) {
-    const int L = seq_len_checked(seq_lens, bb, capacity);
+  int W = wincl - wsum;
+  for_chunk([&](int bb, int L) {
     const int t = tiles_of(L);
     const int v = count_of(t);
     if (write_table) table[bb] = run;
@@ -1007,31 +1036,52 @@ __device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacit
         pl.start = muldiv(jj, t, v);
         pl.end = muldiv(jj + 1, t, v);
         pl.b_end = bb + 1;
+        found_start = found_end = true;
       }
-    } else if (t > 0 && start_g < end_g && run <= start_g && start_g < run + t) {
-      pl.b0 = bb;
-      pl.len0 = L;
-      pl.off0 = run;
-      pl.start = start_g;
-      pl.end = end_g;
-      pl.b_end = B;
+    } else if (t > 0) {
+      if (W <= x0 && x0 < W + kSegCost + t) {
+        pl.b0 = bb;
+        pl.len0 = L;
+        pl.off0 = run;
+        pl.start = run + max(0, x0 - W - kSegCost);
+        pl.b_end = B;
+        found_start = true;
+      }
+      if (W <= x1 && x1 < W + kSegCost + t) {
+        pl.end = run + max(0, x1 - W - kSegCost);
+        found_end = true;
+      }
+      W += kSegCost + t;
     }
     run += v;
-  }
+  });
   if (write_table && lane == 0) {
     table[B] = total;
     table[B + 1] = per_seq ? kPlanPerSequence : kPlanBalanced;
   }
-  // the lane that found the piece (at most one) hands it to the warp; otherwise the pair is idle
-  const unsigned found = __ballot_sync(0xffffffffu, pl.end > pl.start);
-  const int src = found ? __ffs(found) - 1 : 0;
+  // the lanes that found the start and the end (at most one each) hand them to the warp;
+  // otherwise the pair is idle (or, balanced, its range ends at T)
+  const unsigned fs = __ballot_sync(0xffffffffu, found_start);
+  const unsigned fe = __ballot_sync(0xffffffffu, found_end);
+  const int ss = fs ? __ffs(fs) - 1 : 0;
+  const int se = fe ? __ffs(fe) - 1 : 0;
   TcPlan r;
-  r.start = __shfl_sync(0xffffffffu, pl.start, src);
-  r.end = __shfl_sync(0xffffffffu, pl.end, src);
-  r.b0 = __shfl_sync(0xffffffffu, pl.b0, src);
-  r.off0 = __shfl_sync(0xffffffffu, pl.off0, src);
-  r.b_end = __shfl_sync(0xffffffffu, pl.b_end, src);
-  r.len0 = __shfl_sync(0xffffffffu, pl.len0, src);
+  r.start = __shfl_sync(0xffffffffu, pl.start, ss);
+  r.end = __shfl_sync(0xffffffffu, pl.end, se);
+  r.b0 = __shfl_sync(0xffffffffu, pl.b0, ss);
+  r.off0 = __shfl_sync(0xffffffffu, pl.off0, ss);
+  r.b_end = __shfl_sync(0xffffffffu, pl.b_end, ss);
+  r.len0 = __shfl_sync(0xffffffffu, pl.len0, ss);
+  if (!per_seq) {
+    if (!fe) r.end = T;
+    if (!fs) r.start = r.end = 0;   // no tiles at all (T = 0)
+    if (write_bound && lane == 0) {
+      bounds[pair] = fs ? r.start : T;
+      if (pair == P - 1) bounds[P] = T;
+    }
+  } else if (!fs) {
+    r.start = r.end = 0;
+  }
   return r;
 }
 
@@ -1111,7 +1161,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc_threads(kFp8), 1)
   // The producer warp computes the plan and hands it to the other warps through named barrier 2
   // (it only arrives, so its first copies need not wait for them).
   if (warp == kTcProducerWarp) {
-    const TcPlan w = tc_make_plan(a.seq_lens, a.capacity, a.batch, a.P, a.ws.off, pair, pair == 0 && rank == 0);
+    const TcPlan w = tc_make_plan(a.seq_lens, a.capacity, a.batch, a.P, a.ws.off, ws_bounds(a.ws, a.P), pair,
+                                  pair == 0 && rank == 0, rank == 0);
     if ((threadIdx.x & 31) == 0) *plan = w;
     __syncwarp();
     named_bar_arrive(2, tc_threads(kFp8));

@@ -72,7 +72,9 @@ def test_partial_segments_follow_the_plan():
     assert bench.partial_segments([4096] * 32, 74) == 64             # 32 tiles each: 2 ranges per sequence
     assert bench.partial_segments([131072] * 4, 512) == 512          # 128 ranges of 8 tiles per sequence
     assert bench.partial_segments([1280, 1280], 4) == 4              # tiles 10, 10: 2 ranges each
-    assert bench.partial_segments([256, 128, 384], 4) == 4           # balanced: ranges [0,1) [1,3) [3,4) [4,6)
+    # balanced: tiles 2, 1, 3 on a cost line of 12 (2 per sequence start): ranges [0,1) [1,2) [2,3) [3,6)
+    assert bench.plan_bounds([2, 1, 3], 4) == [0, 1, 2, 3, 6]
+    assert bench.partial_segments([256, 128, 384], 4) == 2
     assert bench.partial_segments([128, 128], 2) == 0                # one range per sequence: no partials
     assert bench.partial_segments([0, 0], 4) == 0
 

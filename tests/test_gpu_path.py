@@ -164,6 +164,37 @@ def test_decode_vs_oracle(env, lens, splits):
         assert_lse(g_lse[i], r["lse"])
 
 
+def test_decode_rescales_on_growing_scores(env):
+    """Scores that grow along the sequence: latent dim 0 of token t is 0.05 t and q_full's dim 0 runs
+    from -40 to 40 over the heads, so the running maximum of the steepest heads rises by far more
+    than the lazy-rescale threshold (2^8) on every tile and O is corrected on almost every tile,
+    gentler heads are corrected every few tiles and falling heads never.  Partner warps of the
+    softmax (the two token halves of a head) must take the same decision; checked contiguous with
+    the automatic plan and paged with forced work ranges, against the oracle."""
+    m, hz, torch = env
+    lens = [1000, 700, 130, 64]
+    b = mi.decode_batch(530, lens)
+    for i, L in enumerate(lens):
+        c = f64(b.c[i])
+        c[:L, 0] = 0.05 * np.arange(L)
+        b.c[i] = mi.f64_to_bf16(c)
+    q = 0.5 * np.random.default_rng(531).standard_normal((len(lens), 128, 576))
+    q[:, :, 0] = np.linspace(-40.0, 40.0, 128)
+    qf_bits = mi.f64_to_bf16(q)
+    for paged, splits in ((False, 0), (True, 3)):
+        table, nblk = mi.block_permutation(532, lens) if paged else (None, 0)
+        cache = hz.Cache(lens, paged, table, nblk, fill_value=float("nan") if paged else 0.0)
+        cache.fill(b.c, b.kr)
+        out_lat, lse = hz.decode(hz.bf16_tensor(qf_bits), cache, num_splits=splits)
+        torch.cuda.synchronize()
+        _clear(m)
+        g_lat, g_lse = f64(hz.bf16_bits(out_lat)), lse.cpu().numpy()
+        for i in range(len(lens)):
+            r = _ref_rows(b, qf_bits, i)
+            assert_out_lat(g_lat[i], r["out_lat"])
+            assert_lse(g_lse[i], r["lse"])
+
+
 def test_decode_paged_bit_identical_to_contiguous(env):
     lens = [1, 64, 65, 333, 1000]
     _, _, lat_c, lse_c = _decode_case(env, lens, 500, paged=False)
