@@ -178,10 +178,9 @@ int32_t mla_decode_num_splits(int32_t batch, int32_t max_seq_len, int32_t num_sp
 
 /*
  * Bytes of workspace mla_decode_attn needs, with P = mla_decode_num_splits(batch, max_seq_len,
- * num_splits): range partials O [2P, 128, 512] fp32 and (m, l) [2P, 128] fp32 each, the first
- * tile of each range [P + 1] int32 (padded to a multiple of 4), then the plan table [batch + 2]
- * int32 (per sequence its first global tile or first range, the total, the plan kind; rounded up
- * to 16 bytes).
+ * num_splits): range partials O [2P, 128, 512] fp32 and (m, l) [2P, 128] fp32 each, then the
+ * plan table [batch + 2] int32 (per sequence its cost-line offset or first range, the total, the
+ * plan kind; rounded up to 16 bytes).
  */
 size_t mla_decode_workspace_size(int32_t batch, int32_t max_seq_len, int32_t num_splits);
 

@@ -20,7 +20,9 @@
 //    boundary x_p = floor(p C / P) (C the total cost) falls in one such span and becomes global
 //    tile off_b + max(0, x_p - W_b - kSegCost) (off_b itself when it falls in the sequence's
 //    segment charge), or T when p = P.  Range p takes tiles [bound_p, bound_{p+1}) (possibly none);
-//    the part of each sequence a range touches is a segment.
+//    the part of each sequence a range touches is a segment.  Tile j of sequence b sits at cost
+//    y = W_b + kSegCost + j, and bound_p <= its global index exactly when x_p <= y, so the ranges
+//    holding a sequence's tiles follow from W_b, tiles_b and C in closed form (the combine).
 // A segment that covers its whole sequence is finished by the decode kernel; otherwise (in the
 // balanced plan at most the first and the last segment of a range) its partial goes to
 // workspace slot 2p (the range's first segment) or 2p + 1 (its last) and the combine merges the
@@ -48,31 +50,26 @@ constexpr float kLn2 = 0.6931471805599453f;
 //   O      [2P][128][512] fp32   (unnormalised partial sums of c)
 //   m      [2P][128]      fp32   (running max, log2 domain)
 //   l      [2P][128]      fp32   (running sum of exp2(s - m))
-//   bounds [P + 1]        int32  (balanced plan: first global tile of each range, [P] = T;
-//                                 written by the decode kernel; padded to a multiple of 4)
-//   plan   [batch + 2]    int32  (balanced: global tile offset of each sequence, [batch] = T;
+//   plan   [batch + 2]    int32  (balanced: cost prefix W_b of each sequence, [batch] = C;
 //                                 per sequence: first range of each sequence, [batch] = ranges used;
 //                                 [batch + 1] = the plan kind)
 struct Workspace {
   float* o;
   float* m;
   float* l;
-  int32_t* off;   // the plan table; the range bounds sit just before it (ws_bounds)
+  int32_t* off;
 };
-__host__ __device__ __forceinline__ int ws_bounds_ints(int P) { return (P + 1 + 3) / 4 * 4; }
 __host__ __device__ __forceinline__ Workspace ws_carve(void* base, int P) {
   Workspace w;
   w.o = reinterpret_cast<float*>(base);
   w.m = w.o + static_cast<int64_t>(2 * P) * kHeads * kDLat;
   w.l = w.m + static_cast<int64_t>(2 * P) * kHeads;
-  w.off = reinterpret_cast<int32_t*>(w.l + static_cast<int64_t>(2 * P) * kHeads) + ws_bounds_ints(P);
+  w.off = reinterpret_cast<int32_t*>(w.l + static_cast<int64_t>(2 * P) * kHeads);
   return w;
 }
-__host__ __device__ __forceinline__ int32_t* ws_bounds(const Workspace& w, int P) { return w.off - ws_bounds_ints(P); }
 __host__ __device__ __forceinline__ size_t ws_bytes(int batch, int P) {
   const size_t partials = static_cast<size_t>(2 * P) * kHeads * (kDLat + 2) * sizeof(float);
-  return partials + static_cast<size_t>(ws_bounds_ints(P)) * sizeof(int32_t) +
-         ((static_cast<size_t>(batch) + 2) * sizeof(int32_t) + 15) / 16 * 16;
+  return partials + ((static_cast<size_t>(batch) + 2) * sizeof(int32_t) + 15) / 16 * 16;
 }
 
 // Effective length of sequence b: seq_lens[b] clamped to [0, capacity] (error word set if it
@@ -96,15 +93,12 @@ __host__ __device__ __forceinline__ int muldiv(int x, int y, int z) {
   return muldiv_wide(p, static_cast<uint32_t>(z));
 }
 
-// The (non-empty) range of the balanced plan that holds global tile t (0 <= t < T): the last p
-// with bounds[p] <= t, by bisection over the P + 1 ascending bounds.
-__device__ __forceinline__ int range_of_tile(const int32_t* bounds, int t, int P) {
-  int lo = 0, hi = P - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (bounds[mid] <= t) lo = mid; else hi = mid - 1;
-  }
-  return lo;
+// The (non-empty) range of the balanced plan that holds the tile at cost y (0 <= y < C): the last
+// p with x_p = floor(p C / P) <= y, i.e. ceil((y + 1) P / C) - 1.
+__host__ __device__ __forceinline__ int range_of_cost(int y, int P, int C) {
+  const uint64_t x = static_cast<uint64_t>(y + 1) * static_cast<uint32_t>(P) + static_cast<uint32_t>(C - 1);
+  if (x <= 0xffffffffull) return static_cast<int>(static_cast<uint32_t>(x) / static_cast<uint32_t>(C)) - 1;
+  return muldiv_wide(x, static_cast<uint32_t>(C)) - 1;
 }
 
 constexpr int kPlanBalanced = 0;
@@ -176,7 +170,7 @@ __global__ void __launch_bounds__(128, hpw == 1 ? 8 : 4) combine_kernel(Workspac
   const int B = gridDim.x;
   const bool per_seq = ws.off[B + 1] == kPlanPerSequence;
   const int off = ws.off[b];
-  const int span = ws.off[b + 1] - off;   // tiles (balanced) or ranges (per sequence) of b
+  const int span = ws.off[b + 1] - off;   // kSegCost + tiles (balanced) or ranges (per sequence) of b
   if (span == 0) {
     for (int h = h0; h < h0 + hpw; ++h) {
       __nv_bfloat16* dst = out_lat + (static_cast<int64_t>(b) * kHeads + h) * kDLat;
@@ -186,8 +180,11 @@ __global__ void __launch_bounds__(128, hpw == 1 ? 8 : 4) combine_kernel(Workspac
     return;
   }
   // Ranges [p0, p1] that hold pieces of b; in the per-sequence plan each holds one (slot 2p).
-  const int p0 = per_seq ? off : range_of_tile(ws_bounds(ws, P), off, P);
-  const int p1 = per_seq ? off + span - 1 : range_of_tile(ws_bounds(ws, P), off + span - 1, P);
+  // Ranges [p0, p1] that hold pieces of b; in the per-sequence plan each holds one (slot 2p); in
+  // the balanced plan those holding its first and last tiles, at costs off + kSegCost and off + span - 1.
+  const int C = ws.off[B];
+  const int p0 = per_seq ? off : range_of_cost(off + kSegCost, P, C);
+  const int p1 = per_seq ? off + span - 1 : range_of_cost(off + span - 1, P, C);
   if (p0 == p1) return;
   // The merge over the ranges, with the slot and emptiness of range p given by the plan kind (two
   // copies of the loop, so that each keeps only what its kind needs live).
@@ -254,9 +251,10 @@ __global__ void __launch_bounds__(128, hpw == 1 ? 8 : 4) combine_kernel(Workspac
   if (per_seq) {
     merge_rows([](int p) { return 2 * p; }, [](int) { return true; });   // one piece per range: slot 2p
   } else {
-    const int32_t* bounds = ws_bounds(ws, P);
-    merge_rows([&](int p) { return bounds[p] < off ? 2 * p + 1 : 2 * p; },
-               [&](int p) { return bounds[p] < bounds[p + 1]; });
+    // Range p began before b (b is not its first segment: slot 2p + 1) when x_p < W_b = off, and is
+    // empty when x_{p+1} = x_p (then the kernel wrote nothing for it).
+    merge_rows([&](int p) { return muldiv(p, C, P) < off ? 2 * p + 1 : 2 * p; },
+               [&](int p) { return muldiv(p, C, P) < muldiv(p + 1, C, P); });
   }
 }
 

@@ -916,9 +916,9 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
 }
 
 // ------------------------------------------------------------------------------ work plan
-// One warp computes the plan; every CTA computes it for itself (it only reads seq_lens), the even
-// CTA of range 0 also writes the table the combine reads, and the even CTA of every range writes
-// its first tile to bounds (the balanced plan; range P - 1 also writes bounds[P] = T).  Lane l
+// One warp computes the plan; every CTA computes it for itself (it only reads seq_lens), and the
+// even CTA of range 0 also writes the table the combine reads (balanced: the cost prefix of each
+// sequence and the total cost; per sequence: the first range of each and the ranges used).  Lane l
 // walks the contiguous chunk of sequences [l per, (l + 1) per): three passes over it (tile totals,
 // the smallest and largest sequence and the non-empty count; per-chunk sums of the prefix counts
 // and, balanced, of the costs; the prefixes themselves, the table and this pair's piece), with warp
@@ -927,7 +927,7 @@ __device__ void tc_softmax(const DecodeTcArgs& a, const TcPlan& plan, int pair, 
 // in registers for the three passes.
 constexpr int kTcPlanCached = 4;
 __device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacity, int B, int P, int32_t* table,
-                                               int32_t* bounds, int pair, bool write_table, bool write_bound) {
+                                               int pair, bool write_table) {
   const int lane = threadIdx.x & 31;
   const int per = (B + 31) / 32;
   const int lo = min(B, lane * per), hi = min(B, lo + per);
@@ -1027,7 +1027,7 @@ __device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacit
   for_chunk([&](int bb, int L) {
     const int t = tiles_of(L);
     const int v = count_of(t);
-    if (write_table) table[bb] = run;
+    if (write_table) table[bb] = per_seq ? run : W;
     if (per_seq) {
       if (v > 0 && run <= pair && pair < run + v) {
         const int jj = pair - run;
@@ -1056,7 +1056,7 @@ __device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacit
     run += v;
   });
   if (write_table && lane == 0) {
-    table[B] = total;
+    table[B] = per_seq ? total : C;
     table[B + 1] = per_seq ? kPlanPerSequence : kPlanBalanced;
   }
   // the lanes that found the start and the end (at most one each) hand them to the warp;
@@ -1075,10 +1075,6 @@ __device__ __noinline__ TcPlan tc_make_plan(const int32_t* seq_lens, int capacit
   if (!per_seq) {
     if (!fe) r.end = T;
     if (!fs) r.start = r.end = 0;   // no tiles at all (T = 0)
-    if (write_bound && lane == 0) {
-      bounds[pair] = fs ? r.start : T;
-      if (pair == P - 1) bounds[P] = T;
-    }
   } else if (!fs) {
     r.start = r.end = 0;
   }
@@ -1161,8 +1157,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc_threads(kFp8), 1)
   // The producer warp computes the plan and hands it to the other warps through named barrier 2
   // (it only arrives, so its first copies need not wait for them).
   if (warp == kTcProducerWarp) {
-    const TcPlan w = tc_make_plan(a.seq_lens, a.capacity, a.batch, a.P, a.ws.off, ws_bounds(a.ws, a.P), pair,
-                                  pair == 0 && rank == 0, rank == 0);
+    const TcPlan w = tc_make_plan(a.seq_lens, a.capacity, a.batch, a.P, a.ws.off, pair, pair == 0 && rank == 0);
     if ((threadIdx.x & 31) == 0) *plan = w;
     __syncwarp();
     named_bar_arrive(2, tc_threads(kFp8));

@@ -99,8 +99,7 @@ def test_decode_validation_and_workspace(host_only):
     S = lib.mla_decode_num_splits(8, 4096, 16)
     assert S == 16 and lib.mla_decode_num_splits(8, 4096, 5000) == 1024
     need = lib.mla_decode_workspace_size(8, 4096, 16)
-    # partials of 16 ranges + 17 range bounds (padded to 20) + 9 tile offsets and 2 plan words, 16-B rounded
-    assert need == 2 * 16 * 128 * (512 + 2) * 4 + 20 * 4 + 48
+    assert need == 2 * 16 * 128 * (512 + 2) * 4 + 48     # partials of 16 ranges + the plan table [8 + 2], 16-B rounded
     # auto: at most one range per two 128-token tiles of batch x max_seq_len (the resident-pair
     # bound is 74 without a device to ask)
     assert lib.mla_decode_num_splits(1, 256, 0) == 1

@@ -64,6 +64,36 @@ def test_step_work_counts_bytes_and_flops():
     assert dec_bytes == cache_bytes + 2 * 128 * (576 + 512) * 2
 
 
+def test_balanced_plan_ranges_in_closed_form():
+    """The identity the combine relies on: with the balanced plan's bounds (plan_bounds, the
+    kernel's rule), tile j of sequence b sits in range ceil((y + 1) P / C) - 1 with y = W_b +
+    SEG_COST + j its cost; range p began before b exactly when x_p = floor(p C / P) < W_b; and a
+    range holding part of b is empty exactly when x_{p+1} = x_p.  Checked on random length mixes."""
+    import random
+    import bench
+    rnd = random.Random(7)
+    for _ in range(1500):
+        P = rnd.randint(1, 80)
+        tiles = [rnd.choice([0, 1, 2, 3, 5, 8, 13, 30, 64]) for _ in range(rnd.randint(1, 40))]
+        if sum(tiles) == 0:
+            continue
+        C = sum(t + bench.SEG_COST for t in tiles if t > 0)
+        bounds = bench.plan_bounds(tiles, P)
+        x = [p * C // P for p in range(P + 1)]
+        W = off = 0
+        for t in tiles:
+            if t == 0:
+                continue
+            for j in range(t):
+                assert max(p for p in range(P) if bounds[p] <= off + j) == -(-(W + bench.SEG_COST + j + 1) * P // C) - 1
+            for p in range(P):
+                assert (bounds[p] < off) == (x[p] < W)
+                if bounds[p] <= off + t - 1 and bounds[p + 1] > off:
+                    assert (bounds[p] < bounds[p + 1]) == (x[p] < x[p + 1])
+            W += bench.SEG_COST + t
+            off += t
+
+
 def test_partial_segments_follow_the_plan():
     """Range partials a decode call writes: per-sequence plan (r_b ranges of sequence b, partials
     only when r_b > 1) and the balanced plan (tiles end to end, a partial for every range that
