@@ -297,9 +297,11 @@ mla_status mla_unabsorb_v(const mla_bf16* out_lat, const mla_bf16* w_uv, mla_bf1
  * (6) Output projection — [DR] §2.3 (W_U^V belongs with the output projection W_O), §3.3 (model
  *     width d = 5120):  y[b] = W_O [ out[b, 0, :] | ... | out[b, 127, :] ]   (5120 <- 16384)
  * on the heads' outputs of mla_unabsorb_v, concatenated head-major.  Products in fp32 (exact for
- * bf16), sums over the 16384 inputs in fp32, one bf16 rounding of y.
+ * bf16), sums over the 16384 inputs in fp32 (the same order on every call), one bf16 rounding of y.
  *   out [batch, 128, 128] bf16     w_o [5120, 16384] bf16 (output index first)     y [batch, 5120] bf16
- * batch == 0 is a no-op; batch must be <= 65536.
+ * batch == 0 is a no-op; batch must be <= 65536.  The partial sums pass through a library-owned
+ * device buffer (23.5 MB, allocated when the library loads): calls of this entry point on different
+ * streams must not overlap in time.
  */
 mla_status mla_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y, int32_t batch, void* stream);
 

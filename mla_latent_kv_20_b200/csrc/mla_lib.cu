@@ -239,22 +239,33 @@ bool cluster16_ok(K kernel, int threads, int smem) {
 }
 
 // One output-projection launch with K split over SPLIT-CTA clusters.
-template <int SPLIT, int NT>
+// The output projection for one tile size NT: per N tile of NT sequences, the split kernel (one
+// CTA per SM, each an equal share of W_O) and the kernel that sums its partials.
+template <int NT, int R>
 mla_status launch_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y, int32_t batch, void* stream) {
-  using Sh = mla::OpShape<NT>;
+  using Sh = mla::OpShape<NT, R>;
   CUtensorMap tw, tx;
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kOpIn) * 2, 128};
   const cuuint64_t dw[3] = {64, static_cast<cuuint64_t>(mla::kOpOut), mla::kOpIn / 64};
   const cuuint64_t dx[3] = {64, static_cast<cuuint64_t>(batch), mla::kOpIn / 64};
-  const cuuint32_t bw[3] = {64, 128, static_cast<cuuint32_t>(mla::kOpKS / 64)};
-  const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(NT), static_cast<cuuint32_t>(mla::kOpKS / 64)};
+  const cuuint32_t bw[3] = {64, static_cast<cuuint32_t>(R), static_cast<cuuint32_t>(Sh::Z)};
+  const cuuint32_t bx[3] = {64, static_cast<cuuint32_t>(NT), static_cast<cuuint32_t>(Sh::Z)};
   if (!make_map_3d(&tw, w_o, dw, strides, bw) || !make_map_3d(&tx, out, dx, strides, bx)) return MLA_ERR_CUDA;
-  auto kern = mla::out_proj_kernel<SPLIT, NT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmemBytes) != cudaSuccess)
+  auto split = mla::out_proj_split_kernel<NT, R>;
+  if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
-  const dim3 grid(SPLIT, mla::kOpMTiles, (batch + NT - 1) / NT);
-  return launch_chained_cluster(kern, grid, dim3(mla::kOpThreads), static_cast<size_t>(Sh::kSmemBytes),
-                                as_stream(stream), SPLIT, tw, tx, reinterpret_cast<__nv_bfloat16*>(y), batch);
+  // one CTA per SM; a CTA's run of units must fit in one M tile's units (at most one boundary)
+  const int G = std::max(mla::kOpUnits / Sh::kUnitsPerTile, std::min(mla::kOpMaxCtas, device_sm_count()));
+  cudaStream_t s = as_stream(stream);
+  for (int n0 = 0; n0 < batch; n0 += NT) {
+    mla_status st = launch_chained(split, dim3(G), dim3(mla::kOpThreads), static_cast<size_t>(Sh::kSmemBytes), s, tw,
+                                   tx, n0);
+    if (st != MLA_OK) return st;
+    st = launch_chained(mla::out_proj_sum_kernel<NT, R>, dim3(Sh::kMTiles, NT / 8), dim3(R), 0, s,
+                        reinterpret_cast<__nv_bfloat16*>(y), batch, n0, G);
+    if (st != MLA_OK) return st;
+  }
+  return MLA_OK;
 }
 
 // One down-projection + append launch with K split over SPLIT-CTA clusters.
@@ -354,11 +365,12 @@ mla_status mla_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16* y
   if (batch == 0) return MLA_OK;
   if (out == nullptr || w_o == nullptr || y == nullptr) return MLA_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(w_o) || !aligned16(y)) return MLA_ERR_INVALID_ARG;
-  // 8-CTA clusters: twice as many clusters are resident at once as with 16 (measured 57 vs 72 us
-  // per call on 32 sequences with the weight coming from HBM).
-  // Tiles of 32 sequences up to 32, else of 128 (W_O then streams once per 128 sequences).
-  if (batch <= 32) return launch_output_proj<8, 32>(out, w_o, y, batch, stream);
-  return launch_output_proj<8, 128>(out, w_o, y, batch, stream);
+  // Tiles of 32 sequences up to 32, else of 128 (W_O then streams once per 128 sequences).  Units
+  // of 128 rows x 512 columns for the small tile (512 contiguous bytes per weight row and box:
+  // 46 vs 48 us at one sequence, 63 vs 69 us at 32), of 256 x 256 for the large one, whose
+  // activation box then stays half the weight box.
+  if (batch <= 32) return launch_output_proj<32, 128>(out, w_o, y, batch, stream);
+  return launch_output_proj<128, 256>(out, w_o, y, batch, stream);
 }
 
 }  // extern "C"

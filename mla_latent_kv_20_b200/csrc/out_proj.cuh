@@ -6,16 +6,18 @@
 // on the un-absorbed heads' outputs.  Products exact in fp32, sums over the 16384 inputs in fp32,
 // one rounding of y to bf16.
 //
-// B200 mapping.  The weight (5120 x 16384 bf16, 168 MB) streams from HBM once per N tile and is the
-// M operand ("swap-AB": M = output dims in 40 tiles of 128, N = sequences in tiles of NT = 32, or
-// of 128 for batches above 32 so that the weight streams once per 128 sequences, K = 16384); K is
-// split over the SPLIT CTAs of a cluster (8: twice as many such clusters are resident at once as
-// 16-CTA ones), each streaming its share through a ring of 40 KB (NT = 32, 4 stages) or 64 KB
-// (NT = 128, 3 stages) stages while two threads issue the MMAs into two TMEM accumulators; the
-// SPLIT partial tiles are reduced through distributed shared memory (CTA r sums rows [R r, R r + R),
-// R = 128 / SPLIT) and written as bf16.
-// grid = (SPLIT, 40, ceil(B / NT)), clusters of SPLIT along x (set at launch); 224 threads: warps
-// 0-3 epilogue and reduction, warp 4 TMA producer, warps 5-6 MMA issuers.
+// B200 mapping.  The weight (5120 x 16384 bf16, 168 MB) is the M operand ("swap-AB": M = output
+// dims, N = sequences in tiles of NT = 32, or of 128 for batches above 32, K = 16384) and streams
+// from HBM once per N tile.  Streaming it is the whole cost, so every SM streams an equal share in
+// one wave: the work is 2560 units of R rows x 65536 / R columns (R = 256: 20 M tiles x 128 units;
+// R = 128: 40 x 64), laid out M tile by M tile, and CTA c of G (one per SM) takes units
+// [c U / G, (c + 1) U / G) (17 or 18 on 148 SMs), which cross at most one M-tile boundary, so a CTA
+// accumulates at most two segments (two accumulators each, one per MMA-issuing warp, in TMEM).  Each segment's fp32 partial goes to a
+// library-owned scratch buffer (so calls on different streams must not overlap), and a second
+// kernel sums the partials of each M tile in CTA order (fp32, the same order every call) and
+// rounds y to bf16.  (Clusters that reduce through distributed shared memory cannot give every SM
+// an equal share: 8-CTA clusters ran 16 at a time, so 40 of them took three waves, the last on a
+// fifth of the SMs.)
 #pragma once
 
 #include <cuda_bf16.h>
@@ -27,62 +29,77 @@ namespace mla {
 
 constexpr int kOpIn = kHeads * kDHead;   // 16384 inputs
 constexpr int kOpOut = kDHidden;         // 5120 outputs
-constexpr int kOpMTiles = kOpOut / 128;
-constexpr int kOpKS = 128;               // contraction columns per stage
-constexpr int kOpThreads = 224;
-constexpr int kOpWBytes = kOpKS * 128 * 2;
-static_assert(kOpOut % 128 == 0, "M tiles");
-// Per N tile of NT sequences (32, or 128 for larger batches, so that W_O streams once per 128
-// sequences): stages in flight, stage and shared-memory bytes.
-template <int NT>
+constexpr int kOpUnitElems = 256 * 128;  // W elements of a unit: R rows x (65536 / R) columns
+constexpr int kOpUnits = kOpOut * kOpIn / kOpUnitElems;   // 2560
+constexpr int kOpThreads = 224;          // warps 0-3 epilogue, warp 4 TMA producer, warps 5-6 MMA issuers
+constexpr int kOpMaxCtas = 160;          // CTAs of the split kernel (one per SM)
+constexpr int kOpMaxNt = 128;
+constexpr int kOpMaxRows = 256;
+constexpr int kOpMaxMTiles = kOpOut / 128;
+// Scratch slots of [NT][256] fp32 partials: slot c for CTA c's first segment, kOpMaxCtas + k - 1
+// for the segment of M tile k that a CTA starts after crossing the boundary into it.
+constexpr int kOpSlots = kOpMaxCtas + kOpMaxMTiles - 1;
+__device__ float g_op_partial[static_cast<size_t>(kOpSlots) * kOpMaxRows * kOpMaxNt];
+
+// A unit is R rows (256: one 128-row half per MMA-issuing warp; 128: the warps split its K steps)
+// by Z 64-column chunks (Z = 512 / R: every row of a unit's weight box is 128 Z contiguous bytes).
+template <int NT, int R>
 struct OpShape {
-  static constexpr int kRing = NT <= 32 ? 4 : 3;
-  static constexpr int kXBytes = kOpKS * NT * 2;
-  static constexpr int kStageBytes = kOpWBytes + kXBytes;
+  static constexpr int Z = 512 / R;
+  static constexpr int kMTiles = kOpOut / R;
+  static constexpr int kUnitsPerTile = kOpIn / (64 * Z);
+  static constexpr int kWBytes = R * Z * 128;
+  static constexpr int kXBytes = NT * Z * 128;
+  static constexpr int kStageBytes = kWBytes + kXBytes;
+  static constexpr int kRing = (227 * 1024 - 2048) / kStageBytes < 4 ? (227 * 1024 - 2048) / kStageBytes : 4;
   static constexpr int kSmemBytes = 1024 + kRing * kStageBytes + 256;
-  static_assert(128 * (NT + 1) * 4 <= kRing * kStageBytes, "reduction tile fits in the operand ring");
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(R == 128 || R == 256, "unit rows");
+  static_assert(kRing >= 2 && kSmemBytes <= 232448, "shared memory budget");
+  static_assert(NT <= kOpMaxNt && 4 * NT <= 512, "TMEM: two segments x two accumulators of NT columns");
+  static_assert(kMTiles * kUnitsPerTile == kOpUnits, "units");
 };
 
-// tmW: 3-D view of W_O [5120][16384] (64-column chunk, row, chunk index), box {64, 128, 2}.
-// tmX: the same view of out [B][16384], box {64, NT, 2} (rows past B arrive as zeros).
-template <int SPLIT, int NT>
+// Units [u0, u1) of CTA c of G, and the scratch slot of segment `seg` (0 or 1) of M tile m.
+__host__ __device__ __forceinline__ int op_unit0(int c, int G) { return c * kOpUnits / G; }
+__device__ __forceinline__ int op_slot(int c, int seg, int m) { return seg == 0 ? c : kOpMaxCtas + m - 1; }
+// The CTA whose units hold unit u: the last c with op_unit0(c) <= u, i.e. ceil((u + 1) G / U) - 1.
+__device__ __forceinline__ int op_cta_of(int u, int G) { return ((u + 1) * G + kOpUnits - 1) / kOpUnits - 1; }
+
+// tmW: 3-D view of W_O [5120][16384] (64-column chunk, row, chunk index), box {64, R, Z}.
+// tmX: the same view of out [B][16384], box {64, NT, Z} (rows past B arrive as zeros).
+// grid = G (kOpUnits / G <= units per M tile, G <= kOpMaxCtas), one CTA per SM; N tile of
+// sequences [n0, n0 + NT).
+template <int NT, int R>
 __global__ void __launch_bounds__(kOpThreads, 1)
-    out_proj_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                    __nv_bfloat16* __restrict__ y, int batch) {
-  static_assert(SPLIT == 8 || SPLIT == 16, "cluster sizes");
-  constexpr int KPER = kOpIn / SPLIT;       // contraction columns of one CTA
-  constexpr int NST = KPER / kOpKS;         // its stages
-  constexpr int R = 128 / SPLIT;            // tile rows each CTA reduces
-  constexpr int JN = NT * R / 128;          // outputs per thread in the reduction
-  using Sh = OpShape<NT>;
-  constexpr int kOpRing = Sh::kRing;
-  constexpr int kOpStageBytes = Sh::kStageBytes;
+    out_proj_split_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int n0) {
+  using Sh = OpShape<NT, R>;
+  constexpr int kRing = Sh::kRing;
+  constexpr int kStage = Sh::kStageBytes;
+  constexpr int Z = Sh::Z;
+  constexpr int kStages = Sh::kUnitsPerTile;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kOpRing * kOpStageBytes);
-  uint64_t* empty = full + kOpRing;
-  uint64_t* done = empty + kOpRing;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
-  float* red = reinterpret_cast<float*>(smem);   // reuses the ring once the MMAs are done
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRing * kStage);
+  uint64_t* empty = full + kRing;
+  uint64_t* seg_done = empty + kRing;   // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(seg_done + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int rank = static_cast<int>(cluster_ctarank());
-  const int mt = blockIdx.y;
-  const int n0 = blockIdx.z * NT;
-  const int kc0 = rank * KPER / 64;   // first 64-column chunk of this CTA
-  constexpr uint32_t kAccCols = NT;
-  constexpr uint32_t kTmemCols = 2 * NT;
+  const int G = gridDim.x;
+  const int c = blockIdx.x;
+  const int u0 = op_unit0(c, G), u1 = op_unit0(c + 1, G);
+  const int m_first = u0 / kStages;
+  const int n_seg = (u1 > u0) ? (u1 - 1) / kStages - m_first + 1 : 0;
+  constexpr uint32_t kTmemCols = 4 * NT < 32 ? 32 : 4 * NT;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kOpRing; ++s) {
+    for (int s = 0; s < kRing; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 2);   // one commit per issuing warp
     }
-    mbar_init(done, 2);
-    *abort_flag = 0;
+    mbar_init(&seg_done[0], 2);
+    mbar_init(&seg_done[1], 2);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -92,127 +109,124 @@ __global__ void __launch_bounds__(kOpThreads, 1)
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
-    // The weight does not depend on earlier kernels: pull this CTA's share into L2 meanwhile.
-    for (int q = 0; q < NST; ++q) tma_prefetch_l2_3d(&tmW, 0, 128 * mt, kc0 + q * (kOpKS / 64));
+    // The weight does not depend on earlier kernels: pull this CTA's first units into L2 meanwhile.
+    for (int u = u0; u < u1 && u < u0 + 8; ++u) tma_prefetch_l2_3d(&tmW, 0, R * (u / kStages), (u % kStages) * Z);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
   pdl_trigger();
-  pdl_wait();
+  pdl_wait();   // the activation, and the scratch (read by the previous call's sum kernel)
 
   if (warp == 4 && lane == 0) {
     // ---------------- TMA producer
     int q = 0;
-    for (; q < NST; ++q) {
-      const int s = q % kOpRing;
-      if (q >= kOpRing && !mbar_wait(&empty[s], static_cast<uint32_t>((q / kOpRing) - 1) & 1u)) {
-        *abort_flag = 1;
-        break;
-      }
-      uint8_t* sa = smem + s * kOpStageBytes;
-      mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kOpStageBytes));
-      tma_load_3d(sa, &tmW, &full[s], 0, 128 * mt, kc0 + q * (kOpKS / 64));
-      tma_load_3d(sa + kOpWBytes, &tmX, &full[s], 0, n0, kc0 + q * (kOpKS / 64));
+    for (; q < u1 - u0; ++q) {
+      const int s = q % kRing;
+      if (q >= kRing && !mbar_wait(&empty[s], static_cast<uint32_t>((q / kRing) - 1) & 1u)) break;
+      const int u = u0 + q;
+      uint8_t* sa = smem + s * kStage;
+      mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kStage));
+      tma_load_3d(sa, &tmW, &full[s], 0, R * (u / kStages), (u % kStages) * Z);
+      tma_load_3d(sa + Sh::kWBytes, &tmX, &full[s], 0, n0, (u % kStages) * Z);
     }
-    // never leave (or let the ring be reused) while a copy is still landing
-    for (int t = q > kOpRing ? q - kOpRing : 0; t < q; ++t)
-      if (!mbar_wait(&full[t % kOpRing], static_cast<uint32_t>(t / kOpRing) & 1u)) *abort_flag = 1;
+    // never leave while a copy is still landing
+    for (int t = q > kRing ? q - kRing : 0; t < q; ++t) mbar_wait(&full[t % kRing], static_cast<uint32_t>(t / kRing) & 1u);
   } else if (warp >= 5 && lane == 0) {
-    // ---------------- MMA issuers: warp 5 + j takes the 16-deep K steps with index % 2 == j
+    // ---------------- MMA issuers, warp 5 + j: R = 256, rows [128 j, 128 j + 128) of each unit over
+    // all its K steps; R = 128, the K steps of parity j.  Each into its own accumulator of the segment.
     const int j = warp - 5;
-    const uint32_t acc = tmem_d + j * kAccCols;
     const uint32_t idesc = idesc_bf16_f32(128, NT, /*a_mn_major=*/false, /*b_mn_major=*/false);
-    bool first = true;
-    for (int q = 0; q < NST; ++q) {
-      const int s = q % kOpRing;
-      if (!mbar_wait(&full[s], static_cast<uint32_t>(q / kOpRing) & 1u)) {
-        *abort_flag = 1;
-        break;
-      }
+    constexpr int kSteps = 4 * Z;                    // 16-deep K steps of a unit
+    constexpr int kStep = R == 256 ? 1 : 2;
+    for (int q = 0; q < u1 - u0; ++q) {
+      const int s = q % kRing;
+      const int u = u0 + q;
+      const int seg = u / kStages - m_first;
+      const bool seg_start = q == 0 || u % kStages == 0;
+      if (!mbar_wait(&full[s], static_cast<uint32_t>(q / kRing) & 1u)) break;
       tc_fence_after();
-      const uint32_t sa = smem_u32(smem + s * kOpStageBytes);
-      const uint32_t sb = sa + kOpWBytes;
+      const uint32_t acc = tmem_d + static_cast<uint32_t>((2 * seg + j) * NT);
+      const uint32_t sa = smem_u32(smem + s * kStage) + (R == 256 ? j * (128 * 128) : 0);
+      const uint32_t sb = smem_u32(smem + s * kStage) + Sh::kWBytes;
 #pragma unroll
-      for (int kk = j; kk < kOpKS / 16; kk += 2) {
-        // A (K-major): chunk kk / 4 of 128 rows x 128 B; B (K-major): chunk kk / 4 of 32 rows x 128 B.
-        const uint64_t adesc = sdesc_sw128(sa + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+      for (int kk = (R == 256 ? 0 : j); kk < kSteps; kk += kStep) {
+        // A (K-major): chunk kk / 4 of R rows x 128 B; B (K-major): chunk kk / 4 of NT rows x
+        // 128 B.  16 K elements = 32 B into each row.
+        const uint64_t adesc = sdesc_sw128(sa + (kk >> 2) * (R * 128) + (kk & 3) * 32, 16, 1024);
         const uint64_t bdesc = sdesc_sw128(sb + (kk >> 2) * (NT * 128) + (kk & 3) * 32, 16, 1024);
-        umma_bf16_ss(acc, adesc, bdesc, idesc, first ? 0u : 1u);
-        first = false;
+        umma_bf16_ss(acc, adesc, bdesc, idesc, (seg_start && kk == (R == 256 ? 0 : j)) ? 0u : 1u);
       }
       umma_commit(&empty[s]);
+      if (u % kStages == kStages - 1 || q == u1 - u0 - 1) umma_commit(&seg_done[seg]);
     }
-    umma_commit(done);   // also fires when nothing was issued, so the epilogue never waits forever
   } else if (warp < 4) {
-    // ---------------- epilogue part 1: this CTA's partial tile into its reduction tile red[m][n]
-    const bool ok = mbar_wait(done, 0);
-    tc_fence_after();
-    const int m = warp * 32 + lane;
-    const uint32_t trow = tmem_d + (static_cast<uint32_t>(warp * 32) << 16);
-    uint32_t r0[16], r1[16];
-#pragma unroll
-    for (int c = 0; c < NT; c += 16) {
-      tmem_ld16(trow + c, r0);
-      tmem_ld16(trow + kAccCols + c, r1);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        red[m * (NT + 1) + c + i] = ok ? __uint_as_float(r0[i]) + __uint_as_float(r1[i]) : 0.f;
-    }
-    if (!ok) *abort_flag = 1;
-    // Cluster barrier 1 (each thread arrives once; warps 4-6 arrive below, after their roles).
-    tc_fence_before();
-    __syncwarp();
-    cluster_arrive_release();
-    cluster_wait_acquire();
-
-    // ---------------- epilogue part 2: rows [R rank, R rank + R) of the cluster's sum
-    const int t = threadIdx.x;
-    const int mr = R * rank + (t % R);
-    const uint32_t red_addr = smem_u32(red);
-    int flags = 0;
-    {
-      float f[SPLIT];
-#pragma unroll
-      for (int q = 0; q < SPLIT; ++q) f[q] = ld_shared_cluster_f32(mapa_shared(smem_u32(abort_flag), q));
-#pragma unroll
-      for (int q = 0; q < SPLIT; ++q) flags |= __float_as_int(f[q]);
-    }
-    constexpr int kJC = JN < 4 ? JN : 4;   // outputs per batch of loads
+    // ---------------- epilogue: each segment's partial [NT][256] fp32 to its scratch slot (for a
+    // given n the 32 lanes' rows are contiguous: one 128-byte store per warp and n)
+    for (int seg = 0; seg < n_seg; ++seg) {
+      const bool ok = mbar_wait(&seg_done[seg], 0);
+      tc_fence_after();
+      const int m = m_first + seg;
+      float* dst = g_op_partial + static_cast<size_t>(op_slot(c, seg, m)) * kOpMaxRows * kOpMaxNt;
+      const uint32_t trow = tmem_d + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(2 * seg * NT);
+      if constexpr (R == 256) {
 #pragma unroll 1
-    for (int j0 = 0; j0 < JN; j0 += kJC) {
-      float part[kJC][SPLIT];   // a batch's loads all in flight at once, then the sums in rank order
+        for (int j = 0; j < 2; ++j) {
+          const int r = 128 * j + 32 * warp + lane;
+#pragma unroll 1
+          for (int cc = 0; cc < NT; cc += 16) {
+            uint32_t v[16];
+            tmem_ld16(trow + static_cast<uint32_t>(j * NT + cc), v);
+            tmem_ld_wait();
 #pragma unroll
-      for (int jj = 0; jj < kJC; ++jj) {
-        const int nl = t / R + (128 / R) * (j0 + jj);
-        const uint32_t off = red_addr + 4u * static_cast<uint32_t>(mr * (NT + 1) + nl);
+            for (int i = 0; i < 16; ++i) dst[(cc + i) * R + r] = ok ? __uint_as_float(v[i]) : 0.f;
+          }
+        }
+      } else {
+        const int r = 32 * warp + lane;   // the two accumulators hold the same rows: their sum
+#pragma unroll 1
+        for (int cc = 0; cc < NT; cc += 16) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(trow + static_cast<uint32_t>(cc), v0);
+          tmem_ld16(trow + static_cast<uint32_t>(NT + cc), v1);
+          tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < SPLIT; ++q) part[jj][q] = ld_shared_cluster_f32(mapa_shared(off, q));
-      }
-#pragma unroll
-      for (int jj = 0; jj < kJC; ++jj) {
-        float sum = 0.f;
-#pragma unroll
-        for (int q = 0; q < SPLIT; ++q) sum += part[jj][q];
-        const int n = n0 + t / R + (128 / R) * (j0 + jj);
-        if (n < batch && flags == 0)
-          y[static_cast<int64_t>(n) * kOpOut + 128 * mt + mr] = __float2bfloat16_rn(sum);
+          for (int i = 0; i < 16; ++i)
+            dst[(cc + i) * R + r] = ok ? __uint_as_float(v0[i]) + __uint_as_float(v1[i]) : 0.f;
+        }
       }
     }
   }
-  if (warp >= 4) {
-    // producer and issuer warps (all lanes, reconverged): cluster barrier 1
-    __syncwarp();
-    tc_fence_before();
-    cluster_arrive_release();
-    cluster_wait_acquire();
-  }
-  cluster_sync();   // no CTA leaves while a peer may still read its reduction tile
+  tc_fence_before();
+  __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_d, kTmemCols);
+  }
+}
+
+// Sum of the partials of M tile blockIdx.x for sequences n0 + 8 blockIdx.y + [0, 8): thread r takes
+// row r (R threads); the CTAs whose runs hold units of the tile are summed in CTA order.
+template <int NT, int R>
+__global__ void __launch_bounds__(R) out_proj_sum_kernel(__nv_bfloat16* __restrict__ y, int batch, int n0, int G) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int kStages = OpShape<NT, R>::kUnitsPerTile;
+  const int m = blockIdx.x;
+  const int r = threadIdx.x;
+  const int c_lo = op_cta_of(m * kStages, G), c_hi = op_cta_of(m * kStages + kStages - 1, G);
+#pragma unroll 1
+  for (int nn = 0; nn < 8; ++nn) {
+    const int n = 8 * blockIdx.y + nn;
+    if (n0 + n >= batch) break;
+    float sum = 0.f;
+#pragma unroll 1
+    for (int c = c_lo; c <= c_hi; ++c) {
+      const int seg = m - op_unit0(c, G) / kStages;
+      sum += g_op_partial[static_cast<size_t>(op_slot(c, seg, m)) * kOpMaxRows * kOpMaxNt + n * R + r];
+    }
+    y[static_cast<int64_t>(n0 + n) * kOpOut + R * m + r] = __float2bfloat16_rn(sum);
   }
 }
 
