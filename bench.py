@@ -314,12 +314,12 @@ TRAFFIC_SOURCES = ("csrc/decode_tc.cuh", "csrc/decode_common.cuh", "csrc/ptx.cuh
                    "csrc/decode_launch.cuh")
 MEASURED_TRAFFIC = {   # workload[@ranges] -> {"bytes": int, "sha256": str, "profile": str}
     "b128_u1024_8192_paged": {
-        "bytes": 693064192 + 27741184 + 37912832,
-        "sha256": "86b9eb1ac8b66e99ad9405569e62e03a92b23b9a3adebbfdf528ddb344c3adf3",
+        "bytes": 692713728 + 27520512 + 36337664,
+        "sha256": "8a3f5dfa12b42f6720b1337f7e46a5337e6e4a9823a12bd11a065ea0c4e23e0d",
         "profile": "profiles/decode_tc_b128_u1024_8192_paged.md (decode + combine, ncu cache flush per kernel)"},
     "b32_l4096": {
-        "bytes": 155815936 + 3915776 + 16858624,
-        "sha256": "86b9eb1ac8b66e99ad9405569e62e03a92b23b9a3adebbfdf528ddb344c3adf3",
+        "bytes": 155804416 + 3546368 + 16862976,
+        "sha256": "8a3f5dfa12b42f6720b1337f7e46a5337e6e4a9823a12bd11a065ea0c4e23e0d",
         "profile": "profiles/decode_tc_b32_l4096.md (decode + combine, ncu cache flush per kernel)"},
 }
 

@@ -261,7 +261,8 @@ mla_status launch_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16
     mla_status st = launch_chained(split, dim3(G), dim3(mla::kOpThreads), static_cast<size_t>(Sh::kSmemBytes), s, tw,
                                    tx, n0);
     if (st != MLA_OK) return st;
-    st = launch_chained(mla::out_proj_sum_kernel<NT, R>, dim3(Sh::kMTiles, NT / 8), dim3(R), 0, s,
+    static_assert(Sh::kUnitsPerTile * mla::kOpMaxCtas / mla::kOpUnits + 2 <= mla::kOpSumMaxCtas, "CTAs per M tile");
+    st = launch_chained(mla::out_proj_sum_kernel<NT, R>, dim3(Sh::kMTiles, NT), dim3(R), 0, s,
                         reinterpret_cast<__nv_bfloat16*>(y), batch, n0, G);
     if (st != MLA_OK) return st;
   }

@@ -206,28 +206,34 @@ __global__ void __launch_bounds__(kOpThreads, 1)
   }
 }
 
-// Sum of the partials of M tile blockIdx.x for sequences n0 + 8 blockIdx.y + [0, 8): thread r takes
-// row r (R threads); the CTAs whose runs hold units of the tile are summed in CTA order.
+// Sum of the partials of M tile blockIdx.x for sequence n0 + blockIdx.y: thread r takes row r (R
+// threads); the CTAs whose runs hold units of the tile (at most kOpSumMaxCtas) are summed in CTA
+// order, their loads all in flight at once.
+constexpr int kOpSumMaxCtas = 16;
 template <int NT, int R>
 __global__ void __launch_bounds__(R) out_proj_sum_kernel(__nv_bfloat16* __restrict__ y, int batch, int n0, int G) {
   pdl_trigger();
   pdl_wait();
   constexpr int kStages = OpShape<NT, R>::kUnitsPerTile;
   const int m = blockIdx.x;
+  const int n = blockIdx.y;
   const int r = threadIdx.x;
+  if (n0 + n >= batch) return;
   const int c_lo = op_cta_of(m * kStages, G), c_hi = op_cta_of(m * kStages + kStages - 1, G);
-#pragma unroll 1
-  for (int nn = 0; nn < 8; ++nn) {
-    const int n = 8 * blockIdx.y + nn;
-    if (n0 + n >= batch) break;
-    float sum = 0.f;
-#pragma unroll 1
-    for (int c = c_lo; c <= c_hi; ++c) {
+  float v[kOpSumMaxCtas];
+#pragma unroll
+  for (int i = 0; i < kOpSumMaxCtas; ++i) {
+    const int c = c_lo + i;
+    v[i] = 0.f;
+    if (c <= c_hi) {
       const int seg = m - op_unit0(c, G) / kStages;
-      sum += g_op_partial[static_cast<size_t>(op_slot(c, seg, m)) * kOpMaxRows * kOpMaxNt + n * R + r];
+      v[i] = g_op_partial[static_cast<size_t>(op_slot(c, seg, m)) * kOpMaxRows * kOpMaxNt + n * R + r];
     }
-    y[static_cast<int64_t>(n0 + n) * kOpOut + R * m + r] = __float2bfloat16_rn(sum);
   }
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < kOpSumMaxCtas; ++i) sum += v[i];   // ascending CTA order; the zeros past c_hi add nothing
+  y[static_cast<int64_t>(n0 + n) * kOpOut + R * m + r] = __float2bfloat16_rn(sum);
 }
 
 }  // namespace mla
