@@ -136,7 +136,9 @@ mla_status mla_cache_append_fp8(const mla_bf16* c_new, const mla_bf16* kr_new, c
  *   h      [n_tokens, 5120] bf16          w_dkv [512, 5120] bf16 (output index first)
  *   w_kr   [64, 5120] bf16                seq_ids [n_tokens] int32 or NULL    pos [n_tokens] int32
  *   cache  per desc (written)             block_table per desc or NULL
- * n_tokens == 0 is a no-op; n_tokens must be <= 65536.  Device checks as mla_cache_append.
+ * n_tokens == 0 is a no-op; n_tokens must be <= 65536.  Device checks as mla_cache_append.  The
+ * partial sums pass through a library-owned device buffer (6.8 MB, allocated when the library
+ * loads): calls of this entry point on different streams must not overlap in time.
  */
 mla_status mla_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const mla_bf16* w_kr,
                               const int32_t* seq_ids, const int32_t* pos, mla_bf16* cache,

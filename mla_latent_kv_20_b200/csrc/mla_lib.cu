@@ -54,32 +54,6 @@ mla_status launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   return MLA_OK;
 }
 
-// As launch_chained, with the cluster shape set at launch (cluster_x CTAs along x).
-template <typename... KArgs, typename... Args>
-mla_status launch_chained_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                                  unsigned cluster_x, Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = cluster_x;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    return MLA_ERR_CUDA;
-  }
-  return MLA_OK;
-}
-
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -210,35 +184,6 @@ mla::RopeFreq rope_freq(float rope_base) {
   return f;
 }
 
-// Whether the device places 16-CTA clusters of `kernel` (non-portable size) with this block size
-// and dynamic shared memory; sets the attributes the launch needs.
-template <typename K>
-bool cluster16_ok(K kernel, int threads, int smem) {
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
-      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return false;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(16, 1, 1);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 16;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) {
-    (void)cudaGetLastError();
-    n = 0;
-  }
-  return n >= 1;
-}
-
-// One output-projection launch with K split over SPLIT-CTA clusters.
 // The output projection for one tile size NT: per N tile of NT sequences, the split kernel (one
 // CTA per SM, each an equal share of W_O) and the kernel that sums its partials.
 template <int NT, int R>
@@ -269,31 +214,41 @@ mla_status launch_output_proj(const mla_bf16* out, const mla_bf16* w_o, mla_bf16
   return MLA_OK;
 }
 
-// One down-projection + append launch with K split over SPLIT-CTA clusters.
-template <int SPLIT>
+// The down-projection + append for one tile size NT: per N tile of NT tokens, the split kernel
+// (each CTA an equal share of the weights' 200 units) and the kernel that sums the partials,
+// rotates the keys and writes the cache rows.
+template <int NT>
 mla_status launch_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const mla_bf16* w_kr,
                                  const int32_t* seq_ids, const int32_t* pos, mla_bf16* cache, const CacheView& v,
                                  int32_t n_tokens, float rope_base, void* stream) {
-  using Sh = mla::DpShape<SPLIT>;
+  using Sh = mla::DpShape<NT>;
   // 3-D views (64-column chunk, row, chunk index) of the row-major [rows][5120] matrices.
   CUtensorMap tw, tk, th;
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDHidden) * 2, 128};
   const cuuint64_t dw[3] = {64, static_cast<cuuint64_t>(mla::kDLat), mla::kDHidden / 64};
   const cuuint64_t dk[3] = {64, static_cast<cuuint64_t>(mla::kDRope), mla::kDHidden / 64};
   const cuuint64_t dh[3] = {64, static_cast<cuuint64_t>(n_tokens), mla::kDHidden / 64};
-  const cuuint32_t bw[3] = {64, 128, static_cast<cuuint32_t>(Sh::kChunks)};
-  const cuuint32_t bk[3] = {64, static_cast<cuuint32_t>(mla::kDRope), static_cast<cuuint32_t>(Sh::kChunks)};
-  const cuuint32_t bh[3] = {64, static_cast<cuuint32_t>(mla::kDpNt), static_cast<cuuint32_t>(Sh::kChunks)};
+  const cuuint32_t bw[3] = {64, 128, static_cast<cuuint32_t>(mla::kDpKS / 64)};
+  const cuuint32_t bk[3] = {64, static_cast<cuuint32_t>(mla::kDRope), static_cast<cuuint32_t>(mla::kDpKS / 64)};
+  const cuuint32_t bh[3] = {64, static_cast<cuuint32_t>(NT), static_cast<cuuint32_t>(mla::kDpKS / 64)};
   if (!make_map_3d(&tw, w_dkv, dw, strides, bw) || !make_map_3d(&tk, w_kr, dk, strides, bk) ||
       !make_map_3d(&th, h, dh, strides, bh))
     return MLA_ERR_CUDA;
-  auto kern = mla::down_proj_append_kernel<SPLIT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmemBytes) != cudaSuccess)
+  auto split = mla::dp_split_kernel<NT>;
+  if (cudaFuncSetAttribute(split, cudaFuncAttributeMaxDynamicSharedMemorySize, Sh::kSmemBytes) != cudaSuccess)
     return MLA_ERR_CUDA;
-  const dim3 grid(SPLIT, mla::kDpMTiles, (n_tokens + mla::kDpNt - 1) / mla::kDpNt);
-  return launch_chained_cluster(kern, grid, dim3(mla::kDpThreads), static_cast<size_t>(Sh::kSmemBytes),
-                                as_stream(stream), SPLIT, tw, tk, th, seq_ids, pos,
-                                reinterpret_cast<__nv_bfloat16*>(cache), v, n_tokens, rope_freq(rope_base));
+  const int G = std::max(mla::kDpMTiles, std::min(mla::kDpMaxCtas, device_sm_count()));
+  cudaStream_t s = as_stream(stream);
+  const mla::RopeFreq rope = rope_freq(rope_base);
+  for (int n0 = 0; n0 < n_tokens; n0 += NT) {
+    mla_status st = launch_chained(split, dim3(G), dim3(mla::kDpThreads), static_cast<size_t>(Sh::kSmemBytes), s, tw,
+                                   tk, th, n0);
+    if (st != MLA_OK) return st;
+    st = launch_chained(mla::dp_sum_kernel<NT>, dim3(mla::kDpMTiles, NT), dim3(128), 0, s, seq_ids, pos,
+                        reinterpret_cast<__nv_bfloat16*>(cache), v, n_tokens, rope, n0, G);
+    if (st != MLA_OK) return st;
+  }
+  return MLA_OK;
 }
 
 }  // namespace
@@ -348,11 +303,9 @@ mla_status mla_project_append(const mla_bf16* h, const mla_bf16* w_dkv, const ml
   if (!aligned16(h) || !aligned16(w_dkv) || !aligned16(w_kr)) return MLA_ERR_INVALID_ARG;
   if (seq_ids == nullptr && n_tokens > desc.num_seqs) return MLA_ERR_INVALID_ARG;
   if (n_tokens > kMaxBatch) return MLA_ERR_UNSUPPORTED;
-  // K split over 16-CTA clusters where the device places them, else over 8-CTA clusters.
-  static const int split = cluster16_ok(mla::down_proj_append_kernel<16>, mla::kDpThreads,
-                                        mla::DpShape<16>::kSmemBytes) ? 16 : 8;
-  return split == 16 ? launch_project_append<16>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream)
-                     : launch_project_append<8>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream);
+  // Tiles of 32 tokens up to 32, else of 128 (the weights then stream once per 128 tokens).
+  if (n_tokens <= 32) return launch_project_append<32>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream);
+  return launch_project_append<128>(h, w_dkv, w_kr, seq_ids, pos, cache, v, n_tokens, rope_base, stream);
 }
 
 mla_status mla_selftest_wait_timeout(uint32_t limit_us, int32_t* result, void* stream) {
